@@ -1,0 +1,350 @@
+// api.cu -- the C ABI of include/entmax_attn.h: argument checks, workspace layout and caching,
+// and the launch sequence of the two passes.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "entmax_attn.h"
+#include "kernels.h"
+
+// Per-device status word: kernels set ENTMAX_ATTN_ETIMEOUT here when a bounded wait gives up.
+__device__ int g_entmax_status;
+
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+
+int cuda_fail(cudaError_t e) {
+  std::snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return ENTMAX_ATTN_ECUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+  int slots;      // query tiles (slots) per head
+  int W;          // mask words per query tile
+  int nkt_max;    // longest compact list
+  int64_t tiles;  // query tiles over all (batch, head)
+};
+
+bool make_layout(int B, int Hq, int T, int has_cu, Layout* L) {
+  if (B < 1 || Hq < 1 || T < 1) return false;
+  const int64_t nt = (static_cast<int64_t>(T) + ea::kTile - 1) / ea::kTile;
+  const int64_t slots = has_cu ? static_cast<int64_t>(T) / ea::kTile + B : nt;
+  if (slots > (1 << 24)) return false;
+  L->slots = static_cast<int>(slots);
+  L->W = static_cast<int>((nt + 31) / 32);
+  L->nkt_max = static_cast<int>(nt);
+  L->tiles = (has_cu ? 1 : static_cast<int64_t>(B)) * Hq * slots;
+  return L->tiles < (int64_t(1) << 31);
+}
+
+// Workspace: [queue_count | count[tiles] | queue[tiles] | list[tiles][nkt_max]], each section
+// 256-byte aligned.
+struct WsView {
+  int* queue_count;
+  int* count;
+  int* queue;
+  int* list;
+  size_t bytes;
+};
+
+WsView ws_view(void* base, const Layout& L) {
+  WsView v;
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  v.queue_count = reinterpret_cast<int*>(p + off);
+  off += 256;
+  v.count = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * L.tiles);
+  v.queue = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * L.tiles);
+  v.list = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * static_cast<size_t>(L.tiles) * L.nkt_max);
+  v.bytes = off;
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+std::mutex g_mu;
+
+int* status_ptr(int* err) {
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    *err = cuda_fail(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_entmax_status);
+    if (e != cudaSuccess) {
+      *err = cuda_fail(e);
+      return nullptr;
+    }
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int num_sms() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
+      v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
+
+// Shared checks of both passes; fills the problem description (without workspace pointers).
+int check_and_describe(const void* q, const void* k, int B, int Hq, int Hkv, int T, int d,
+                       float alpha, int n_iter, int causal, const int32_t* cu, int dtype,
+                       Layout* L, ea::Problem* P) {
+  if (!q || !k) return ENTMAX_ATTN_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0) return ENTMAX_ATTN_EINVAL;
+  if (d != 64 && d != 128) return ENTMAX_ATTN_EINVAL;
+  if (!std::isfinite(alpha) || !(alpha > 1.f)) return ENTMAX_ATTN_EINVAL;
+  if (n_iter < 1 || n_iter > 1000) return ENTMAX_ATTN_EINVAL;
+  if (dtype != ENTMAX_ATTN_FP32 && dtype != ENTMAX_ATTN_BF16) return ENTMAX_ATTN_EINVAL;
+  if (causal != 0 && causal != 1) return ENTMAX_ATTN_EINVAL;
+  if (!make_layout(B, Hq, T, cu != nullptr, L)) return ENTMAX_ATTN_EINVAL;
+  if (L->W > ea::kMaxWords) return ENTMAX_ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || (cu && !aligned16(cu))) return ENTMAX_ATTN_EALIGN;
+  const double a = static_cast<double>(alpha);
+  const float beta = static_cast<float>(1.0 / (a - 1.0));
+  if (!std::isfinite(beta)) return ENTMAX_ATTN_EINVAL;
+  std::memset(P, 0, sizeof(*P));
+  P->q = q;
+  P->k = k;
+  P->cu = cu;
+  P->B = B;
+  P->Hq = Hq;
+  P->Hkv = Hkv;
+  P->T = T;
+  P->d = d;
+  P->G = Hq / Hkv;
+  P->causal = causal;
+  P->n_iter = n_iter;
+  P->alpha = alpha;
+  P->beta = beta;
+  P->c = static_cast<float>((a - 1.0) / std::sqrt(static_cast<double>(d)));
+  P->slots = L->slots;
+  P->W = L->W;
+  P->nkt_max = L->nkt_max;
+  return ENTMAX_ATTN_OK;
+}
+
+void attach_workspace(ea::Problem* P, const WsView& v) {
+  P->list = v.list;
+  P->count = v.count;
+  P->queue = v.queue;
+  P->queue_count = v.queue_count;
+}
+
+bool use_tensor_cores(int dtype, unsigned flags) {
+  return dtype == ENTMAX_ATTN_BF16 && !(flags & ENTMAX_ATTN_FLAG_CUDA_CORES);
+}
+
+struct CachedWs {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, cudaStream_t>, CachedWs> g_ws;
+
+}  // namespace
+
+extern "C" {
+
+size_t entmax_attn_mask_words(int B, int Hq, int T, int has_cu_seqlens) {
+  Layout L;
+  if (!make_layout(B, Hq, T, has_cu_seqlens != 0, &L)) return 0;
+  return static_cast<size_t>(L.tiles) * L.W;
+}
+
+int entmax_attn_mask_layout(int B, int Hq, int T, int has_cu_seqlens, int* tiles_per_head,
+                            int* words_per_tile) {
+  Layout L;
+  if (!make_layout(B, Hq, T, has_cu_seqlens != 0, &L)) return ENTMAX_ATTN_EINVAL;
+  if (tiles_per_head) *tiles_per_head = L.slots;
+  if (words_per_tile) *words_per_tile = L.W;
+  return ENTMAX_ATTN_OK;
+}
+
+size_t entmax_attn_workspace_bytes(int B, int Hq, int T, int has_cu_seqlens) {
+  Layout L;
+  if (!make_layout(B, Hq, T, has_cu_seqlens != 0, &L)) return 0;
+  return ws_view(nullptr, L).bytes;
+}
+
+int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
+                         void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
+                         int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
+                         int dtype, unsigned flags, cudaStream_t stream) {
+  Layout L;
+  ea::Problem P;
+  int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
+                              &L, &P);
+  if (rc != ENTMAX_ATTN_OK) return rc;
+  if (!tau || !block_mask || !workspace) return ENTMAX_ATTN_EINVAL;
+  if (!aligned16(tau) || !aligned16(block_mask) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ENTMAX_ATTN_EALIGN;
+  const WsView v = ws_view(workspace, L);
+  if (workspace_bytes < v.bytes) return ENTMAX_ATTN_ENOMEM;
+  int err = ENTMAX_ATTN_OK;
+  P.status = status_ptr(&err);
+  if (!P.status) return err;
+  P.tau = tau;
+  P.mask = block_mask;
+  attach_workspace(&P, v);
+  P.force_fallback = (flags & ENTMAX_ATTN_FLAG_ALL_FALLBACK) ? 1 : 0;
+
+  cudaError_t e = cudaMemsetAsync(v.queue_count, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = use_tensor_cores(dtype, flags) ? ea::launch_tau_tc(P, stream)
+                                     : ea::launch_tau_simt(P, dtype, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int64_t ctas = std::min<int64_t>(L.tiles, 2 * num_sms());
+  e = ea::launch_tau_fallback(P, dtype, static_cast<int>(ctas), stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ENTMAX_ATTN_OK;
+}
+
+int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,
+                         const void* workspace, size_t workspace_bytes, void* out, int B, int Hq,
+                         int Hkv, int T, int d, float alpha, int causal,
+                         const int32_t* cu_seqlens, int dtype, unsigned flags,
+                         cudaStream_t stream) {
+  Layout L;
+  ea::Problem P;
+  int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, 1, causal, cu_seqlens, dtype, &L,
+                              &P);
+  if (rc != ENTMAX_ATTN_OK) return rc;
+  if (!v || !tau || !out || !workspace) return ENTMAX_ATTN_EINVAL;
+  if (!aligned16(v) || !aligned16(tau) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ENTMAX_ATTN_EALIGN;
+  const WsView wv = ws_view(const_cast<void*>(workspace), L);
+  if (workspace_bytes < wv.bytes) return ENTMAX_ATTN_ENOMEM;
+  int err = ENTMAX_ATTN_OK;
+  P.status = status_ptr(&err);
+  if (!P.status) return err;
+  P.v = v;
+  P.out = out;
+  P.tau = const_cast<float*>(tau);
+  attach_workspace(&P, wv);
+  cudaError_t e = use_tensor_cores(dtype, flags) ? ea::launch_out_tc(P, stream)
+                                                 : ea::launch_out_simt(P, dtype, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ENTMAX_ATTN_OK;
+}
+
+int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
+                    uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
+                    int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                    cudaStream_t stream) {
+  Layout L;
+  ea::Problem P;
+  int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
+                              &L, &P);
+  if (rc != ENTMAX_ATTN_OK) return rc;
+  if (!v || !out || !tau || !block_mask) return ENTMAX_ATTN_EINVAL;
+  const size_t need = ws_view(nullptr, L).bytes;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    CachedWs& c = g_ws[{dev, stream}];
+    if (c.bytes < need) {
+      if (c.ptr) {
+        e = cudaFreeAsync(c.ptr, stream);
+        c.ptr = nullptr;
+        c.bytes = 0;
+        if (e != cudaSuccess) return cuda_fail(e);
+      }
+      e = cudaMallocAsync(&c.ptr, need, stream);
+      if (e != cudaSuccess) {
+        c.ptr = nullptr;
+        return ENTMAX_ATTN_ENOMEM;
+      }
+      c.bytes = need;
+    }
+    ws = c.ptr;
+  }
+  rc = entmax_attn_tau_pass(q, k, tau, block_mask, ws, need, B, Hq, Hkv, T, d, alpha, n_iter,
+                            causal, cu_seqlens, dtype, 0u, stream);
+  if (rc != ENTMAX_ATTN_OK) return rc;
+  return entmax_attn_out_pass(q, k, v, tau, ws, need, out, B, Hq, Hkv, T, d, alpha, causal,
+                              cu_seqlens, dtype, 0u, stream);
+}
+
+int entmax_attn_fallback_tiles(const void* workspace, cudaStream_t stream) {
+  if (!workspace) return -1;
+  int n = 0;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemcpy(&n, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    cuda_fail(e);
+    return -1;
+  }
+  return n;
+}
+
+int entmax_attn_status(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_entmax_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_entmax_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return v;
+}
+
+void entmax_attn_release_workspaces(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_ws) {
+    if (!kv.second.ptr) continue;
+    cudaSetDevice(kv.first.first);
+    cudaDeviceSynchronize();
+    cudaFree(kv.second.ptr);
+  }
+  g_ws.clear();
+  cudaSetDevice(cur);
+}
+
+const char* entmax_attn_strerror(int code) {
+  switch (code) {
+    case ENTMAX_ATTN_OK: return "ok";
+    case ENTMAX_ATTN_EINVAL: return "invalid argument";
+    case ENTMAX_ATTN_EALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case ENTMAX_ATTN_ECUDA: return "CUDA runtime error";
+    case ENTMAX_ATTN_ETIMEOUT: return "device-side bounded wait timed out";
+    case ENTMAX_ATTN_ENOMEM: return "workspace too small or allocation failed";
+    default: return "unknown error code";
+  }
+}
+
+const char* entmax_attn_last_cuda_error(void) { return g_cuda_err; }
+
+}  // extern "C"

@@ -1,0 +1,365 @@
+// common.cuh -- problem description, query-tile map, and the per-row candidate buffer + tau
+// solve shared by the tau-pass kernels of the entmax attention library.
+//
+// Notation (AdaSplash: Adaptive Sparse Flash Attention, "AdaSplash with Block Masking"):
+//   raw score   r_ij = q_i . k_j                      (fp32 accumulate)
+//   z_ij        = c * r_ij,  c = (alpha - 1) / sqrt(d)
+//   p_ij        = [z_ij - tau_i]_+ ^ beta,  beta = 1 / (alpha - 1)
+// Because p_ij <= 1, tau_i >= m_i - 1 with m_i = max_j z_ij, so only keys with z > m - 1 can
+// carry p > 0.  The tau pass keeps exactly those keys ("candidates") per row while it sweeps
+// the key tiles, then runs the bracketed Halley + bisection search of the "Triton Entmax
+// (Optimized Entmax Activation)" section over the candidates alone.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ea {
+
+constexpr int kTile = 128;      // query-tile rows and key-tile keys (block-mask granularity)
+constexpr int kCand = 64;       // candidate slots per row held in shared memory
+constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
+
+enum BetaKind { kBetaOne = 0, kBetaTwo = 1, kBetaGeneral = 2 };
+
+// Everything a kernel needs; passed by value.
+struct Problem {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* tau;
+  uint32_t* mask;
+  const int32_t* cu;   // nullptr = fixed length
+  int B, Hq, Hkv, T, d, G;
+  int causal;
+  int n_iter;
+  float alpha;
+  float beta;          // 1 / (alpha - 1)
+  float c;             // (alpha - 1) / sqrt(d)
+  int slots;           // query tiles (slots) per head
+  int W;               // mask words per query tile
+  int nkt_max;         // stride of a compact list
+  // workspace
+  int* list;           // [tiles][nkt_max]
+  int* count;          // [tiles]
+  int* queue;          // [tiles] overflow queue
+  int* queue_count;    // 1 int
+  int* status;         // per-device status word
+  int force_fallback;  // every tile takes the overflow path
+};
+
+struct TileInfo {
+  int valid;        // 0 = unused slot of a packed batch
+  int h;            // q head
+  int qt;           // query tile index inside its sequence
+  int seq_start;    // first packed token of the sequence (0 for fixed length)
+  int seq_len;
+  int row0;         // position (inside the sequence) of the tile's first row
+  int nrows;        // rows of this tile (<= 128)
+  int nkt;          // key tiles the tile visits: qt + 1 causal, all of the sequence otherwise
+  int64_t qhead;    // row offset of this (batch, q head) in q / out / tau
+  int64_t khead;    // row offset of this (batch, kv head) in k / v
+  int64_t tile_id;  // (batch * Hq + h) * slots + slot
+};
+
+// Maps a (slot, head, batch) grid coordinate to its query tile.  For a packed batch, sequence s
+// owns slots floor(cu[s] / 128) + s + [0, ceil(len_s / 128)); the base is nondecreasing in s,
+// so the sequence of a slot is found by binary search (batch must be 0 then).
+__device__ __forceinline__ TileInfo map_tile(const Problem& P, int slot, int h, int b) {
+  TileInfo t;
+  t.h = h;
+  if (P.cu == nullptr) {
+    t.seq_start = 0;
+    t.seq_len = P.T;
+    t.qt = slot;
+    t.qhead = ((int64_t)b * P.Hq + h) * P.T;
+    t.khead = ((int64_t)b * P.Hkv + h / P.G) * P.T;
+  } else {
+    int lo = 0, hi = P.B - 1;
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (P.cu[mid] / kTile + mid <= slot) lo = mid;
+      else hi = mid - 1;
+    }
+    t.seq_start = P.cu[lo];
+    t.seq_len = P.cu[lo + 1] - P.cu[lo];
+    t.qt = slot - (P.cu[lo] / kTile + lo);
+    t.qhead = (int64_t)h * P.T;
+    t.khead = (int64_t)(h / P.G) * P.T;
+  }
+  const int nqt = (t.seq_len + kTile - 1) / kTile;
+  t.valid = (t.qt >= 0 && t.qt < nqt);
+  t.row0 = t.qt * kTile;
+  t.nrows = t.valid ? min(kTile, t.seq_len - t.row0) : 0;
+  t.nkt = P.causal ? t.qt + 1 : nqt;
+  t.tile_id = ((int64_t)b * P.Hq + h) * P.slots + slot;
+  return t;
+}
+
+__device__ __forceinline__ float load_elem(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float* p, int64_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, int64_t i, float x) {
+  p[i] = __float2bfloat16_rn(x);
+}
+
+// x^beta and the two lower powers needed by the Halley step, for x > 0.
+template <int BK>
+__device__ __forceinline__ void entmax_powers(float x, float beta, float& p0, float& p1,
+                                              float& p2) {
+  if (BK == kBetaOne) {
+    p0 = x; p1 = 1.f; p2 = 0.f;
+  } else if (BK == kBetaTwo) {
+    p0 = x * x; p1 = x; p2 = 1.f;
+  } else {
+    p0 = exp2f(beta * __log2f(x));
+    const float inv = __frcp_rn(x);
+    p1 = p0 * inv;
+    p2 = p1 * inv;
+  }
+}
+
+// p = [x]_+^beta
+template <int BK>
+__device__ __forceinline__ float entmax_p(float x, float beta) {
+  if (!(x > 0.f)) return 0.f;
+  if (BK == kBetaOne) return x;
+  if (BK == kBetaTwo) return x * x;
+  return exp2f(beta * __log2f(x));
+}
+
+// One step of the bracketed Halley + bisection search, given the sums over the keys with
+// z > tau of (z - tau)^beta, ^(beta-1), ^(beta-2).  f = S0 - 1, f' = -beta S1,
+// f'' = beta (beta - 1) S2.  The bracket [lo, hi] is narrowed by the sign of f.  The Halley
+// step is taken when its denominator 2 f'^2 - f f'' is positive and finite (then it moves
+// toward the root), otherwise the Newton step; a step outside the closed bracket becomes the
+// bracket midpoint.
+template <int BK>
+__device__ __forceinline__ float halley_step(float tau, float s0, float s1, float s2, float beta,
+                                             float& lo, float& hi) {
+  const float f = s0 - 1.f;
+  const float f1 = -beta * s1;
+  const float f2 = (BK == kBetaOne) ? 0.f : beta * (beta - 1.f) * s2;
+  if (f > 0.f) lo = tau;
+  else hi = tau;
+  const float den = 2.f * f1 * f1 - f * f2;
+  float nt;
+  if (den > 0.f && den < INFINITY) nt = tau - 2.f * f * f1 / den;
+  else nt = tau - f / f1;
+  if (!(nt >= lo && nt <= hi)) nt = 0.5f * (lo + hi);
+  return nt;
+}
+
+// Initial bracket of the search: p_max <= 1 gives tau >= m - 1; n keys all at most m give
+// tau <= m - n^(1 - alpha).
+__device__ __forceinline__ void initial_bracket(float m, int n, float alpha, float& lo,
+                                                float& hi) {
+  lo = m - 1.f;
+  hi = m - exp2f((1.f - alpha) * __log2f((float)n));
+}
+
+// ---------------------------------------------------------------------------------------------
+// Candidate buffer: per row (thread r of the 128 owning rows) up to kCand (raw score, key tile)
+// pairs in shared memory, entry e of row r at [e * 128 + r] so that a warp's rows hit distinct
+// banks whatever their fill levels.
+// ---------------------------------------------------------------------------------------------
+struct CandSmem {
+  float s[kCand * kTile];
+  uint16_t kt[kCand * kTile];
+  float m[kTile];       // row max of raw scores
+  float floor_[kTile];  // pruning floor (raw); -inf when the row was never pruned
+  int cnt[kTile];
+  int lost[kTile];
+  uint32_t words[kMaxWords];
+  int fallback;         // some row of the tile needs the overflow path
+};
+
+struct RowCand {
+  float m;       // running max of raw scores
+  float thr;     // keep threshold: max(m - 1/c, floor)
+  float floor_;  // pruning floor, -inf if never raised
+  float inv_c;   // 1 / c
+  int cnt;
+  int lost;
+
+  __device__ __forceinline__ void init(float inv_c_) {
+    m = -INFINITY;
+    thr = -INFINITY;
+    floor_ = -INFINITY;
+    inv_c = inv_c_;
+    cnt = 0;
+    lost = 0;
+  }
+
+  // Drops entries at or below the threshold; while more than half the slots stay in use, raises
+  // the floor halfway to the running max (entries below the floor can only matter if tau ends
+  // up at or below it, which the solve checks).
+  __device__ __noinline__ void compact(CandSmem& cs, int r) {
+    int n = 0;
+    for (int e = 0; e < cnt; ++e) {
+      const float x = cs.s[e * kTile + r];
+      if (x > thr) {
+        cs.s[n * kTile + r] = x;
+        cs.kt[n * kTile + r] = cs.kt[e * kTile + r];
+        ++n;
+      }
+    }
+    cnt = n;
+    for (int guard = 0; cnt > kCand / 2 && guard < 8; ++guard) {
+      floor_ = thr + 0.5f * (m - thr);
+      thr = floor_;
+      n = 0;
+      for (int e = 0; e < cnt; ++e) {
+        const float x = cs.s[e * kTile + r];
+        if (x > thr) {
+          cs.s[n * kTile + r] = x;
+          cs.kt[n * kTile + r] = cs.kt[e * kTile + r];
+          ++n;
+        }
+      }
+      cnt = n;
+    }
+  }
+
+  __device__ __forceinline__ void push(CandSmem& cs, int r, float x, int kt) {
+    if (lost) return;
+    if (cnt == kCand) {
+      compact(cs, r);
+      if (cnt == kCand) {
+        lost = 1;
+        return;
+      }
+    }
+    cs.s[cnt * kTile + r] = x;
+    cs.kt[cnt * kTile + r] = (uint16_t)kt;
+    ++cnt;
+  }
+
+  // Feeds N raw scores of key tile kt (invalid keys already -inf).
+  template <int N>
+  __device__ __forceinline__ void feed(CandSmem& cs, int r, const float (&x)[N], int kt) {
+    float cmax = x[0];
+#pragma unroll
+    for (int i = 1; i < N; ++i) cmax = fmaxf(cmax, x[i]);
+    if (cmax > thr) {
+      if (cmax > m) {
+        m = cmax;
+        thr = fmaxf(m - inv_c, floor_);
+      }
+#pragma unroll
+      for (int i = 0; i < N; ++i)
+        if (x[i] > thr) push(cs, r, x[i], kt);
+    }
+  }
+
+  __device__ __forceinline__ void publish(CandSmem& cs, int r) const {
+    cs.m[r] = m;
+    cs.floor_[r] = floor_;
+    cs.cnt[r] = cnt;
+    cs.lost[r] = lost;
+  }
+};
+
+// Solves tau for every row of the tile from the published candidate buffers, writes tau and
+// sets the tile's mask words in shared memory.  Rows are handled by groups of 4 lanes that
+// split a row's candidates and combine their partial sums with warp shuffles.  nthreads must be
+// a multiple of 32; call from all threads of the block after a __syncthreads() that follows
+// publish().
+template <int BK>
+__device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, int tid,
+                           int nthreads) {
+  const int lane4 = tid & 3;
+  const int groups = nthreads >> 2;
+  // Every lane runs the same number of row iterations and search steps (the shuffles need the
+  // whole warp); rows past the end of the tile run on an empty candidate list and store nothing.
+  for (int r = tid >> 2; r < kTile; r += groups) {
+    const bool valid = r < t.nrows;
+    const int cnt = valid ? cs.cnt[r] : 0;
+    const float mz = valid ? P.c * cs.m[r] : 0.f;
+    const int pos = t.row0 + r;
+    const int n = valid ? (P.causal ? pos + 1 : t.seq_len) : 1;
+    float lo, hi;
+    initial_bracket(mz, n, P.alpha, lo, hi);
+    float tau = lo;
+    for (int it = 0; it < P.n_iter; ++it) {
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+      for (int e = lane4; e < cnt; e += 4) {
+        const float x = P.c * cs.s[e * kTile + r] - tau;
+        if (x > 0.f) {
+          float a, b, c2;
+          entmax_powers<BK>(x, P.beta, a, b, c2);
+          s0 += a;
+          s1 += b;
+          s2 += c2;
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      }
+      tau = halley_step<BK>(tau, s0, s1, s2, P.beta, lo, hi);
+    }
+    if (!valid) continue;
+    if (lane4 == 0) P.tau[t.qhead + t.seq_start + pos] = tau;
+    const bool floored = cs.floor_[r] > -INFINITY;
+    if (cs.lost[r] || (floored && !(tau > P.c * cs.floor_[r]))) cs.fallback = 1;
+    for (int e = lane4; e < cnt; e += 4) {
+      if (P.c * cs.s[e * kTile + r] > tau) {
+        const int kt = cs.kt[e * kTile + r];
+        atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
+      }
+    }
+  }
+}
+
+// Writes the tile's mask words and its compact list of active key tiles (ascending) and count,
+// or queues the tile for the overflow path.  Call from warp 0 after a __syncthreads().
+__device__ __forceinline__ void emit_tile(const Problem& P, const TileInfo& t,
+                                          const uint32_t* words, int fallback, int lane) {
+  if (fallback) {
+    if (lane == 0) {
+      const int i = atomicAdd(P.queue_count, 1);
+      P.queue[i] = (int)t.tile_id;
+    }
+    return;
+  }
+  uint32_t* mw = P.mask + t.tile_id * P.W;
+  int* list = P.list + t.tile_id * P.nkt_max;
+  int base = 0;
+  for (int w0 = 0; w0 < P.W; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t bits = (w < P.W) ? words[w] : 0u;
+    if (w < P.W) mw[w] = bits;
+    const int c = __popc(bits);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int at = base + incl - c;
+    uint32_t b = bits;
+    while (b) {
+      const int bit = __ffs(b) - 1;
+      b &= b - 1;
+      list[at++] = w * 32 + bit;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) P.count[t.tile_id] = base;
+}
+
+// Unused slot of a packed batch: zero mask words, empty list.
+__device__ __forceinline__ void emit_empty(const Problem& P, const TileInfo& t, int tid,
+                                           int nthreads) {
+  for (int w = tid; w < P.W; w += nthreads) P.mask[t.tile_id * P.W + w] = 0u;
+  if (tid == 0) P.count[t.tile_id] = 0;
+}
+
+}  // namespace ea

@@ -1,0 +1,23 @@
+// kernels.h -- host-side launchers of the entmax attention kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ea {
+
+// dtype: 0 = fp32, 1 = bf16.  Each returns cudaSuccess or the launch error.
+cudaError_t launch_tau_simt(const Problem& P, int dtype, cudaStream_t s);
+cudaError_t launch_tau_fallback(const Problem& P, int dtype, int num_ctas, cudaStream_t s);
+cudaError_t launch_out_simt(const Problem& P, int dtype, cudaStream_t s);
+
+// Tensor-core (tcgen05) kernels, bf16 only, d in {64, 128}.
+cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s);
+cudaError_t launch_out_tc(const Problem& P, cudaStream_t s);
+
+inline int beta_kind(float beta) {
+  return beta == 1.f ? kBetaOne : (beta == 2.f ? kBetaTwo : kBetaGeneral);
+}
+
+}  // namespace ea

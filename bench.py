@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the causal alpha-entmax attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+A step is one full forward pass (tau pass + output pass) over the workload's synthetic batch,
+with the inputs already resident in HBM.  The metric is effective TFLOP/s: 4 d FLOPs per
+causally valid (query, key) pair inside the active 128 x 128 tiles (recomputed scores + p V),
+summed over heads and batch, divided by the step time; tokens/s and the fraction of the
+measured bf16 dense tensor-core peak ride along.  Rank 0 prints one JSON line.
+
+Multi-GPU (torchrun): every (batch, kv-head group) is independent, so each rank runs its own
+full-size problem (weak scaling, no collective on the data path); the step time is the max over
+ranks.  --impl reference times the fp64 CPU oracle instead, on a bounded sample of whole query
+tiles of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from adaptive_sparse_attention_b200 import api as ea  # noqa: E402
+from adaptive_sparse_attention_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "b2_t16k_gqa4_bf16_d128_a2"
+METRIC = "effective TFLOP/s and tokens/s of entmax attention fwd; % of bf16 TC peak"
+TILE = 128
+L2_BYTES = 126 * 2**20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------ work counts --
+
+def pair_matrix(L: int, causal: bool) -> np.ndarray:
+    """[nqt, nkt] number of valid (query, key) pairs of each tile of one sequence of length L."""
+    nt = (L + TILE - 1) // TILE
+    rows = np.minimum(TILE, L - np.arange(nt) * TILE)
+    if not causal:
+        return np.outer(rows, rows).astype(np.int64)
+    m = np.zeros((nt, nt), dtype=np.int64)
+    for qt in range(nt):
+        m[qt, :qt] = rows[qt] * rows[:qt]
+        r = rows[qt]
+        m[qt, qt] = r * (r + 1) // 2  # diagonal tile: keys <= own position
+    return m
+
+
+def count_pairs(w, bits, cu):
+    """(pairs inside active tiles, all valid pairs) summed over batch and heads."""
+    table = ea.tile_slot_table(w.B, w.T, None if cu is None else cu.tolist())
+    act = dense = 0
+    nb = 1 if cu is not None else w.B
+    for b in range(nb):
+        seqs = range(len(table)) if cu is not None else [b]
+        for s in seqs:
+            slot0, nqt, start, L = table[s]
+            if nqt == 0:
+                continue
+            pm = pair_matrix(L, w.causal)
+            blk = bits[b, :, slot0:slot0 + nqt, :pm.shape[1]]  # [Hq, nqt, nkt]
+            act += int((blk * pm[None]).sum())
+            dense += int(pm.sum()) * w.Hq
+    return act, dense
+
+
+# --------------------------------------------------------------------------------- helpers --
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [x for x in sm if x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------- oracle sampling --
+
+def oracle_tile_sample(w, inputs, budget_s: float, seed: int = 0):
+    """Times the oracle on whole query tiles of the workload until about budget_s seconds of
+    CPU work; returns (effective flops, rows, seconds, n tiles, threads)."""
+    from oracle import oracle
+    q, k, v, cu = inputs
+    alpha = oracle.alpha_as_float32(w.alpha)
+    table = ea.tile_slot_table(w.B, w.T, None if cu is None else cu.tolist())
+    rng = np.random.default_rng(seed)
+    nb = 1 if cu is not None else w.B
+    # candidate tiles: (b, h, s, qt) drawn uniformly over all query tiles
+    all_t = [(b, h, s, qt) for b in range(nb) for h in range(w.Hq)
+             for s in (range(len(table)) if cu is not None else [b]) for qt in range(table[s][1])]
+    order = rng.permutation(len(all_t))
+    flops = rows_done = 0
+    spent = 0.0
+    ntiles = 0
+    batch = 1
+    threads = oracle.host_threads()
+    for i0 in range(0, len(order)):
+        if spent >= budget_s or ntiles >= len(order):
+            break
+        pick = [all_t[j] for j in order[ntiles:ntiles + batch]]
+        rows, meta = [], []
+        for b, h, s, qt in pick:
+            slot0, nqt, start, L = table[s]
+            pos = np.arange(qt * TILE, min((qt + 1) * TILE, L))
+            r = ((b * w.Hq + h) * w.T + pos) if cu is None else (h * w.T + start + pos)
+            rows.append(r)
+            meta.append((L, qt, pos.size))
+        rr = np.concatenate(rows)
+        t0 = time.perf_counter()
+        res = oracle.attention_rows(q, k, v, alpha, w.causal, cu, rr, nthreads=threads)
+        dt = time.perf_counter() - t0
+        spent += dt
+        off = 0
+        for (L, qt, n) in meta:
+            active = (res["maxp"][off:off + n] > 0).any(axis=0)
+            pm = pair_matrix(L, w.causal)[qt]
+            flops += 4 * w.d * int((active[:pm.size] * pm).sum())
+            off += n
+        rows_done += rr.size
+        ntiles += len(pick)
+        batch = max(1, min(64, int(batch * 2))) if dt < budget_s / 8 else batch
+    return flops, rows_done, spent, ntiles, threads
+
+
+# -------------------------------------------------------------------------------- arms --
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inputs = make_inputs(w, seed=0)
+    per_step = max(1.0, min(20.0, 150.0 / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_tile_sample(w, inputs, per_step, seed=1)
+    vals, times, rows, tiles = [], [], 0, 0
+    threads = 0
+    for i in range(args.steps):
+        fl, nr, dt, nt, threads = oracle_tile_sample(w, inputs, per_step, seed=100 + i)
+        vals.append(fl / dt / 1e12)
+        times.append(dt)
+        rows += nr
+        tiles += nt
+    value = float(np.mean(vals))
+    sample = (f"{tiles} whole 128-row query tiles drawn uniformly over (batch, head, tile) "
+              f"({rows} rows) across {args.steps} steps of ~{per_step:.0f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "T": w.T, "d": w.d,
+            "alpha": w.alpha, "n_iter": w.n_iter, "causal": w.causal, "input_dtype": w.dtype,
+            "seqlens": list(w.seqlens) if w.seqlens else None,
+            "spikes": f"{w.spike_frac:g} of keys x{w.spike_scale:g}" if w.spike_frac else None,
+            "tile": "128x128", "parallelism": f"dp{world} (independent per-rank problems)"}
+
+
+def run_native(args, rank, world, local):
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    q, k, v, cu = make_inputs(w, seed=rank)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    cud = cu.to(dev) if cu is not None else None
+    from oracle.oracle import alpha_as_float32  # the fp32 rounding of alpha, no oracle work
+    alpha = alpha_as_float32(w.alpha)
+    stream = torch.cuda.current_stream(dev)
+    out, tau, mask = ea.alloc_outputs(qd, kd, cud)
+    ws = ea.alloc_workspace(qd, kd, cud)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ea.status(stream) == 0
+    nfb = ea.fallback_tiles(ws, stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(stop)
+    t_tau = [e[0].elapsed_time(e[1]) for e in evs]
+    t_out = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+    st = ea.status(stream)
+    assert st == 0, f"device status {st}"
+
+    bits = ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, cu)
+    act_pairs, dense_pairs = count_pairs(w, bits, cu)
+    eff_flops = 4 * w.d * act_pairs
+    tau_flops = 2 * w.d * dense_pairs
+    out_flops = 4 * w.d * act_pairs
+    tokens = w.B * w.T * w.Hq if cu is None else w.T * w.Hq  # query rows (token x head)
+    tokens_seq = w.B * w.T if cu is None else w.T
+    value = world * eff_flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the C ABI entry point: H2D of q, k, v from pinned host memory, the
+    # forward pass, D2H of out, every step
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+    for _ in range(1):
+        qd.copy_(qh, non_blocking=True)
+        ea.entmax_attn_fwd(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau, mask,
+                           stream=stream)
+        outh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        ea.entmax_attn_fwd(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau, mask,
+                           stream=stream)
+        outh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    assert ea.status(stream) == 0
+
+    if rank != 0:
+        return 0
+    peaks, peak_src = load_peaks()
+    tc = w.dtype == "bf16"
+    mean_tau = float(np.mean(t_tau))
+    mean_out = float(np.mean(t_out))
+    dom_tau = mean_tau >= mean_out
+    timed_s = total_ms * 1e-3
+    sustained = timed_s > 1.0
+    peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    if tc:
+        bound, unit, peak = "tensor", "TFLOP/s", float(peaks[peak_key])
+        peak_note = f"{peak_src} {peak_key}"
+    else:
+        # fp32 on the CUDA cores: 148 SMs x 128 FMA/clk x 2 FLOP x max SM clock
+        bound, unit = "alu", "TFLOP/s"
+        peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock"
+    achieved = (tau_flops / (mean_tau * 1e-3) if dom_tau else out_flops / (mean_out * 1e-3)) / 1e12
+    roofline = {"kernel": "tau_pass" if dom_tau else "out_pass", "bound": bound,
+                "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": None, "peak_source": peak_note,
+                "algorithmic": ("2 d flops per causally valid pair (dense scores)" if dom_tau
+                                else "4 d flops per valid pair inside active tiles")}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        fl, nr, dt, nt, thr = oracle_tile_sample(w, (q, k, v, cu), args.cpu_budget)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"{nt} whole 128-row query tiles ({nr} rows) drawn uniformly, "
+                         f"{dt:.1f} s of fp64 oracle work"}
+
+    bf16_peak = float(peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": dict(workload_config(w, world),
+                       l2=f"inputs {in_bytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB L2; "
+                          f"no flush" if in_bytes > L2_BYTES else "inputs fit in L2; no flush"),
+        "tokens_per_s": world * tokens_seq / (ms_step * 1e-3),
+        "query_rows_per_s": world * tokens / (ms_step * 1e-3),
+        "frac_of_bf16_peak": value / world / bf16_peak,
+        "dense_equiv_tflops": world * 4 * w.d * dense_pairs / (ms_step * 1e-3) / 1e12,
+        "active_tile_pair_fraction": act_pairs / dense_pairs,
+        "ms_tau_pass": mean_tau, "ms_out_pass": mean_out,
+        "tau_pass_hbm_gbs": (q.numel() * q.element_size() + k.numel() * k.element_size()
+                             + tau.numel() * 4 + mask.numel() * 4) / (mean_tau * 1e-3) / 1e9,
+        "overflow_tiles": nfb,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * eff_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": out.numel() * out.element_size()},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline figure")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        return run_reference(args, rank, world)
+    rank, world, local = dist_setup(args)
+    try:
+        return run_native(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,138 @@
+/*
+ * entmax_attn.h -- C ABI of the B200 (sm_100a) forward pass of causal alpha-entmax attention
+ * with adaptive block skipping.
+ *
+ * The operation (AdaSplash: Adaptive Sparse Flash Attention, section "AdaSplash with Block
+ * Masking"; alpha and causality as in its "Adaptive Sparsity Control" and "Causal and
+ * Non-causal Masking" sections; packed batches as in "Variable Length Sequences"; grouped kv
+ * heads as the enable_gqa option of the MiniCPM-4-8B-NSA page's "Usage" section):
+ *
+ *   s_ij = q_i . k_j / sqrt(d)                  k, v of kv head floor(h / (Hq / Hkv))
+ *   p_ij = [(alpha - 1) s_ij - tau_i]_+ ^ (1 / (alpha - 1)),  tau_i such that sum_j p_ij = 1
+ *   o_i  = sum_j p_ij v_j                          (p is used as computed; no renormalisation)
+ *
+ * over the valid keys j of row i: j <= i within the row's own sequence when causal, the whole
+ * sequence otherwise.  tau_i is found by n_iter steps of a bracketed Halley + bisection search
+ * ("Triton Entmax (Optimized Entmax Activation)" section of the same page).  The block mask
+ * holds one bit per (128-row query tile, 128-key key tile): set iff some valid pair of the tile
+ * has p > 0 ("Requires O(Tr x Tc) bits ... binary mask per block").  The output pass visits
+ * only the key tiles whose bit is set.
+ *
+ * Conventions for every entry point below:
+ *   - Pointers named q, k, v, out, tau, block_mask, cu_seqlens, workspace are DEVICE pointers
+ *     on the current CUDA device, owned by the caller, 16-byte aligned.  q, k, v, cu_seqlens
+ *     are only read.
+ *   - Layout, fixed length (cu_seqlens == NULL): q and out [B, Hq, T, d], k and v [B, Hkv, T, d],
+ *     tau [B, Hq, T], all contiguous, row-major.
+ *     Packed variable length (cu_seqlens != NULL): B is the number of sequences and T the total
+ *     token count; q and out [Hq, T, d], k and v [Hkv, T, d], tau [Hq, T]; cu_seqlens int32
+ *     [B + 1] with cu_seqlens[0] = 0, nondecreasing, cu_seqlens[B] = T.  cu_seqlens is read on
+ *     the device only (no host synchronisation).  Attention never crosses sequences.
+ *   - dtype: ENTMAX_ATTN_FP32 (q, k, v, out are float) or ENTMAX_ATTN_BF16 (bfloat16).  Scores
+ *     and p are computed in fp32; BF16 products run on the tensor cores, FP32 ones on the CUDA
+ *     cores in true fp32.
+ *   - d must be 64 or 128; 1 < alpha, finite; n_iter >= 1; B, Hq, Hkv, T >= 1; Hq % Hkv == 0.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).  Errors found on the
+ *     host are returned at once and nothing is launched; errors found on the device (a bounded
+ *     wait that gave up) are latched in a per-device status word read by entmax_attn_status().
+ *     No error is sticky: the next call starts clean.
+ *
+ * Block-mask layout (uint32 words, bit (kt & 31) of word (kt >> 5) stands for key tile kt,
+ * key tiles counted from the start of the row's sequence):
+ *   fixed length: [B, Hq, nQt, W] with nQt = ceil(T / 128) query tiles per head and
+ *                 W = ceil(nQt / 32) words per query tile.
+ *   packed:       [Hq, S, W] with S = floor(T / 128) + B query-tile slots per head and
+ *                 W = ceil(ceil(T / 128) / 32).  Sequence b owns the slots starting at
+ *                 floor(cu_seqlens[b] / 128) + b, one per query tile of the sequence, in order;
+ *                 every other slot is all-zero.
+ *   Every word is written; bits outside a tile's valid key range are zero.
+ */
+#ifndef ENTMAX_ATTN_H_
+#define ENTMAX_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define ENTMAX_ATTN_OK 0
+#define ENTMAX_ATTN_EINVAL 1   /* an argument is out of range or inconsistent */
+#define ENTMAX_ATTN_EALIGN 2   /* a pointer is not 16-byte aligned */
+#define ENTMAX_ATTN_ECUDA 3    /* a CUDA runtime call failed (see entmax_attn_last_cuda_error) */
+#define ENTMAX_ATTN_ETIMEOUT 4 /* a device-side bounded wait gave up (status word) */
+#define ENTMAX_ATTN_ENOMEM 5   /* workspace too small, or the library's allocation failed */
+
+/* dtype codes. */
+#define ENTMAX_ATTN_FP32 0
+#define ENTMAX_ATTN_BF16 1
+
+/* flags of the two-pass entry points (0 = the normal path). */
+#define ENTMAX_ATTN_FLAG_CUDA_CORES 1u    /* run BF16 products on the CUDA cores too */
+#define ENTMAX_ATTN_FLAG_ALL_FALLBACK 2u  /* send every query tile through the multi-sweep tau
+                                             search that handles candidate-buffer overflow */
+
+/* Full forward pass: tau search + block mask, then the output pass over active tiles.
+ * Writes out, tau and every word of block_mask.  Scratch memory (compact tile lists, overflow
+ * queue) is allocated by the library on first use per (device, stream) with cudaMallocAsync on
+ * `stream`, grown when a larger problem arrives, and kept until entmax_attn_release_workspaces().
+ * Returns ENTMAX_ATTN_OK or an error code. */
+int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
+                    uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
+                    int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                    cudaStream_t stream);
+
+/* Number of uint32 words block_mask must hold (layout above); 0 on bad sizes. */
+size_t entmax_attn_mask_words(int B, int Hq, int T, int has_cu_seqlens);
+
+/* Query tiles (or slots) per head and words per query tile of the mask layout above.
+ * Returns ENTMAX_ATTN_OK or ENTMAX_ATTN_EINVAL. */
+int entmax_attn_mask_layout(int B, int Hq, int T, int has_cu_seqlens, int* tiles_per_head,
+                            int* words_per_tile);
+
+/* Two-pass form, for callers that own the scratch memory or time the passes apart.
+ * workspace: device memory of at least entmax_attn_workspace_bytes(...) bytes, 256-byte
+ * aligned, owned by the caller; the tau pass fills it and the output pass reads it, so both
+ * must see the same workspace, sizes and cu_seqlens, in stream order. */
+size_t entmax_attn_workspace_bytes(int B, int Hq, int T, int has_cu_seqlens);
+
+/* Tau pass: writes tau, every word of block_mask, and the compact list of active key tiles of
+ * every query tile into the workspace. */
+int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
+                         void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
+                         int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
+                         int dtype, unsigned flags, cudaStream_t stream);
+
+/* Output pass: o_i = sum over the listed key tiles of p_ij v_j, with p recomputed from tau. */
+int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,
+                         const void* workspace, size_t workspace_bytes, void* out, int B, int Hq,
+                         int Hkv, int T, int d, float alpha, int causal,
+                         const int32_t* cu_seqlens, int dtype, unsigned flags,
+                         cudaStream_t stream);
+
+/* Number of query tiles that the last tau pass on this workspace sent through the multi-sweep
+ * overflow path.  Synchronises `stream`.  Returns -1 on a CUDA error. */
+int entmax_attn_fallback_tiles(const void* workspace, cudaStream_t stream);
+
+/* Synchronises `stream`, returns the device status word of the current device
+ * (ENTMAX_ATTN_OK or ENTMAX_ATTN_ETIMEOUT) and clears it. */
+int entmax_attn_status(cudaStream_t stream);
+
+/* Frees the workspaces entmax_attn_fwd cached (synchronises the device first). */
+void entmax_attn_release_workspaces(void);
+
+/* Static text for a return code. */
+const char* entmax_attn_strerror(int code);
+
+/* Text of the CUDA error behind the last ENTMAX_ATTN_ECUDA of this thread ("" if none). */
+const char* entmax_attn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTMAX_ATTN_H_ */

@@ -153,10 +153,11 @@ int oracle_entmax_vec(const double* z, int n, double alpha, int force_general, d
 /* Exported: the fixed-iteration bracketed Halley + bisection search for tau, in fp64.
  * Start tau = m - 1 with bracket [m - 1, m - n^(1 - alpha)].  Each of the n_iter steps
  * evaluates f = sum [z - tau]_+^beta - 1 and its first two derivatives, narrows the bracket by
- * the sign of f, and takes the Halley step tau - 2 f f' / (2 f'^2 - f f''), or the bracket
- * midpoint when that step is not finite or falls outside the closed bracket [lo, hi].  (With
- * an open bracket, a tau that has converged onto an end of the bracket would be thrown back to
- * the midpoint by the next step.)  Returns the last tau. */
+ * the sign of f, and takes the Halley step tau - 2 f f' / (2 f'^2 - f f'') when its denominator
+ * is positive and finite (the step then points at the root), else the Newton step - f / f'.  A
+ * step that is not finite or falls outside the closed bracket [lo, hi] becomes the bracket
+ * midpoint.  (With an open bracket, a tau that has converged onto an end of the bracket would
+ * be thrown back to the midpoint by the next step.)  Returns the last tau. */
 double oracle_tau_halley(const double* z, int n, double alpha, int n_iter) {
   double beta = 1.0 / (alpha - 1.0);
   double m = -INFINITY;
@@ -180,7 +181,8 @@ double oracle_tau_halley(const double* z, int n, double alpha, int n_iter) {
     double f2 = (beta != 1.0) ? beta * (beta - 1.0) * s2 : 0.0;
     if (f > 0.0) lo = tau;
     else hi = tau;
-    double nt = tau - 2.0 * f * f1 / (2.0 * f1 * f1 - f * f2);
+    double den = 2.0 * f1 * f1 - f * f2;
+    double nt = (den > 0.0 && isfinite(den)) ? tau - 2.0 * f * f1 / den : tau - f / f1;
     if (!isfinite(nt) || !(nt >= lo && nt <= hi)) nt = 0.5 * (lo + hi);
     tau = nt;
   }
@@ -281,6 +283,8 @@ int oracle_entmax_attn_rows(const float* q, const float* k, const float* v, int 
         for (int j = 0; j < n; ++j) {
           const float* kj = kbase + (seq0 + j) * d;
           double dot = 0.0;
+          /* the simd reduction only lets the compiler split the sum into partial sums */
+#pragma omp simd reduction(+ : dot)
           for (int c = 0; c < d; ++c) dot += qd[c] * (double)kj[c];
           double s = dot * scale;
           z[j] = (alpha - 1.0) * s;

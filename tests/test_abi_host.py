@@ -1,0 +1,160 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports every symbol that
+include/*.h declares, and its host-side layout and argument checks behave as documented."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def native():
+    from adaptive_sparse_attention_b200 import build, _native
+    build.build()
+    return _native
+
+
+def declared_functions():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if not f.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"\b(entmax_attn_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(native):
+    lib = native.lib()
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    # and every binding signature names a declared function
+    assert set(native.SIGNATURES) == set(names)
+
+
+def test_strerror(native):
+    lib = native.lib()
+    for code in range(6):
+        assert lib.entmax_attn_strerror(code)
+    assert b"unknown" in lib.entmax_attn_strerror(99)
+
+
+@pytest.mark.parametrize("B,Hq,T,packed", [(1, 2, 256, 0), (2, 32, 16384, 0), (1, 3, 1, 0),
+                                           (4, 32, 32192, 1), (1, 8, 129, 0), (3, 1, 10, 1),
+                                           (1, 32, 131072, 0)])
+def test_mask_layout_matches_documentation(native, B, Hq, T, packed):
+    from adaptive_sparse_attention_b200 import api
+    nt = -(-T // 128)
+    slots = T // 128 + B if packed else nt
+    W = -(-nt // 32)
+    assert api.mask_layout(B, Hq, T, bool(packed)) == (slots, W)
+    assert api.mask_words(B, Hq, T, bool(packed)) == (1 if packed else B) * Hq * slots * W
+    ws = api.workspace_bytes(B, Hq, T, bool(packed))
+    tiles = (1 if packed else B) * Hq * slots
+    assert ws >= 4 * tiles * (2 + nt)
+
+
+def test_packed_slots_never_overlap():
+    """The slot base floor(cu[s] / 128) + s leaves room for every query tile of sequence s."""
+    from adaptive_sparse_attention_b200.api import tile_slot_table
+    rng = np.random.default_rng(0)
+    for _ in range(200):
+        lens = rng.integers(0, 700, size=rng.integers(1, 9))
+        cu = np.concatenate([[0], np.cumsum(lens)])
+        T = int(cu[-1])
+        if T == 0:
+            continue
+        tab = tile_slot_table(len(lens), T, cu)
+        used = set()
+        for slot0, nqt, start, length in tab:
+            for i in range(nqt):
+                assert slot0 + i not in used
+                assert slot0 + i < T // 128 + len(lens)
+                used.add(slot0 + i)
+
+
+def test_decode_block_mask_bit_order():
+    from adaptive_sparse_attention_b200.api import decode_block_mask
+    B, Hq, T = 1, 1, 128 * 40  # 40 key tiles -> 2 words per query tile
+    words = np.zeros((40, 2), dtype=np.uint32)
+    words[3, 0] = 1 | (1 << 31)
+    words[39, 1] = 1 << 7  # key tile 39
+    bits = decode_block_mask(words.view(np.int32), B, Hq, T)
+    assert bits.shape == (1, 1, 40, 40)
+    assert list(np.nonzero(bits[0, 0, 3])[0]) == [0, 31]
+    assert list(np.nonzero(bits[0, 0, 39])[0]) == [39]
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+@pytest.mark.parametrize("case", ["d96", "hq_not_multiple", "alpha1", "alpha_nan", "niter0",
+                                  "dtype", "null_q", "causal2", "too_long"])
+def test_argument_errors_are_reported_before_any_launch(native, case):
+    lib = native.lib()
+    args = dict(B=1, Hq=4, Hkv=2, T=256, d=64, alpha=1.5, n_iter=10, causal=1, dtype=1, q=0x1000)
+    if case == "d96":
+        args["d"] = 96
+    elif case == "hq_not_multiple":
+        args["Hq"] = 3
+    elif case == "alpha1":
+        args["alpha"] = 1.0
+    elif case == "alpha_nan":
+        args["alpha"] = float("nan")
+    elif case == "niter0":
+        args["n_iter"] = 0
+    elif case == "dtype":
+        args["dtype"] = 7
+    elif case == "null_q":
+        args["q"] = 0
+    elif case == "causal2":
+        args["causal"] = 2
+    elif case == "too_long":
+        args["T"] = 128 * 32 * 64 + 1  # more key tiles than the kernels' mask words
+    a = args
+    rc = lib.entmax_attn_tau_pass(_fake(a["q"]) if a["q"] else None, _fake(0x2000),
+                                  _fake(0x3000), _fake(0x4000), _fake(0x10000), 1 << 40,
+                                  a["B"], a["Hq"], a["Hkv"], a["T"], a["d"], a["alpha"],
+                                  a["n_iter"], a["causal"], None, a["dtype"], 0, None)
+    assert rc == native.EINVAL
+    rc = lib.entmax_attn_fwd(_fake(a["q"]) if a["q"] else None, _fake(0x2000), _fake(0x3000),
+                             _fake(0x5000), _fake(0x6000), _fake(0x7000), a["B"], a["Hq"],
+                             a["Hkv"], a["T"], a["d"], a["alpha"], a["n_iter"], a["causal"],
+                             None, a["dtype"], None)
+    assert rc == native.EINVAL
+
+
+def test_misaligned_pointers_are_rejected(native):
+    lib = native.lib()
+    rc = lib.entmax_attn_tau_pass(_fake(0x1008), _fake(0x2000), _fake(0x3000), _fake(0x4000),
+                                  _fake(0x10000), 1 << 40, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
+                                  0, None)
+    assert rc == native.EALIGN
+    rc = lib.entmax_attn_tau_pass(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000),
+                                  _fake(0x10010), 1 << 40, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
+                                  0, None)
+    assert rc == native.EALIGN  # workspace must be 256-byte aligned
+
+
+def test_small_workspace_is_rejected(native):
+    lib = native.lib()
+    need = lib.entmax_attn_workspace_bytes(1, 2, 256, 0)
+    rc = lib.entmax_attn_tau_pass(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000),
+                                  _fake(0x10000), need - 1, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
+                                  0, None)
+    assert rc == native.ENOMEM
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from adaptive_sparse_attention_b200 import _native
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(_native.NativeLibraryError):
+        _native.lib()

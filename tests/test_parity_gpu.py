@@ -1,0 +1,154 @@
+"""GPU parity: the CUDA library through its C ABI against the fp64 oracle, element by element,
+on the same seeded inputs.  See parity.py for the tolerances.
+
+Covered: the five named workloads (whole at the small sizes; at the large sizes, whole query
+tiles sampled two-sided plus loose rows one-sided, through the same entry points bench.py
+times), ragged and tiny sequence lengths, non-causal attention, GQA, packed batches with empty
+and one-token sequences, d = 64 and 128, alpha in {1.333, 1.5, 2, 3}, the CUDA-core path for
+bf16, the multi-sweep overflow path forced on every tile, and inputs that overflow the
+candidate buffers naturally.
+"""
+import numpy as np
+import pytest
+import torch
+
+from adaptive_sparse_attention_b200 import _native
+from adaptive_sparse_attention_b200.workloads import WORKLOADS, make_inputs, random_case
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for -m gpu tests")
+    _native.lib()
+
+
+def _sample_tiles(w, cu, per_head, rng, include_ends=True):
+    tiles = []
+    table = parity.seq_table(w, cu)
+    nb = 1 if cu is not None else w.B
+    for b in range(nb):
+        for h in range(w.Hq):
+            seqs = range(len(table)) if cu is not None else [b]
+            for s in seqs:
+                nqt = table[s][1]
+                if nqt == 0:
+                    continue
+                pick = set(rng.choice(nqt, size=min(per_head, nqt), replace=False).tolist())
+                if include_ends:
+                    pick |= {0, nqt - 1}
+                tiles += [(b, h, s, int(qt)) for qt in sorted(pick)]
+    return tiles
+
+
+@pytest.mark.parametrize("name", ["t256_fp32_d64_a1.5", "t4k_bf16_d64_a1.5"])
+def test_small_workloads_every_row(oracle, name):
+    w = WORKLOADS[name]
+    inputs = make_inputs(w)
+    g = parity.run_gpu(w, inputs)
+    s = parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=name)
+    print(name, s, "fallback tiles", g.fallback_tiles)
+
+
+def test_small_workload_full_forward_entry_point(oracle):
+    w = WORKLOADS["t4k_bf16_d64_a1.5"]
+    inputs = make_inputs(w)
+    g = parity.run_gpu(w, inputs, use_fwd=True)
+    parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label="fwd")
+
+
+def test_16k_gqa_sparsemax_sampled(oracle):
+    w = WORKLOADS["b2_t16k_gqa4_bf16_d128_a2"]
+    inputs = make_inputs(w)
+    g = parity.run_gpu(w, inputs)
+    rng = np.random.default_rng(1000)
+    tiles = _sample_tiles(w, None, 1, rng, include_ends=False)
+    tiles += [(b, h, 0, 127) for b in range(2) for h in (0, 31)]  # longest rows
+    loose = rng.choice(w.B * w.Hq * w.T, size=2048, replace=False)
+    s = parity.compare(w, inputs, g, tiles, loose, label=w.name)
+    print(w.name, s, "fallback tiles", g.fallback_tiles)
+
+
+def test_varlen_gqa_alpha1333_sampled(oracle):
+    w = WORKLOADS["varlen4_32k_gqa4_bf16_d128_a1.333"]
+    inputs = make_inputs(w)
+    g = parity.run_gpu(w, inputs)
+    rng = np.random.default_rng(1001)
+    tiles = _sample_tiles(w, inputs[3], 1, rng, include_ends=True)
+    loose = rng.choice(w.Hq * w.T, size=2048, replace=False)
+    s = parity.compare(w, inputs, g, tiles, loose, label=w.name)
+    print(w.name, s, "fallback tiles", g.fallback_tiles)
+
+
+def test_128k_sampled_rows(oracle):
+    """512 seeded rows per head (one-sided mask) plus 4 whole query tiles per head
+    (two-sided)."""
+    w = WORKLOADS["t128k_gqa4_bf16_d128_a1.5"]
+    inputs = make_inputs(w)
+    g = parity.run_gpu(w, inputs)
+    loose, tiles = [], []
+    for h in range(w.Hq):
+        rng = np.random.default_rng(1000 + h)
+        loose.append(h * w.T + rng.choice(w.T, size=512, replace=False))
+        tiles += [(0, h, 0, int(qt)) for qt in rng.choice(w.T // 128, size=4, replace=False)]
+    s = parity.compare(w, inputs, g, tiles, np.concatenate(loose), label=w.name)
+    print(w.name, s, "fallback tiles", g.fallback_tiles)
+
+
+SMALL = [
+    # name, kwargs for random_case
+    ("t1", dict(B=1, Hq=1, Hkv=1, T=1, d=64)),
+    ("t2_gqa", dict(B=2, Hq=4, Hkv=1, T=2, d=128)),
+    ("t127", dict(B=1, Hq=2, Hkv=2, T=127, d=64, alpha=2.0)),
+    ("t129", dict(B=1, Hq=2, Hkv=1, T=129, d=128, alpha=1.333)),
+    ("t300_a3", dict(B=2, Hq=2, Hkv=2, T=300, d=64, alpha=3.0, spike_frac=0.05, spike_scale=4.0)),
+    ("t1000_spk", dict(B=1, Hq=4, Hkv=2, T=1000, d=128, alpha=1.5, spike_frac=0.02,
+                       spike_scale=4.0)),
+    ("noncausal", dict(B=1, Hq=2, Hkv=1, T=333, d=64, alpha=1.5, causal=False)),
+    ("noncausal_a2", dict(B=2, Hq=4, Hkv=4, T=520, d=128, alpha=2.0, causal=False,
+                          spike_frac=0.02, spike_scale=4.0)),
+    ("varlen_ragged", dict(B=None, Hq=4, Hkv=2, T=None, d=128, alpha=1.5,
+                           seqlens=(5, 0, 300, 1, 129, 256))),
+    ("varlen_noncausal", dict(B=None, Hq=2, Hkv=1, T=None, d=64, alpha=1.333, causal=False,
+                              seqlens=(130, 7, 250))),
+]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] for s in SMALL])
+def test_small_cases(oracle, name, kw, dtype):
+    w, inputs = random_case(dtype=dtype, name=name, seed=7, **kw)
+    g = parity.run_gpu(w, inputs)
+    parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"{name}/{dtype}")
+
+
+@pytest.mark.parametrize("flags", [_native.FLAG_CUDA_CORES, _native.FLAG_ALL_FALLBACK,
+                                   _native.FLAG_CUDA_CORES | _native.FLAG_ALL_FALLBACK],
+                         ids=["cuda_cores", "all_fallback", "cuda_cores_all_fallback"])
+@pytest.mark.parametrize("name,kw", [SMALL[5], SMALL[7], SMALL[8]],
+                         ids=[SMALL[5][0], SMALL[7][0], SMALL[8][0]])
+def test_alternate_paths(oracle, name, kw, flags):
+    w, inputs = random_case(dtype="bf16", name=name, seed=11, **kw)
+    g = parity.run_gpu(w, inputs, flags=flags)
+    if flags & _native.FLAG_ALL_FALLBACK:
+        assert g.fallback_tiles == sum(1 for _ in parity.all_tiles(w, inputs[3]))
+    parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"{name}/{flags}")
+
+
+@pytest.mark.parametrize("alpha", [1.333, 1.5, 2.0])
+def test_candidate_overflow_is_exact(oracle, alpha):
+    """Tiny score spread (q, k scaled by 1/16) puts hundreds of keys within 1 of the row max, so
+    rows overflow the 64-slot candidate buffers; tied keys (repeated rows of k) defeat the
+    pruning too.  The result must stay exact."""
+    w, (q, k, v, cu) = random_case(B=1, Hq=2, Hkv=1, T=700, d=64, dtype="bf16", alpha=alpha,
+                                   name="overflow", seed=3)
+    q = (q.float() / 16).to(torch.bfloat16)
+    k = (k.float() / 16).to(torch.bfloat16)
+    k[:, :, 200:400] = k[:, :, 200:201]  # 200 identical keys
+    inputs = (q, k, v, cu)
+    g = parity.run_gpu(w, inputs)
+    assert g.fallback_tiles > 0
+    parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"overflow/{alpha}")
