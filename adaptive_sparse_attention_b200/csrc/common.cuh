@@ -13,6 +13,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <float.h>
 #include <stdint.h>
 
 namespace ea {
@@ -132,35 +133,43 @@ __device__ __forceinline__ float entmax_p(float x, float beta) {
   return exp2f(beta * __log2f(x));
 }
 
-// One step of the bracketed Halley + bisection search, given the sums over the keys with
-// z > tau of (z - tau)^beta, ^(beta-1), ^(beta-2).  f = S0 - 1, f' = -beta S1,
-// f'' = beta (beta - 1) S2.  The bracket [lo, hi] is narrowed by the sign of f.  The Halley
-// step is taken when its denominator 2 f'^2 - f f'' is positive and finite (then it moves
-// toward the root), otherwise the Newton step; a step outside the closed bracket becomes the
-// bracket midpoint.
-template <int BK>
-__device__ __forceinline__ float halley_step(float tau, float s0, float s1, float s2, float beta,
-                                             float& lo, float& hi) {
-  const float f = s0 - 1.f;
-  const float f1 = -beta * s1;
-  const float f2 = (BK == kBetaOne) ? 0.f : beta * (beta - 1.f) * s2;
-  if (f > 0.f) lo = tau;
-  else hi = tau;
-  const float den = 2.f * f1 * f1 - f * f2;
-  float nt;
-  if (den > 0.f && den < INFINITY) nt = tau - 2.f * f * f1 / den;
-  else nt = tau - f / f1;
-  if (!(nt >= lo && nt <= hi)) nt = 0.5f * (lo + hi);
-  return nt;
-}
+// State of the bracketed Halley + bisection search for one row: the iterate, the bracket, and
+// the lengths of the last two steps.
+struct Search {
+  float tau, lo, hi, dx, dxold;
 
-// Initial bracket of the search: p_max <= 1 gives tau >= m - 1; n keys all at most m give
-// tau <= m - n^(1 - alpha).
-__device__ __forceinline__ void initial_bracket(float m, int n, float alpha, float& lo,
-                                                float& hi) {
-  lo = m - 1.f;
-  hi = m - exp2f((1.f - alpha) * __log2f((float)n));
-}
+  // p_max <= 1 gives tau >= m - 1; n keys all at most m give tau <= m - n^(1 - alpha).
+  __device__ __forceinline__ void init(float m, int n, float alpha) {
+    lo = m - 1.f;
+    hi = m - exp2f((1.f - alpha) * __log2f((float)n));
+    tau = lo;
+    dx = dxold = hi - lo;
+  }
+
+  // One step, given the sums over the keys with z > tau of (z - tau)^beta, ^(beta-1) and
+  // ^(beta-2): f = S0 - 1, f' = -beta S1, f'' = beta (beta - 1) S2.  The bracket is narrowed by
+  // the sign of f.  The proposal is the Halley step when its denominator 2 f'^2 - f f'' is
+  // positive and finite (it then points at the root), else the Newton step.  It is taken if it
+  // lies in the closed bracket and is either within rounding of tau or at most half as long as
+  // the step before last (the progress test of the safeguarded Newton method "rtsafe",
+  // Numerical Recipes); otherwise the bracket midpoint is taken.
+  template <int BK>
+  __device__ __forceinline__ void step(float s0, float s1, float s2, float beta) {
+    const float f = s0 - 1.f;
+    const float f1 = -beta * s1;
+    const float f2 = (BK == kBetaOne) ? 0.f : beta * (beta - 1.f) * s2;
+    if (f > 0.f) lo = tau;
+    else hi = tau;
+    const float den = 2.f * f1 * f1 - f * f2;
+    float nt = (den > 0.f && den < INFINITY) ? tau - 2.f * f * f1 / den : tau - f / f1;
+    const float len = fabsf(nt - tau);
+    const bool small = len <= 4.f * FLT_EPSILON * fmaxf(1.f, fabsf(tau));
+    if (!(nt >= lo && nt <= hi && (small || len <= 0.5f * dxold))) nt = 0.5f * (lo + hi);
+    dxold = dx;
+    dx = fabsf(nt - tau);
+    tau = nt;
+  }
+};
 
 // ---------------------------------------------------------------------------------------------
 // Candidate buffer: per row (thread r of the 128 owning rows) up to kCand (raw score, key tile)
@@ -282,10 +291,10 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     const float mz = valid ? P.c * cs.m[r] : 0.f;
     const int pos = t.row0 + r;
     const int n = valid ? (P.causal ? pos + 1 : t.seq_len) : 1;
-    float lo, hi;
-    initial_bracket(mz, n, P.alpha, lo, hi);
-    float tau = lo;
+    Search sr;
+    sr.init(mz, n, P.alpha);
     for (int it = 0; it < P.n_iter; ++it) {
+      const float tau = sr.tau;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f;
       for (int e = lane4; e < cnt; e += 4) {
         const float x = P.c * cs.s[e * kTile + r] - tau;
@@ -303,8 +312,9 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
         s1 += __shfl_xor_sync(0xffffffffu, s1, o);
         s2 += __shfl_xor_sync(0xffffffffu, s2, o);
       }
-      tau = halley_step<BK>(tau, s0, s1, s2, P.beta, lo, hi);
+      sr.step<BK>(s0, s1, s2, P.beta);
     }
+    const float tau = sr.tau;
     if (!valid) continue;
     if (lane4 == 0) P.tau[t.qhead + t.seq_start + pos] = tau;
     const bool floored = cs.floor_[r] > -INFINITY;

@@ -165,10 +165,10 @@ __global__ void __launch_bounds__(kThreads) tau_fallback_kernel(Problem P) {
     });
     const float mz = row_ok ? P.c * m : 0.f;
     const int n = row_ok ? (P.causal ? pos + 1 : t.seq_len) : 1;
-    float lo, hi;
-    initial_bracket(mz, n, P.alpha, lo, hi);
-    float tau = lo;
+    Search sr;
+    sr.init(mz, n, P.alpha);
     for (int it = 0; it < P.n_iter; ++it) {
+      const float tau = sr.tau;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f;
       sweep_keys<T, D>(P, t, sm, tid, [&](int) {
         for (int jj = 0; jj < kChunk; ++jj) {
@@ -182,8 +182,9 @@ __global__ void __launch_bounds__(kThreads) tau_fallback_kernel(Problem P) {
           }
         }
       });
-      tau = halley_step<BK>(tau, s0, s1, s2, P.beta, lo, hi);
+      sr.step<BK>(s0, s1, s2, P.beta);
     }
+    const float tau = sr.tau;
     if (row_ok) P.tau[t.qhead + t.seq_start + pos] = tau;
     sweep_keys<T, D>(P, t, sm, tid, [&](int kt) {
       bool any = false;

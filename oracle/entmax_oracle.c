@@ -152,12 +152,15 @@ int oracle_entmax_vec(const double* z, int n, double alpha, int force_general, d
 
 /* Exported: the fixed-iteration bracketed Halley + bisection search for tau, in fp64.
  * Start tau = m - 1 with bracket [m - 1, m - n^(1 - alpha)].  Each of the n_iter steps
- * evaluates f = sum [z - tau]_+^beta - 1 and its first two derivatives, narrows the bracket by
- * the sign of f, and takes the Halley step tau - 2 f f' / (2 f'^2 - f f'') when its denominator
- * is positive and finite (the step then points at the root), else the Newton step - f / f'.  A
- * step that is not finite or falls outside the closed bracket [lo, hi] becomes the bracket
- * midpoint.  (With an open bracket, a tau that has converged onto an end of the bracket would
- * be thrown back to the midpoint by the next step.)  Returns the last tau. */
+ * evaluates f = sum [z - tau]_+^beta - 1 and its first two derivatives and narrows the bracket
+ * by the sign of f.  It proposes the Halley step tau - 2 f f' / (2 f'^2 - f f'') when that
+ * denominator is positive and finite (the step then points at the root), else the Newton step
+ * - f / f'.  The proposal is taken if it lies in the closed bracket [lo, hi] and either is
+ * within rounding of tau or is at most half as long as the step before last (the progress test
+ * of the safeguarded Newton method "rtsafe", Press et al., Numerical Recipes); otherwise the
+ * bracket midpoint is taken.  The closed bracket keeps a converged tau in place; the progress
+ * test breaks the two-cycles that the infinite slope of [z - tau]_+^beta at a support edge
+ * causes when beta < 1.  Returns the last tau. */
 double oracle_tau_halley(const double* z, int n, double alpha, int n_iter) {
   double beta = 1.0 / (alpha - 1.0);
   double m = -INFINITY;
@@ -166,6 +169,7 @@ double oracle_tau_halley(const double* z, int n, double alpha, int n_iter) {
   double lo = m - 1.0;
   double hi = m - pow((double)n, 1.0 - alpha);
   double tau = lo;
+  double dx = hi - lo, dxold = hi - lo; /* the last two step lengths */
   for (int it = 0; it < n_iter; ++it) {
     double s0 = 0.0, s1 = 0.0, s2 = 0.0;
     for (int j = 0; j < n; ++j) {
@@ -183,7 +187,12 @@ double oracle_tau_halley(const double* z, int n, double alpha, int n_iter) {
     else hi = tau;
     double den = 2.0 * f1 * f1 - f * f2;
     double nt = (den > 0.0 && isfinite(den)) ? tau - 2.0 * f * f1 / den : tau - f / f1;
-    if (!isfinite(nt) || !(nt >= lo && nt <= hi)) nt = 0.5 * (lo + hi);
+    double step = fabs(nt - tau);
+    int small = step <= 4.0 * DBL_EPSILON * fmax(1.0, fabs(tau));
+    if (!isfinite(nt) || !(nt >= lo && nt <= hi) || !(small || step <= 0.5 * dxold))
+      nt = 0.5 * (lo + hi);
+    dxold = dx;
+    dx = fabs(nt - tau);
     tau = nt;
   }
   return tau;

@@ -104,7 +104,8 @@ SMALL = [
     ("t2_gqa", dict(B=2, Hq=4, Hkv=1, T=2, d=128)),
     ("t127", dict(B=1, Hq=2, Hkv=2, T=127, d=64, alpha=2.0)),
     ("t129", dict(B=1, Hq=2, Hkv=1, T=129, d=128, alpha=1.333)),
-    ("t300_a3", dict(B=2, Hq=2, Hkv=2, T=300, d=64, alpha=3.0, spike_frac=0.05, spike_scale=4.0)),
+    ("t300_a3", dict(B=2, Hq=2, Hkv=2, T=300, d=64, alpha=3.0, spike_frac=0.05, spike_scale=4.0,
+                     n_iter=20)),
     ("t1000_spk", dict(B=1, Hq=4, Hkv=2, T=1000, d=128, alpha=1.5, spike_frac=0.02,
                        spike_scale=4.0)),
     ("noncausal", dict(B=1, Hq=2, Hkv=1, T=333, d=64, alpha=1.5, causal=False)),
