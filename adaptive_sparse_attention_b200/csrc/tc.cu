@@ -1,10 +1,657 @@
-// tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16.
-// Placeholder launchers until the tcgen05 kernels land: they run the CUDA-core kernels.
+// tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16, sm_100a.
+//
+// tau_tc_kernel (one CTA of 256 threads per 128-row query tile):
+//   warp 0      TMA producer: the query tile once, then the tile's key tiles through a
+//               kStages-deep shared-memory ring (128B-swizzled, K-major).
+//   warp 1      allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
+//               K = d, fp32 accumulators) into one of two TMEM score buffers.
+//   warps 4..7  score warps: tcgen05.ld of their 32 TMEM lanes (thread = query row), the
+//               running row max and the candidate buffers of common.cuh.
+//   then all 256 threads solve tau per row (4-lane groups) and warp 0 writes the block mask
+//   and the compact tile list.
+//
+// out_tc_kernel (one CTA of 256 threads per query tile, over the listed key tiles only):
+//   warp 0      TMA producer: query tile once, then (K, V) tile pairs through a 2-stage ring.
+//   warp 1      tcgen05.mma: S = Q K^T into TMEM (double buffered), then O += P V with P read
+//               from TMEM as the A operand and V (MN-major in shared memory) as B.
+//   warps 4..7  p warps: load S, p = [c s - tau]_+^beta (0 off the causal / sequence range),
+//               store p as packed bf16 into TMEM; at the end read O from TMEM and store it.
+// tau is known before this pass, so p needs neither a running max nor a final normalisation.
+//
+// Every mbarrier wait is bounded (about 2 s of %globaltimer): on expiry the waiting thread
+// records ENTMAX_ATTN_ETIMEOUT in the status word and raises a CTA-wide abort flag; every role
+// then leaves its loop, waits (bounded) for the copies and MMAs it issued, and the CTA frees its
+// tensor memory and returns.  No trap, no unbounded spin.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
 #include "kernels.h"
 
 namespace ea {
+namespace {
 
-cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s) { return launch_tau_simt(P, 1, s); }
-cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) { return launch_out_simt(P, 1, s); }
+constexpr int kThreads = 256;
+constexpr int kScoreWarp0 = 4;            // warps 4..7 own TMEM lane quarters 0..3
+constexpr int kTauStages = 4;             // key tiles in flight in the tau pass
+constexpr int kOutStages = 2;             // (key, value) tile pairs in flight in the out pass
+constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every mbarrier wait
+constexpr int kTimeoutCode = 4;           // ENTMAX_ATTN_ETIMEOUT
+
+// ------------------------------------------------------------------------------ PTX wrappers --
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (and raises the abort flag,
+// recording the timeout) if the phase did not complete within kWaitNs, or if another thread of
+// the CTA has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitNs) {
+        *abort = 1;
+        atomicExch(status, kTimeoutCode);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* holder, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(holder)),
+               "r"(ncols));
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
+                                                  bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (lane = thread).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Descriptor of a K-major 128B-swizzled operand tile of R rows whose d columns sit in 64-column
+// halves of R x 128 bytes; k16 selects the 16-column (32-byte) slice of the K dimension.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int rows, int k16) {
+  const uint32_t half = static_cast<uint32_t>(k16 >> 2) * static_cast<uint32_t>(rows) * 128u;
+  return sw128_desc(base + half + static_cast<uint32_t>(k16 & 3) * 32u, 16u, 1024u);
+}
+
+// Descriptor of the value tile as the MN-major B operand of O += P V: 128 keys (K) x d (N),
+// stored as 64-column halves of 128 rows x 128 bytes; k16 selects keys [16 k16, 16 k16 + 16).
+__device__ __forceinline__ uint64_t value_desc(uint32_t base, int k16) {
+  return sw128_desc(base + static_cast<uint32_t>(k16) * 2048u, 128u * 128u, 1024u);
+}
+
+// ------------------------------------------------------------------------------- tau kernel --
+
+template <int D>
+struct TauSmem {
+  alignas(1024) __nv_bfloat16 q[kTile * D];
+  alignas(1024) __nv_bfloat16 k[kTauStages][kTile * D];
+  CandSmem cand;
+  uint64_t q_full;
+  uint64_t k_full[kTauStages];
+  uint64_t k_empty[kTauStages];
+  uint64_t s_full[2];
+  uint64_t s_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  Problem P) {
+  extern __shared__ unsigned char smem_raw[];
+  TauSmem<D>& sm = *reinterpret_cast<TauSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  CandSmem& cs = sm.cand;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int slot = gridDim.x - 1 - blockIdx.x;  // longest query tiles first
+  const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
+  if (!t.valid) {
+    emit_empty(P, t, tid, kThreads);
+    return;
+  }
+  volatile int* abort = &sm.abort;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kTauStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_empty[b], 4);  // one arrival per score warp
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    cs.fallback = P.force_fallback;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int w = tid; w < kMaxWords; w += kThreads) cs.words[w] = 0u;
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int nkt = t.nkt;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
+      const int krow0 = static_cast<int>(t.khead + t.seq_start);
+      mbar_expect_tx(&sm.q_full, kTileBytes);
+      for (int h = 0; h < D / 64; ++h) tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
+      int issued = 0;
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int s = kt % kTauStages;
+        if (kt >= kTauStages &&
+            !mbar_wait(&sm.k_empty[s], ((kt / kTauStages) - 1) & 1, abort, P.status))
+          break;
+        mbar_expect_tx(&sm.k_full[s], kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64, krow0 + kt * kTile);
+        issued = kt + 1;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int kt = (issued > kTauStages ? issued - kTauStages : 0); kt < issued; ++kt) {
+        const int s = kt % kTauStages;
+        mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status);
+      }
+      mbar_wait(&sm.q_full, 0, abort, P.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      const uint32_t qbase = smem_u32(sm.q);
+      bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
+      int issued = 0;
+      for (int kt = 0; ok && kt < nkt; ++kt) {
+        const int s = kt % kTauStages, b = kt & 1;
+        if (!mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status)) break;
+        if (kt >= 2 && !mbar_wait(&sm.s_empty[b], ((kt >> 1) - 1) & 1, abort, P.status)) break;
+        tc_fence_after();
+        const uint32_t kbase = smem_u32(sm.k[s]);
+        const uint32_t dcol = tmem + static_cast<uint32_t>(b * 128);
+#pragma unroll
+        for (int k16 = 0; k16 < D / 16; ++k16)
+          mma_ss(dcol, kmajor_desc(qbase, kTile, k16), kmajor_desc(kbase, kTile, k16), idesc,
+                 k16 > 0 ? 1u : 0u);
+        mma_commit(&sm.k_empty[s]);
+        mma_commit(&sm.s_full[b]);
+        issued = kt + 1;
+      }
+      if (issued > 0) {  // all issued MMAs complete before tensor memory is released
+        mma_commit(&sm.drain);
+        mbar_wait(&sm.drain, 0, abort, P.status);
+      }
+    }
+  } else if (warp >= kScoreWarp0) {
+    const int quarter = warp - kScoreWarp0;
+    const int r = quarter * 32 + lane;  // query row of the tile == TMEM lane
+    const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+    RowCand rc;
+    rc.init(1.f / P.c);
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int b = kt & 1;
+      if (!mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort, P.status)) break;
+      tc_fence_after();
+      const uint32_t row_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                static_cast<uint32_t>(b * 128);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t u0[32], u1[32];
+        tmem_ld32(row_addr + half * 64, u0);
+        tmem_ld32(row_addr + half * 64 + 32, u1);
+        tmem_wait_ld();
+        float x0[32], x1[32];
+        const int j0 = kt * kTile + half * 64;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x0[i] = (j0 + i < jmax) ? __uint_as_float(u0[i]) : -INFINITY;
+          x1[i] = (j0 + 32 + i < jmax) ? __uint_as_float(u1[i]) : -INFINITY;
+        }
+        rc.feed<32>(cs, r, x0, kt);
+        rc.feed<32>(cs, r, x1, kt);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_empty[b]);
+    }
+    rc.publish(cs, r);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (*abort) return;  // status already records the timeout; outputs of this tile are void
+  solve_rows<BK>(P, t, cs, tid, kThreads);
+  __syncthreads();
+  if (warp == 0) emit_tile(P, t, cs.words, cs.fallback, lane);
+}
+
+// ------------------------------------------------------------------------------- out kernel --
+
+template <int D>
+struct OutSmem {
+  alignas(1024) __nv_bfloat16 q[kTile * D];
+  alignas(1024) __nv_bfloat16 k[kOutStages][kTile * D];
+  alignas(1024) __nv_bfloat16 v[kOutStages][kTile * D];
+  uint64_t q_full;
+  uint64_t kv_full[kOutStages];
+  uint64_t kv_empty[kOutStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t p_free[2];  // PV MMA that read P[b] has completed
+  uint64_t o_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// TMEM columns: S[0], S[1] at 0 and 128; P[0], P[1] (128 keys as 64 packed bf16x2 columns) at
+// 256 and 320; O (d fp32 columns) at 384.
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    out_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv, Problem P) {
+  extern __shared__ unsigned char smem_raw[];
+  OutSmem<D>& sm = *reinterpret_cast<OutSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int slot = gridDim.x - 1 - blockIdx.x;
+  const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
+  if (!t.valid) return;
+  const int cnt = P.count[t.tile_id];
+  const int* list = P.list + t.tile_id * P.nkt_max;
+  volatile int* abort = &sm.abort;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kOutStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.p_full[b], 4);
+      mbar_init(&sm.p_free[b], 1);
+    }
+    mbar_init(&sm.o_full, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
+      const int krow0 = static_cast<int>(t.khead + t.seq_start);
+      mbar_expect_tx(&sm.q_full, kTileBytes);
+      for (int h = 0; h < D / 64; ++h) tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
+      int issued = 0;
+      for (int i = 0; i < cnt; ++i) {
+        const int s = i % kOutStages;
+        if (i >= kOutStages &&
+            !mbar_wait(&sm.kv_empty[s], ((i / kOutStages) - 1) & 1, abort, P.status))
+          break;
+        const int row = krow0 + list[i] * kTile;
+        mbar_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.kv_full[s], h * 64, row);
+          tma_load_2d(sm.v[s] + h * kTile * 64, &tmv, &sm.kv_full[s], h * 64, row);
+        }
+        issued = i + 1;
+      }
+      for (int i = (issued > kOutStages ? issued - kOutStages : 0); i < issued; ++i)
+        mbar_wait(&sm.kv_full[i % kOutStages], (i / kOutStages) & 1, abort, P.status);
+      mbar_wait(&sm.q_full, 0, abort, P.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
+      const uint32_t qbase = smem_u32(sm.q);
+      bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
+      // S(i) = Q K(i)^T into S[i & 1]
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % kOutStages, b = i & 1;
+        if (!mbar_wait(&sm.kv_full[s], (i / kOutStages) & 1, abort, P.status)) return false;
+        // S[b] is free once the p warps have read S(i-2): they signal that through p_full.
+        if (i >= 2 && !mbar_wait(&sm.p_full[b], ((i >> 1) - 1) & 1, abort, P.status))
+          return false;
+        tc_fence_after();
+        const uint32_t kbase = smem_u32(sm.k[s]);
+#pragma unroll
+        for (int k16 = 0; k16 < D / 16; ++k16)
+          mma_ss(tmem + kColS + b * 128, kmajor_desc(qbase, kTile, k16),
+                 kmajor_desc(kbase, kTile, k16), idesc_s, k16 > 0 ? 1u : 0u);
+        mma_commit(&sm.s_full[b]);
+        return true;
+      };
+      int done = 0;  // PV products issued
+      if (ok && cnt > 0) ok = issue_s(0);
+      for (int i = 0; ok && i < cnt; ++i) {
+        const int s = i % kOutStages, b = i & 1;
+        if (i + 1 < cnt && !issue_s(i + 1)) break;
+        if (!mbar_wait(&sm.p_full[b], (i >> 1) & 1, abort, P.status)) break;
+        tc_fence_after();
+        const uint32_t vbase = smem_u32(sm.v[s]);
+#pragma unroll
+        for (int k16 = 0; k16 < kTile / 16; ++k16)
+          mma_ts(tmem + kColO, tmem + kColP + b * 64 + k16 * 8, value_desc(vbase, k16), idesc_o,
+                 (i > 0 || k16 > 0) ? 1u : 0u);
+        mma_commit(&sm.kv_empty[s]);
+        mma_commit(&sm.p_free[b]);
+        done = i + 1;
+      }
+      (void)done;
+      mma_commit(&sm.o_full);  // arrives once every MMA issued so far has completed
+    }
+  } else if (warp >= kScoreWarp0) {
+    const int quarter = warp - kScoreWarp0;
+    const int r = quarter * 32 + lane;
+    const bool row_ok = r < t.nrows;
+    const int pos = t.row0 + r;
+    const int jmax = row_ok ? (P.causal ? pos + 1 : t.seq_len) : 0;
+    const float tau = row_ok ? P.tau[t.qhead + t.seq_start + pos] : INFINITY;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    for (int i = 0; i < cnt; ++i) {
+      const int b = i & 1;
+      const int kt = list[i];
+      if (!mbar_wait(&sm.s_full[b], (i >> 1) & 1, abort, P.status)) break;
+      // P[b] is free once the PV product of step i-2 has completed
+      if (i >= 2 && !mbar_wait(&sm.p_free[b], ((i >> 1) - 1) & 1, abort, P.status)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + kColS + b * 128 + q4 * 32, u);
+        tmem_wait_ld();
+        uint32_t pk[16];
+        const int j0 = kt * kTile + q4 * 32;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float s0 = __uint_as_float(u[2 * e]), s1 = __uint_as_float(u[2 * e + 1]);
+          const float p0 = (j0 + 2 * e < jmax) ? entmax_p<BK>(P.c * s0 - tau, P.beta) : 0.f;
+          const float p1 = (j0 + 2 * e + 1 < jmax) ? entmax_p<BK>(P.c * s1 - tau, P.beta) : 0.f;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tmem + lane_off + kColP + b * 64 + q4 * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[b]);
+    }
+    // epilogue: O rows from TMEM to global memory
+    const bool o_ok = mbar_wait(&sm.o_full, 0, abort, P.status);
+    tc_fence_after();
+    if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (only after a failed tau pass)
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) +
+                                            (t.qhead + t.seq_start + pos) * D);
+      for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+    } else if (o_ok && !*abort) {
+      __nv_bfloat16* op = static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + kColO + c0, u);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(op + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(u[8 * e + 0]), __uint_as_float(u[8 * e + 1]));
+            w.y = pack_bf16x2(__uint_as_float(u[8 * e + 2]), __uint_as_float(u[8 * e + 3]));
+            w.z = pack_bf16x2(__uint_as_float(u[8 * e + 4]), __uint_as_float(u[8 * e + 5]));
+            w.w = pack_bf16x2(__uint_as_float(u[8 * e + 6]), __uint_as_float(u[8 * e + 7]));
+            dst[e] = w;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------------------ host side --
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a [rows, d] bf16 matrix, box of 128 rows x 64 columns, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* map, const void* base, int64_t rows, int d) {
+  auto enc = get_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int64_t q_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) * P.Hq * P.T; }
+int64_t kv_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) * P.Hkv * P.T; }
+
+dim3 tile_grid(const Problem& P) { return dim3(P.slots, P.Hq, P.cu ? 1 : P.B); }
+
+template <int D, int BK>
+cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
+  CUtensorMap mq, mk;
+  cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(TauSmem<D>) + 1024;
+  auto kern = tau_tc_kernel<D, BK>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<tile_grid(P), kThreads, smem, s>>>(mq, mk, P);
+  return cudaGetLastError();
+}
+
+template <int D, int BK>
+cudaError_t launch_out_t(const Problem& P, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mv, P.v, kv_rows(P), D);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(OutSmem<D>) + 1024;
+  auto kern = out_tc_kernel<D, BK>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<tile_grid(P), kThreads, smem, s>>>(mq, mk, mv, P);
+  return cudaGetLastError();
+}
+
+#define EA_TC_DISPATCH(FN)                                          \
+  do {                                                              \
+    const int bk = beta_kind(P.beta);                               \
+    if (P.d == 64) {                                                \
+      if (bk == kBetaOne) return FN<64, kBetaOne>(P, s);            \
+      if (bk == kBetaTwo) return FN<64, kBetaTwo>(P, s);            \
+      return FN<64, kBetaGeneral>(P, s);                            \
+    }                                                               \
+    if (bk == kBetaOne) return FN<128, kBetaOne>(P, s);             \
+    if (bk == kBetaTwo) return FN<128, kBetaTwo>(P, s);             \
+    return FN<128, kBetaGeneral>(P, s);                             \
+  } while (0)
+
+}  // namespace
+
+cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s) { EA_TC_DISPATCH(launch_tau_t); }
+cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) { EA_TC_DISPATCH(launch_out_t); }
 
 }  // namespace ea

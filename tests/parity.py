@@ -22,6 +22,18 @@ from oracle import oracle
 
 TILE = 128
 OUT_TOL = {"fp32": 1e-4, "bf16": 2e-2}
+
+
+def out_tolerance(w: Workload) -> float:
+    """Max-abs bar for o.  For alpha > 2 (beta < 1) the map x -> x^beta has unbounded slope at
+    0, so a rounding error delta of an fp32 score moves p by up to delta^beta near a support
+    edge; with delta <= 2^-20 (a few ulps of |z| <= 8) the fp32 bar becomes
+    1e-4 + 2^(-20 beta).  bf16 inputs keep 2e-2."""
+    tol = OUT_TOL[w.dtype]
+    beta = 1.0 / (oracle.alpha_as_float32(w.alpha) - 1.0)
+    if w.dtype == "fp32" and beta < 1.0:
+        tol += 2.0 ** (-20.0 * beta)
+    return tol
 TAU_RTOL = 1e-4
 MASK_EXEMPT_P = 1e-6
 
@@ -105,7 +117,7 @@ def compare(w: Workload, inputs, g: GpuResult, whole_tiles, loose_rows=None, lab
     rows = np.concatenate(groups + ([np.asarray(loose_rows, dtype=np.int64)]
                                     if loose_rows is not None and len(loose_rows) else []))
     ref = oracle.attention_rows(q, k, v, alpha, w.causal, cu, rows)
-    tol = OUT_TOL[w.dtype]
+    tol = out_tolerance(w)
     err_out = np.abs(g.out[rows] - ref["out"])
     max_out = float(err_out.max()) if err_out.size else 0.0
     tau_g = g.tau[rows].astype(np.float64)
