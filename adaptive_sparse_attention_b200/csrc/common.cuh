@@ -19,7 +19,10 @@
 namespace ea {
 
 constexpr int kTile = 128;      // query-tile rows and key-tile keys (block-mask granularity)
-constexpr int kCand = 64;       // candidate slots per row held in shared memory
+constexpr int kSeg = 2;         // key segments per row (keys 0-63 / 64-127 of every key tile),
+                                // each with its own running max and candidate buffer
+constexpr int kCand = 32;       // candidate slots per (row, segment) held in shared memory
+constexpr int kCols = kSeg * kTile;  // (row, segment) columns of the candidate buffers
 constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
 
 enum BetaKind { kBetaOne = 0, kBetaTwo = 1, kBetaGeneral = 2 };
@@ -172,21 +175,42 @@ struct Search {
 };
 
 // ---------------------------------------------------------------------------------------------
-// Candidate buffer: per row (thread r of the 128 owning rows) up to kCand (raw score, key tile)
-// pairs in shared memory, entry e of row r at [e * 128 + r] so that a warp's rows hit distinct
-// banks whatever their fill levels.
+// Candidate buffers: for every (row r, segment g) -- column c = g * 128 + r -- up to kCand
+// (raw score, key tile) pairs in shared memory, entry e at [e * 256 + c], so that the 32 rows of
+// a warp hit 32 distinct banks whatever their fill levels.  A segment owns the keys 64 g .. 64 g
+// + 63 of every key tile; its running max is a max over those keys only, which keeps a superset
+// of the row's candidates (its threshold is never above the row's).
 // ---------------------------------------------------------------------------------------------
 struct CandSmem {
-  float s[kCand * kTile];
-  uint16_t kt[kCand * kTile];
-  float m[kTile];       // row max of raw scores
-  float floor_[kTile];  // pruning floor (raw); -inf when the row was never pruned
-  int cnt[kTile];
-  int lost[kTile];
+  float s[kCand * kCols];
+  uint16_t kt[kCand * kCols];
+  float m[kCols];       // segment max of raw scores
+  float floor_[kCols];  // pruning floor (raw); -inf when the segment was never pruned
+  int cnt[kCols];
+  int lost[kCols];
   uint32_t words[kMaxWords];
   int fallback;         // some row of the tile needs the overflow path
 };
 
+// max of three floats in one instruction
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max of x[o .. o + 16)
+template <int N>
+__device__ __forceinline__ float max16(const float (&x)[N], int o) {
+  const float a = max3f(x[o], x[o + 1], x[o + 2]);
+  const float b = max3f(x[o + 3], x[o + 4], x[o + 5]);
+  const float c = max3f(x[o + 6], x[o + 7], x[o + 8]);
+  const float d = max3f(x[o + 9], x[o + 10], x[o + 11]);
+  const float e = max3f(x[o + 12], x[o + 13], x[o + 14]);
+  return max3f(max3f(a, b, c), max3f(d, e, x[o + 15]), -INFINITY);
+}
+
+// Candidate state of one (row, segment), held in registers by the thread that owns it.
 struct RowCand {
   float m;       // running max of raw scores
   float thr;     // keep threshold: max(m - 1/c, floor)
@@ -207,77 +231,76 @@ struct RowCand {
   // Drops entries at or below the threshold; while more than half the slots stay in use, raises
   // the floor halfway to the running max (entries below the floor can only matter if tau ends
   // up at or below it, which the solve checks).
-  __device__ __noinline__ void compact(CandSmem& cs, int r) {
-    int n = 0;
-    for (int e = 0; e < cnt; ++e) {
-      const float x = cs.s[e * kTile + r];
-      if (x > thr) {
-        cs.s[n * kTile + r] = x;
-        cs.kt[n * kTile + r] = cs.kt[e * kTile + r];
-        ++n;
-      }
-    }
-    cnt = n;
-    for (int guard = 0; cnt > kCand / 2 && guard < 8; ++guard) {
-      floor_ = thr + 0.5f * (m - thr);
-      thr = floor_;
-      n = 0;
+  __device__ __forceinline__ void compact(CandSmem& cs, int col) {
+    for (int guard = 0; guard < 9; ++guard) {
+      int n = 0;
       for (int e = 0; e < cnt; ++e) {
-        const float x = cs.s[e * kTile + r];
+        const float x = cs.s[e * kCols + col];
         if (x > thr) {
-          cs.s[n * kTile + r] = x;
-          cs.kt[n * kTile + r] = cs.kt[e * kTile + r];
+          cs.s[n * kCols + col] = x;
+          cs.kt[n * kCols + col] = cs.kt[e * kCols + col];
           ++n;
         }
       }
       cnt = n;
+      if (cnt <= kCand / 2) break;
+      floor_ = thr + 0.5f * (m - thr);
+      thr = floor_;
     }
   }
 
-  __device__ __forceinline__ void push(CandSmem& cs, int r, float x, int kt) {
-    if (lost) return;
-    if (cnt == kCand) {
-      compact(cs, r);
-      if (cnt == kCand) {
-        lost = 1;
-        return;
-      }
-    }
-    cs.s[cnt * kTile + r] = x;
-    cs.kt[cnt * kTile + r] = (uint16_t)kt;
-    ++cnt;
-  }
-
-  // Feeds N raw scores of key tile kt (invalid keys already -inf).
+  // Feeds N raw scores of key tile kt (keys outside the row's range already -inf).  The hot path
+  // is the max of each 16-key block; only a block whose max passes the threshold is scanned.
   template <int N>
-  __device__ __forceinline__ void feed(CandSmem& cs, int r, const float (&x)[N], int kt) {
-    float cmax = x[0];
+  __device__ __forceinline__ void feed(CandSmem& cs, int col, const float (&x)[N], int kt) {
+    static_assert(N % 16 == 0, "16-key blocks");
+    constexpr int NB = N / 16;
+    float sub[NB];
 #pragma unroll
-    for (int i = 1; i < N; ++i) cmax = fmaxf(cmax, x[i]);
+    for (int k = 0; k < NB; ++k) sub[k] = max16(x, 16 * k);
+    float cmax = sub[0];
+#pragma unroll
+    for (int k = 1; k < NB; ++k) cmax = fmaxf(cmax, sub[k]);
     if (cmax > thr) {
       if (cmax > m) {
         m = cmax;
         thr = fmaxf(m - inv_c, floor_);
       }
 #pragma unroll
-      for (int i = 0; i < N; ++i)
-        if (x[i] > thr) push(cs, r, x[i], kt);
+      for (int k = 0; k < NB; ++k) {
+        if (sub[k] > thr) {
+          if (cnt > kCand - 16) compact(cs, col);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float v = x[16 * k + i];
+            if (v > thr) {
+              if (cnt < kCand) {
+                cs.s[cnt * kCols + col] = v;
+                cs.kt[cnt * kCols + col] = static_cast<uint16_t>(kt);
+                ++cnt;
+              } else {
+                lost = 1;
+              }
+            }
+          }
+        }
+      }
     }
   }
 
-  __device__ __forceinline__ void publish(CandSmem& cs, int r) const {
-    cs.m[r] = m;
-    cs.floor_[r] = floor_;
-    cs.cnt[r] = cnt;
-    cs.lost[r] = lost;
+  __device__ __forceinline__ void publish(CandSmem& cs, int col) const {
+    cs.m[col] = m;
+    cs.floor_[col] = floor_;
+    cs.cnt[col] = cnt;
+    cs.lost[col] = lost;
   }
 };
 
-// Solves tau for every row of the tile from the published candidate buffers, writes tau and
-// sets the tile's mask words in shared memory.  Rows are handled by groups of 4 lanes that
-// split a row's candidates and combine their partial sums with warp shuffles.  nthreads must be
-// a multiple of 32; call from all threads of the block after a __syncthreads() that follows
-// publish().
+// Solves tau for every row of the tile from the published candidate buffers of both segments,
+// writes tau and sets the tile's mask words in shared memory.  Rows are handled by groups of 4
+// lanes that split a row's candidates and combine their partial sums with warp shuffles.
+// nthreads must be a multiple of 32; call from all threads of the block after a
+// __syncthreads() that follows publish().
 template <int BK>
 __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, int tid,
                            int nthreads) {
@@ -287,8 +310,9 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
   // whole warp); rows past the end of the tile run on an empty candidate list and store nothing.
   for (int r = tid >> 2; r < kTile; r += groups) {
     const bool valid = r < t.nrows;
-    const int cnt = valid ? cs.cnt[r] : 0;
-    const float mz = valid ? P.c * cs.m[r] : 0.f;
+    const int cnt0 = valid ? cs.cnt[r] : 0;
+    const int cnt = valid ? cnt0 + cs.cnt[kTile + r] : 0;
+    const float mz = valid ? P.c * fmaxf(cs.m[r], cs.m[kTile + r]) : 0.f;
     const int pos = t.row0 + r;
     const int n = valid ? (P.causal ? pos + 1 : t.seq_len) : 1;
     Search sr;
@@ -297,7 +321,8 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
       const float tau = sr.tau;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f;
       for (int e = lane4; e < cnt; e += 4) {
-        const float x = P.c * cs.s[e * kTile + r] - tau;
+        const int idx = (e < cnt0) ? e * kCols + r : (e - cnt0) * kCols + kTile + r;
+        const float x = P.c * cs.s[idx] - tau;
         if (x > 0.f) {
           float a, b, c2;
           entmax_powers<BK>(x, P.beta, a, b, c2);
@@ -317,11 +342,17 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     const float tau = sr.tau;
     if (!valid) continue;
     if (lane4 == 0) P.tau[t.qhead + t.seq_start + pos] = tau;
-    const bool floored = cs.floor_[r] > -INFINITY;
-    if (cs.lost[r] || (floored && !(tau > P.c * cs.floor_[r]))) cs.fallback = 1;
+    bool bad = cs.lost[r] || cs.lost[kTile + r];
+#pragma unroll
+    for (int g = 0; g < kSeg; ++g) {
+      const float fl = cs.floor_[g * kTile + r];
+      if (fl > -INFINITY && !(tau > P.c * fl)) bad = true;
+    }
+    if (bad) cs.fallback = 1;
     for (int e = lane4; e < cnt; e += 4) {
-      if (P.c * cs.s[e * kTile + r] > tau) {
-        const int kt = cs.kt[e * kTile + r];
+      const int idx = (e < cnt0) ? e * kCols + r : (e - cnt0) * kCols + kTile + r;
+      if (P.c * cs.s[idx] > tau) {
+        const int kt = cs.kt[idx];
         atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
       }
     }
@@ -363,6 +394,12 @@ __device__ __forceinline__ void emit_tile(const Problem& P, const TileInfo& t,
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (lane == 0) P.count[t.tile_id] = base;
+}
+
+// A compact-list entry forced into [0, nkt): out-of-range values (an unfilled workspace) read
+// key tile 0 instead of memory outside the problem.
+__device__ __forceinline__ int clamp_kt(int kt, int nkt) {
+  return (kt >= 0 && kt < nkt) ? kt : 0;
 }
 
 // Unused slot of a packed batch: zero mask words, empty list.

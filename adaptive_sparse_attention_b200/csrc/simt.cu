@@ -125,15 +125,20 @@ __global__ void __launch_bounds__(kThreads) tau_simt_kernel(Problem P) {
   if (tid == 0) cs.fallback = P.force_fallback;
   load_q_tile<T, D>(P, t, sm.qs, tid);
 
-  RowCand rc;
-  rc.init(1.f / P.c);
+  // chunks 0-1 of a key tile are keys 0-63 (segment 0), chunks 2-3 keys 64-127 (segment 1)
+  RowCand rc0, rc1;
+  rc0.init(1.f / P.c);
+  rc1.init(1.f / P.c);
+  int chunk = 0;
   sweep_keys<T, D>(P, t, sm, tid, [&](int kt) {
     float x[kChunk];
 #pragma unroll
     for (int jj = 0; jj < kChunk; ++jj) x[jj] = sm.xs[jj * kTile + tid];
-    rc.feed<kChunk>(cs, tid, x, kt);
+    if ((chunk++ & 2) == 0) rc0.feed<kChunk>(cs, tid, x, kt);
+    else rc1.feed<kChunk>(cs, kTile + tid, x, kt);
   });
-  rc.publish(cs, tid);
+  rc0.publish(cs, tid);
+  rc1.publish(cs, kTile + tid);
   __syncthreads();
   solve_rows<BK>(P, t, cs, tid, kThreads);
   __syncthreads();
@@ -146,9 +151,11 @@ __global__ void __launch_bounds__(kThreads) tau_fallback_kernel(Problem P) {
   SimtSmem<D>& sm = *reinterpret_cast<SimtSmem<D>*>(smem);
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + sizeof(SimtSmem<D>));
   const int tid = threadIdx.x;
-  const int nq = *P.queue_count;
+  const int ntiles = (P.cu ? 1 : P.B) * P.Hq * P.slots;
+  const int nq = min(*P.queue_count, ntiles);
   for (int i = blockIdx.x; i < nq; i += gridDim.x) {
     const int id = P.queue[i];
+    if (id < 0 || id >= ntiles) continue;  // uniform across the block
     const int slot = id % P.slots;
     const int h = (id / P.slots) % P.Hq;
     const int b = id / (P.slots * P.Hq);
@@ -215,10 +222,10 @@ __global__ void __launch_bounds__(kThreads) out_simt_kernel(Problem P) {
 #pragma unroll
   for (int c = 0; c < D; ++c) o[c] = 0.f;
 
-  const int cnt = P.count[t.tile_id];
+  const int cnt = min(max(P.count[t.tile_id], 0), t.nkt);  // see clamp_kt
   const int* list = P.list + t.tile_id * P.nkt_max;
   for (int i = 0; i < cnt; ++i) {
-    const int kt = list[i];
+    const int kt = clamp_kt(list[i], t.nkt);
     for (int ch = 0; ch < kTile / kChunk; ++ch) {
       const int j0 = kt * kTile + ch * kChunk;
       if (j0 >= t.seq_len) break;

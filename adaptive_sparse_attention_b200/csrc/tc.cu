@@ -1,13 +1,14 @@
 // tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16, sm_100a.
 //
-// tau_tc_kernel (one CTA of 256 threads per 128-row query tile):
+// tau_tc_kernel (one CTA of 384 threads per 128-row query tile):
 //   warp 0      TMA producer: the query tile once, then the tile's key tiles through a
 //               kStages-deep shared-memory ring (128B-swizzled, K-major).
 //   warp 1      allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
 //               K = d, fp32 accumulators) into one of two TMEM score buffers.
-//   warps 4..7  score warps: tcgen05.ld of their 32 TMEM lanes (thread = query row), the
-//               running row max and the candidate buffers of common.cuh.
-//   then all 256 threads solve tau per row (4-lane groups) and warp 0 writes the block mask
+//   warps 4..11 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
+//               columns 64 s .. 64 s + 63 with s = (w - 4) / 4, i.e. one 64-key segment of every
+//               key tile, into the segment's running max and candidate buffer (common.cuh).
+//   then all 384 threads solve tau per row (4-lane groups) and warp 0 writes the block mask
 //   and the compact tile list.
 //
 // out_tc_kernel (one CTA of 256 threads per query tile, over the listed key tiles only):
@@ -36,8 +37,9 @@
 namespace ea {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kScoreWarp0 = 4;            // warps 4..7 own TMEM lane quarters 0..3
+constexpr int kOutThreads = 256;
+constexpr int kTauThreads = 384;
+constexpr int kScoreWarp0 = 4;            // score / p warps start at warp 4 (lane quarter w % 4)
 constexpr int kTauStages = 4;             // key tiles in flight in the tau pass
 constexpr int kOutStages = 2;             // (key, value) tile pairs in flight in the out pass
 constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every mbarrier wait
@@ -223,6 +225,25 @@ __device__ __forceinline__ uint64_t value_desc(uint32_t base, int k16) {
   return sw128_desc(base + static_cast<uint32_t>(k16) * 2048u, 128u * 128u, 1024u);
 }
 
+// 64 raw scores of this thread's row from TMEM columns [ta, ta + 64), keys j0 + i; keys at or
+// past jmax (outside the row's causal / sequence range) read as -inf.
+__device__ __forceinline__ void tmem_row64(uint32_t ta, int j0, int jmax, float (&x)[64]) {
+  uint32_t u0[32], u1[32];
+  tmem_ld32(ta, u0);
+  tmem_ld32(ta + 32, u1);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    x[i] = __uint_as_float(u0[i]);
+    x[32 + i] = __uint_as_float(u1[i]);
+  }
+  if (j0 + 64 > jmax) {  // diagonal or ragged tile
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (j0 + i >= jmax) x[i] = -INFINITY;
+  }
+}
+
 // ------------------------------------------------------------------------------- tau kernel --
 
 template <int D>
@@ -241,7 +262,7 @@ struct TauSmem {
 };
 
 template <int D, int BK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kTauThreads, 1)
     tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   Problem P) {
   extern __shared__ unsigned char smem_raw[];
@@ -253,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int slot = gridDim.x - 1 - blockIdx.x;  // longest query tiles first
   const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
   if (!t.valid) {
-    emit_empty(P, t, tid, kThreads);
+    emit_empty(P, t, tid, kTauThreads);
     return;
   }
   volatile int* abort = &sm.abort;
@@ -267,14 +288,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_empty[b], 4);  // one arrival per score warp
+      mbar_init(&sm.s_empty[b], 8);  // one arrival per score warp
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     cs.fallback = P.force_fallback;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int w = tid; w < kMaxWords; w += kThreads) cs.words[w] = 0u;
+  for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
   if (warp == 1) tmem_alloc(&sm.tmem_base, 256);
   tc_fence_before();
   __syncthreads();
@@ -333,8 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kScoreWarp0) {
-    const int quarter = warp - kScoreWarp0;
+    const int quarter = warp & 3;
+    const int seg = (warp - kScoreWarp0) >> 2;
     const int r = quarter * 32 + lane;  // query row of the tile == TMEM lane
+    const int col = seg * kTile + r;
     const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
     RowCand rc;
     rc.init(1.f / P.c);
@@ -342,36 +365,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = kt & 1;
       if (!mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort, P.status)) break;
       tc_fence_after();
-      const uint32_t row_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                static_cast<uint32_t>(b * 128);
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t u0[32], u1[32];
-        tmem_ld32(row_addr + half * 64, u0);
-        tmem_ld32(row_addr + half * 64 + 32, u1);
-        tmem_wait_ld();
-        float x0[32], x1[32];
-        const int j0 = kt * kTile + half * 64;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x0[i] = (j0 + i < jmax) ? __uint_as_float(u0[i]) : -INFINITY;
-          x1[i] = (j0 + 32 + i < jmax) ? __uint_as_float(u1[i]) : -INFINITY;
-        }
-        rc.feed<32>(cs, r, x0, kt);
-        rc.feed<32>(cs, r, x1, kt);
-      }
+      const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                          static_cast<uint32_t>(b * 128 + seg * 64);
+      float x[64];
+      tmem_row64(ta, kt * kTile + seg * 64, jmax, x);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_empty[b]);
+      if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
+      rc.feed<64>(cs, col, x, kt);
     }
-    rc.publish(cs, r);
+    rc.publish(cs, col);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 256);
   if (*abort) return;  // status already records the timeout; outputs of this tile are void
-  solve_rows<BK>(P, t, cs, tid, kThreads);
+  solve_rows<BK>(P, t, cs, tid, kTauThreads);
   __syncthreads();
   if (warp == 0) emit_tile(P, t, cs.words, cs.fallback, lane);
 }
@@ -399,7 +409,7 @@ struct OutSmem {
 constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 
 template <int D, int BK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kOutThreads, 1)
     out_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, Problem P) {
   extern __shared__ unsigned char smem_raw[];
@@ -410,7 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int slot = gridDim.x - 1 - blockIdx.x;
   const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
-  const int cnt = P.count[t.tile_id];
+  // The list comes from the tau pass; clamping keeps every read inside this tile's list and key
+  // range even if the workspace was never filled.
+  const int cnt = min(max(P.count[t.tile_id], 0), t.nkt);
   const int* list = P.list + t.tile_id * P.nkt_max;
   volatile int* abort = &sm.abort;
   constexpr uint32_t kTileBytes = kTile * D * 2;
@@ -448,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i >= kOutStages &&
             !mbar_wait(&sm.kv_empty[s], ((i / kOutStages) - 1) & 1, abort, P.status))
           break;
-        const int row = krow0 + list[i] * kTile;
+        const int row = krow0 + clamp_kt(list[i], t.nkt) * kTile;
         mbar_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
         for (int h = 0; h < D / 64; ++h) {
           tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.kv_full[s], h * 64, row);
@@ -511,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     for (int i = 0; i < cnt; ++i) {
       const int b = i & 1;
-      const int kt = list[i];
+      const int kt = clamp_kt(list[i], t.nkt);
       if (!mbar_wait(&sm.s_full[b], (i >> 1) & 1, abort, P.status)) break;
       // P[b] is free once the PV product of step i-2 has completed
       if (i >= 2 && !mbar_wait(&sm.p_free[b], ((i >> 1) - 1) & 1, abort, P.status)) break;
@@ -617,7 +629,7 @@ cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
   auto kern = tau_tc_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<tile_grid(P), kThreads, smem, s>>>(mq, mk, P);
+  kern<<<tile_grid(P), kTauThreads, smem, s>>>(mq, mk, P);
   return cudaGetLastError();
 }
 
@@ -632,7 +644,7 @@ cudaError_t launch_out_t(const Problem& P, cudaStream_t s) {
   auto kern = out_tc_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<tile_grid(P), kThreads, smem, s>>>(mq, mk, mv, P);
+  kern<<<tile_grid(P), kOutThreads, smem, s>>>(mq, mk, mv, P);
   return cudaGetLastError();
 }
 
