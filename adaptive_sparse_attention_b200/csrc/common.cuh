@@ -228,66 +228,6 @@ struct RowCand {
     lost = 0;
   }
 
-  // Drops entries at or below the threshold; while more than half the slots stay in use, raises
-  // the floor halfway to the running max (entries below the floor can only matter if tau ends
-  // up at or below it, which the solve checks).
-  __device__ __forceinline__ void compact(CandSmem& cs, int col) {
-    for (int guard = 0; guard < 9; ++guard) {
-      int n = 0;
-      for (int e = 0; e < cnt; ++e) {
-        const float x = cs.s[e * kCols + col];
-        if (x > thr) {
-          cs.s[n * kCols + col] = x;
-          cs.kt[n * kCols + col] = cs.kt[e * kCols + col];
-          ++n;
-        }
-      }
-      cnt = n;
-      if (cnt <= kCand / 2) break;
-      floor_ = thr + 0.5f * (m - thr);
-      thr = floor_;
-    }
-  }
-
-  // Feeds N raw scores of key tile kt (keys outside the row's range already -inf).  The hot path
-  // is the max of each 16-key block; only a block whose max passes the threshold is scanned.
-  template <int N>
-  __device__ __forceinline__ void feed(CandSmem& cs, int col, const float (&x)[N], int kt) {
-    static_assert(N % 16 == 0, "16-key blocks");
-    constexpr int NB = N / 16;
-    float sub[NB];
-#pragma unroll
-    for (int k = 0; k < NB; ++k) sub[k] = max16(x, 16 * k);
-    float cmax = sub[0];
-#pragma unroll
-    for (int k = 1; k < NB; ++k) cmax = fmaxf(cmax, sub[k]);
-    if (cmax > thr) {
-      if (cmax > m) {
-        m = cmax;
-        thr = fmaxf(m - inv_c, floor_);
-      }
-#pragma unroll
-      for (int k = 0; k < NB; ++k) {
-        if (sub[k] > thr) {
-          if (cnt > kCand - 16) compact(cs, col);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float v = x[16 * k + i];
-            if (v > thr) {
-              if (cnt < kCand) {
-                cs.s[cnt * kCols + col] = v;
-                cs.kt[cnt * kCols + col] = static_cast<uint16_t>(kt);
-                ++cnt;
-              } else {
-                lost = 1;
-              }
-            }
-          }
-        }
-      }
-    }
-  }
-
   __device__ __forceinline__ void publish(CandSmem& cs, int col) const {
     cs.m[col] = m;
     cs.floor_[col] = floor_;
@@ -295,6 +235,133 @@ struct RowCand {
     cs.lost[col] = lost;
   }
 };
+
+static_assert(kCand == 32, "one candidate slot per lane in the warp-cooperative compaction");
+
+// Warp-cooperative insertion for lane src (buffer column col_src) when its buffer cannot take
+// all of its passing values: lane e holds old entry e, and lanes e and e + 32 of src's chunk x
+// are spread over the warp by shuffles.  Old entries and new values at or below the threshold
+// are dropped; while more than kCand survive, the floor is raised halfway to the running max
+// (entries below the floor can only matter if tau ends up at or below it, which the solve
+// checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
+// of the buffer.  Call with the whole warp converged; x is read from lane src only.
+template <int N>
+__device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, int col_src,
+                                            const float (&x)[N], int kt, int lane) {
+  static_assert(N == 32 || N == 64, "chunks of 32 or 64 keys");
+  const unsigned full = 0xffffffffu;
+  const int c = __shfl_sync(full, rc.cnt, src);
+  float th = __shfl_sync(full, rc.thr, src);
+  float fl = __shfl_sync(full, rc.floor_, src);
+  const float mm = __shfl_sync(full, rc.m, src);
+  const bool have = lane < c;
+  const float vo = have ? cs.s[lane * kCols + col_src] : -INFINITY;
+  const uint16_t ko = have ? cs.kt[lane * kCols + col_src] : static_cast<uint16_t>(0);
+  float vn0 = -INFINITY, vn1 = -INFINITY;  // src's values lane and 32 + lane
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float t = __shfl_sync(full, x[i], src);
+    if (lane == (i & 31)) {
+      if (i < 32) vn0 = t;
+      else vn1 = t;
+    }
+  }
+  unsigned bo = __ballot_sync(full, vo > th);
+  unsigned b0 = __ballot_sync(full, vn0 > th);
+  unsigned b1 = __ballot_sync(full, vn1 > th);
+  for (int guard = 0; guard < 12 && __popc(bo) + __popc(b0) + __popc(b1) > kCand; ++guard) {
+    fl = th + 0.5f * (mm - th);
+    th = fl;
+    bo = __ballot_sync(full, vo > th);
+    b0 = __ballot_sync(full, vn0 > th);
+    b1 = __ballot_sync(full, vn1 > th);
+  }
+  const unsigned below = (1u << lane) - 1u;
+  const int no = __popc(bo), n0 = __popc(b0), n1 = __popc(b1);
+  __syncwarp();
+  if ((bo >> lane) & 1u) {
+    const int at = __popc(bo & below);
+    cs.s[at * kCols + col_src] = vo;
+    cs.kt[at * kCols + col_src] = ko;
+  }
+  if ((b0 >> lane) & 1u) {
+    const int at = no + __popc(b0 & below);
+    if (at < kCand) {
+      cs.s[at * kCols + col_src] = vn0;
+      cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
+    }
+  }
+  if ((b1 >> lane) & 1u) {
+    const int at = no + n0 + __popc(b1 & below);
+    if (at < kCand) {
+      cs.s[at * kCols + col_src] = vn1;
+      cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
+    }
+  }
+  __syncwarp();
+  if (lane == src) {
+    const int total = no + n0 + n1;
+    rc.cnt = min(total, kCand);
+    if (total > kCand) rc.lost = 1;  // only when 12 halvings could not separate the values
+    rc.thr = th;
+    rc.floor_ = fl;
+  }
+}
+
+// Feeds N raw scores of key tile kt (keys outside the row's range already -inf) for the 32
+// (row, segment) columns of a warp; every lane of the warp must call it together.  The hot path
+// is the max of each 16-key block; only when a lane's block max passes its threshold does that
+// lane count and insert its passing values -- through the cooperative insertion above when its
+// buffer lacks room.
+template <int N>
+__device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, int lane,
+                                          const float (&x)[N], int kt) {
+  static_assert(N % 16 == 0, "16-key blocks");
+  constexpr int NB = N / 16;
+  const unsigned full = 0xffffffffu;
+  float sub[NB];
+#pragma unroll
+  for (int k = 0; k < NB; ++k) sub[k] = max16(x, 16 * k);
+  float cmax = sub[0];
+#pragma unroll
+  for (int k = 1; k < NB; ++k) cmax = fmaxf(cmax, sub[k]);
+  bool pass = cmax > rc.thr;
+  if (!__any_sync(full, pass)) return;
+  int incoming = 0;
+  if (pass) {
+    if (cmax > rc.m) {
+      rc.m = cmax;
+      rc.thr = fmaxf(rc.m - rc.inv_c, rc.floor_);
+    }
+#pragma unroll
+    for (int k = 0; k < NB; ++k)
+      if (sub[k] > rc.thr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) incoming += (x[16 * k + i] > rc.thr) ? 1 : 0;
+      }
+  }
+  const unsigned need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
+  for (unsigned rest = need; rest; rest &= rest - 1u) {
+    const int src = __ffs(rest) - 1;
+    coop_insert<N>(cs, rc, src, col - lane + src, x, kt, lane);
+  }
+  if (pass && !((need >> lane) & 1u)) {
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      if (sub[k] > rc.thr) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float v = x[16 * k + i];
+          if (v > rc.thr) {
+            cs.s[rc.cnt * kCols + col] = v;
+            cs.kt[rc.cnt * kCols + col] = static_cast<uint16_t>(kt);
+            ++rc.cnt;
+          }
+        }
+      }
+    }
+  }
+}
 
 // Solves tau for every row of the tile from the published candidate buffers of both segments,
 // writes tau and sets the tile's mask words in shared memory.  Rows are handled by groups of 4

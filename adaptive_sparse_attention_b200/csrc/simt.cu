@@ -134,8 +134,8 @@ __global__ void __launch_bounds__(kThreads) tau_simt_kernel(Problem P) {
     float x[kChunk];
 #pragma unroll
     for (int jj = 0; jj < kChunk; ++jj) x[jj] = sm.xs[jj * kTile + tid];
-    if ((chunk++ & 2) == 0) rc0.feed<kChunk>(cs, tid, x, kt);
-    else rc1.feed<kChunk>(cs, kTile + tid, x, kt);
+    if ((chunk++ & 2) == 0) feed_warp<kChunk>(rc0, cs, tid, tid & 31, x, kt);
+    else feed_warp<kChunk>(rc1, cs, kTile + tid, tid & 31, x, kt);
   });
   rc0.publish(cs, tid);
   rc1.publish(cs, kTile + tid);

@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     rc.init(1.f / P.c);
     for (int kt = 0; kt < nkt; ++kt) {
       const int b = kt & 1;
-      if (!mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort, P.status)) break;
+      // the warp leaves together: feed_warp needs all 32 lanes
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort, P.status)))
+        break;
       tc_fence_after();
       const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                           static_cast<uint32_t>(b * 128 + seg * 64);
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
-      rc.feed<64>(cs, col, x, kt);
+      feed_warp<64>(rc, cs, col, lane, x, kt);
     }
     rc.publish(cs, col);
   }
