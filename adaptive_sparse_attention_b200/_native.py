@@ -14,6 +14,7 @@ OK, EINVAL, EALIGN, ECUDA, ETIMEOUT, ENOMEM = 0, 1, 2, 3, 4, 5
 FP32, BF16 = 0, 1
 FLAG_CUDA_CORES = 1
 FLAG_ALL_FALLBACK = 2
+NOALLOC_SCRATCH_BYTES = 16 << 20  # ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES
 
 _c_int, _c_float, _c_size_t, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
 _c_uint = ctypes.c_uint
@@ -35,6 +36,9 @@ SIGNATURES = {
     "entmax_attn_fallback_tiles": (_c_int, [_vp, _vp]),
     "entmax_attn_status": (_c_int, [_vp]),
     "entmax_attn_release_workspaces": (None, []),
+    "entmax_attn_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                         _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
+                                         _vp]),
     "entmax_attn_strerror": (ctypes.c_char_p, [_c_int]),
     "entmax_attn_last_cuda_error": (ctypes.c_char_p, []),
 }

@@ -110,6 +110,25 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool 
     return out, tau, block_mask
 
 
+def entmax_attn_fwd_noalloc(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool = True,
+                            cu_seqlens=None, out=None, tau=None, block_mask=None, stream=None):
+    """Forward pass through the allocation-free entry point: the library's scratch is a fixed
+    device array (ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES), so the call allocates no device memory.
+    The outputs are allocated here by torch only when not passed in."""
+    _check_inputs(q, k, v, cu_seqlens)
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    o2, t2, m2 = alloc_outputs(q, k, cu_seqlens) if None in (out, tau, block_mask) else (None,) * 3
+    out = o2 if out is None else out
+    tau = t2 if tau is None else tau
+    block_mask = m2 if block_mask is None else block_mask
+    rc = N.lib().entmax_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(tau),
+                                         _ptr(block_mask), B, Hq, Hkv, T, d, float(alpha),
+                                         int(n_iter), int(bool(causal)), _ptr(cu_seqlens),
+                                         _DT[q.dtype], _stream(stream))
+    N.check(rc, "entmax_attn_fwd_noalloc")
+    return out, tau, block_mask
+
+
 def tau_pass(q, k, tau, block_mask, workspace, alpha=1.5, n_iter=10, causal=True,
              cu_seqlens=None, flags=0, stream=None):
     _check_inputs(q, k, None, cu_seqlens)

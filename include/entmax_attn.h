@@ -125,6 +125,28 @@ int entmax_attn_status(cudaStream_t stream);
 /* Frees the workspaces entmax_attn_fwd cached (synchronises the device first). */
 void entmax_attn_release_workspaces(void);
 
+/* Allocation-free forward pass.  The paper has no counterpart: this is a service for callers
+ * that cannot allocate device memory while they run -- code inside an allocator or memory-pool
+ * callback, where a nested cudaMalloc would recurse or deadlock; runtimes that forbid
+ * allocation after start-up to keep a fixed footprint; launch sequences replayed from a
+ * recording, where a first-use allocation would be an unrecorded side effect.
+ * Same arguments, outputs and semantics as entmax_attn_fwd, but the scratch memory lives in a
+ * file-scope device array of ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES that every GPU loading the
+ * library holds until the process exits; the call allocates and frees nothing.
+ *   - Problems whose scratch (entmax_attn_workspace_bytes) exceeds that size are rejected with
+ *     ENTMAX_ATTN_ENOMEM before anything is launched.
+ *   - The first call on a device, with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the array and it keeps the last call's contents (each call
+ *     rewrites everything it reads); calls that overlap on the GPU race on it, so serialise them
+ *     (one stream, or events). */
+#define ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* tau,
+                            uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d,
+                            float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
+                            int dtype, cudaStream_t stream);
+
 /* Static text for a return code. */
 const char* entmax_attn_strerror(int code);
 
