@@ -11,12 +11,15 @@
 //   then all 384 threads solve tau per row (4-lane groups) and warp 0 writes the block mask
 //   and the compact tile list.
 //
-// out_tc_kernel (one CTA of 256 threads per query tile, over the listed key tiles only):
-//   warp 0      TMA producer: query tile once, then (K, V) tile pairs through a 2-stage ring.
+// out_tc_kernel (one CTA of 384 threads per query tile, over the listed key tiles only):
+//   warp 0      TMA producer of the query tile and the key tiles (3-stage ring; a key tile is
+//               released as soon as its Q K^T product completes).
+//   warp 2      TMA producer of the value tiles (3-stage ring, released after its P V product).
 //   warp 1      tcgen05.mma: S = Q K^T into TMEM (double buffered), then O += P V with P read
 //               from TMEM as the A operand and V (MN-major in shared memory) as B.
-//   warps 4..7  p warps: load S, p = [c s - tau]_+^beta (0 off the causal / sequence range),
-//               store p as packed bf16 into TMEM; at the end read O from TMEM and store it.
+//   warps 4..11 p warps, two per TMEM lane quarter, each owning 64 keys of every tile: load S,
+//               p = [c s - tau]_+^beta (0 off the causal / sequence range), store p as packed
+//               bf16 into TMEM; at the end each reads half of O's columns from TMEM and stores them.
 // tau is known before this pass, so p needs neither a running max nor a final normalisation.
 //
 // Every mbarrier wait is bounded (about 2 s of %globaltimer): on expiry the waiting thread
@@ -37,11 +40,11 @@
 namespace ea {
 namespace {
 
-constexpr int kOutThreads = 256;
+constexpr int kOutThreads = 384;
 constexpr int kTauThreads = 384;
 constexpr int kScoreWarp0 = 4;            // score / p warps start at warp 4 (lane quarter w % 4)
 constexpr int kTauStages = 4;             // key tiles in flight in the tau pass
-constexpr int kOutStages = 2;             // (key, value) tile pairs in flight in the out pass
+constexpr int kOutStages = 3;             // key tiles and value tiles in flight in the out pass
 constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every mbarrier wait
 constexpr int kTimeoutCode = 4;           // ENTMAX_ATTN_ETIMEOUT
 
@@ -396,8 +399,10 @@ struct OutSmem {
   alignas(1024) __nv_bfloat16 k[kOutStages][kTile * D];
   alignas(1024) __nv_bfloat16 v[kOutStages][kTile * D];
   uint64_t q_full;
-  uint64_t kv_full[kOutStages];
-  uint64_t kv_empty[kOutStages];
+  uint64_t k_full[kOutStages];
+  uint64_t k_empty[kOutStages];
+  uint64_t v_full[kOutStages];
+  uint64_t v_empty[kOutStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t p_free[2];  // PV MMA that read P[b] has completed
@@ -432,12 +437,14 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < kOutStages; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.p_full[b], 4);
+      mbar_init(&sm.p_full[b], 8);  // one arrival per p warp
       mbar_init(&sm.p_free[b], 1);
     }
     mbar_init(&sm.o_full, 1);
@@ -450,29 +457,37 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2) {
     if (lane == 0) {
-      const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
+      // warp 0 streams Q and the key tiles, warp 2 the value tiles
+      const bool keys = warp == 0;
+      const CUtensorMap* map = keys ? &tmk : &tmv;
+      __nv_bfloat16(*ring)[kTile * D] = keys ? sm.k : sm.v;
+      uint64_t* full = keys ? sm.k_full : sm.v_full;
+      uint64_t* empty = keys ? sm.k_empty : sm.v_empty;
       const int krow0 = static_cast<int>(t.khead + t.seq_start);
-      mbar_expect_tx(&sm.q_full, kTileBytes);
-      for (int h = 0; h < D / 64; ++h) tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
+      if (keys) {
+        const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
+        mbar_expect_tx(&sm.q_full, kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
+      }
       int issued = 0;
       for (int i = 0; i < cnt; ++i) {
         const int s = i % kOutStages;
         if (i >= kOutStages &&
-            !mbar_wait(&sm.kv_empty[s], ((i / kOutStages) - 1) & 1, abort, P.status))
+            !mbar_wait(&empty[s], ((i / kOutStages) - 1) & 1, abort, P.status))
           break;
         const int row = krow0 + clamp_kt(list[i], t.nkt) * kTile;
-        mbar_expect_tx(&sm.kv_full[s], 2 * kTileBytes);
-        for (int h = 0; h < D / 64; ++h) {
-          tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.kv_full[s], h * 64, row);
-          tma_load_2d(sm.v[s] + h * kTile * 64, &tmv, &sm.kv_full[s], h * 64, row);
-        }
+        mbar_expect_tx(&full[s], kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_2d(ring[s] + h * kTile * 64, map, &full[s], h * 64, row);
         issued = i + 1;
       }
+      // drain: every issued copy has landed before the CTA may exit
       for (int i = (issued > kOutStages ? issued - kOutStages : 0); i < issued; ++i)
-        mbar_wait(&sm.kv_full[i % kOutStages], (i / kOutStages) & 1, abort, P.status);
-      mbar_wait(&sm.q_full, 0, abort, P.status);
+        mbar_wait(&full[i % kOutStages], (i / kOutStages) & 1, abort, P.status);
+      if (keys) mbar_wait(&sm.q_full, 0, abort, P.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -483,7 +498,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       // S(i) = Q K(i)^T into S[i & 1]
       auto issue_s = [&](int i) -> bool {
         const int s = i % kOutStages, b = i & 1;
-        if (!mbar_wait(&sm.kv_full[s], (i / kOutStages) & 1, abort, P.status)) return false;
+        if (!mbar_wait(&sm.k_full[s], (i / kOutStages) & 1, abort, P.status)) return false;
         // S[b] is free once the p warps have read S(i-2): they signal that through p_full.
         if (i >= 2 && !mbar_wait(&sm.p_full[b], ((i >> 1) - 1) & 1, abort, P.status))
           return false;
@@ -493,6 +508,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         for (int k16 = 0; k16 < D / 16; ++k16)
           mma_ss(tmem + kColS + b * 128, kmajor_desc(qbase, kTile, k16),
                  kmajor_desc(kbase, kTile, k16), idesc_s, k16 > 0 ? 1u : 0u);
+        mma_commit(&sm.k_empty[s]);
         mma_commit(&sm.s_full[b]);
         return true;
       };
@@ -502,13 +518,14 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         const int s = i % kOutStages, b = i & 1;
         if (i + 1 < cnt && !issue_s(i + 1)) break;
         if (!mbar_wait(&sm.p_full[b], (i >> 1) & 1, abort, P.status)) break;
+        if (!mbar_wait(&sm.v_full[s], (i / kOutStages) & 1, abort, P.status)) break;
         tc_fence_after();
         const uint32_t vbase = smem_u32(sm.v[s]);
 #pragma unroll
         for (int k16 = 0; k16 < kTile / 16; ++k16)
           mma_ts(tmem + kColO, tmem + kColP + b * 64 + k16 * 8, value_desc(vbase, k16), idesc_o,
                  (i > 0 || k16 > 0) ? 1u : 0u);
-        mma_commit(&sm.kv_empty[s]);
+        mma_commit(&sm.v_empty[s]);
         mma_commit(&sm.p_free[b]);
         done = i + 1;
       }
@@ -516,7 +533,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       mma_commit(&sm.o_full);  // arrives once every MMA issued so far has completed
     }
   } else if (warp >= kScoreWarp0) {
-    const int quarter = warp - kScoreWarp0;
+    const int quarter = warp & 3;
+    const int half = (warp - kScoreWarp0) >> 2;  // keys 64 half .. 64 half + 63 of every tile
     const int r = quarter * 32 + lane;
     const bool row_ok = r < t.nrows;
     const int pos = t.row0 + r;
@@ -530,13 +548,14 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       // P[b] is free once the PV product of step i-2 has completed
       if (i >= 2 && !mbar_wait(&sm.p_free[b], ((i >> 1) - 1) & 1, abort, P.status)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int c0 = half * 64 + q2 * 32;  // S column == key offset in the tile
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + kColS + b * 128 + q4 * 32, u);
+        tmem_ld32(tmem + lane_off + kColS + b * 128 + c0, u);
         tmem_wait_ld();
         uint32_t pk[16];
-        const int j0 = kt * kTile + q4 * 32;
+        const int j0 = kt * kTile + c0;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float s0 = __uint_as_float(u[2 * e]), s1 = __uint_as_float(u[2 * e + 1]);
@@ -544,26 +563,27 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           const float p1 = (j0 + 2 * e + 1 < jmax) ? entmax_p<BK>(P.c * s1 - tau, P.beta) : 0.f;
           pk[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tmem + lane_off + kColP + b * 64 + q4 * 16, pk);
+        tmem_st16(tmem + lane_off + kColP + b * 64 + c0 / 2, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[b]);
     }
-    // epilogue: O rows from TMEM to global memory
+    // epilogue: this warp's half of O's columns, from TMEM to global memory
     const bool o_ok = mbar_wait(&sm.o_full, 0, abort, P.status);
     tc_fence_after();
+    constexpr int kHalfD = D / 2;
+    __nv_bfloat16* op =
+        static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D + half * kHalfD;
     if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (only after a failed tau pass)
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) +
-                                            (t.qhead + t.seq_start + pos) * D);
-      for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      uint4* dst = reinterpret_cast<uint4*>(op);
+      for (int e = 0; e < kHalfD / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
     } else if (o_ok && !*abort) {
-      __nv_bfloat16* op = static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < kHalfD; c0 += 32) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + kColO + c0, u);
+        tmem_ld32(tmem + lane_off + kColO + half * kHalfD + c0, u);
         tmem_wait_ld();
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(op + c0);
