@@ -149,6 +149,12 @@ struct Search {
     dx = dxold = hi - lo;
   }
 
+  // True once the last step moved tau by no more than rounding: later steps can then only move
+  // it by a few ulps.
+  __device__ __forceinline__ bool settled() const {
+    return dx <= 4.f * FLT_EPSILON * fmaxf(1.f, fabsf(tau));
+  }
+
   // One step, given the sums over the keys with z > tau of (z - tau)^beta, ^(beta-1) and
   // ^(beta-2): f = S0 - 1, f' = -beta S1, f'' = beta (beta - 1) S2.  The bracket is narrowed by
   // the sign of f.  The proposal is the Halley step when its denominator 2 f'^2 - f f'' is
@@ -164,7 +170,9 @@ struct Search {
     if (f > 0.f) lo = tau;
     else hi = tau;
     const float den = 2.f * f1 * f1 - f * f2;
-    float nt = (den > 0.f && den < INFINITY) ? tau - 2.f * f * f1 / den : tau - f / f1;
+    // the quotient is only a proposal (the bracket test below guards it): fast division
+    float nt = (den > 0.f && den < INFINITY) ? tau - __fdividef(2.f * f * f1, den)
+                                             : tau - __fdividef(f, f1);
     const float len = fabsf(nt - tau);
     const bool small = len <= 4.f * FLT_EPSILON * fmaxf(1.f, fabsf(tau));
     if (!(nt >= lo && nt <= hi && (small || len <= 0.5f * dxold))) nt = 0.5f * (lo + hi);
@@ -405,6 +413,7 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
         s2 += __shfl_xor_sync(0xffffffffu, s2, o);
       }
       sr.step<BK>(s0, s1, s2, P.beta);
+      if (__all_sync(0xffffffffu, sr.settled())) break;  // every row of the warp has converged
     }
     const float tau = sr.tau;
     if (!valid) continue;

@@ -4,7 +4,8 @@
 //   warp 0      TMA producer: the query tile once, then the tile's key tiles through a
 //               kStages-deep shared-memory ring (128B-swizzled, K-major).
 //   warp 1      allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
-//               K = d, fp32 accumulators) into one of two TMEM score buffers.
+//               K = d, fp32 accumulators) into one of four TMEM score buffers, so that the
+//               score warps can fall up to three tiles behind during a burst of insertions.
 //   warps 4..11 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
 //               columns 64 s .. 64 s + 63 with s = (w - 4) / 4, i.e. one 64-key segment of every
 //               key tile, into the segment's running max and candidate buffer (common.cuh).
@@ -44,6 +45,7 @@ constexpr int kOutThreads = 384;
 constexpr int kTauThreads = 384;
 constexpr int kScoreWarp0 = 4;            // score / p warps start at warp 4 (lane quarter w % 4)
 constexpr int kTauStages = 4;             // key tiles in flight in the tau pass
+constexpr int kTauSBufs = 4;              // TMEM score buffers of the tau pass (128 columns each)
 constexpr int kOutStages = 3;             // key tiles and value tiles in flight in the out pass
 constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every mbarrier wait
 constexpr int kTimeoutCode = 4;           // ENTMAX_ATTN_ETIMEOUT
@@ -257,8 +259,8 @@ struct TauSmem {
   uint64_t q_full;
   uint64_t k_full[kTauStages];
   uint64_t k_empty[kTauStages];
-  uint64_t s_full[2];
-  uint64_t s_empty[2];
+  uint64_t s_full[kTauSBufs];
+  uint64_t s_empty[kTauSBufs];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kTauSBufs; ++b) {
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.s_empty[b], 8);  // one arrival per score warp
     }
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
-  if (warp == 1) tmem_alloc(&sm.tmem_base, 256);
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 128 * kTauSBufs);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -337,9 +339,11 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
       int issued = 0;
       for (int kt = 0; ok && kt < nkt; ++kt) {
-        const int s = kt % kTauStages, b = kt & 1;
+        const int s = kt % kTauStages, b = kt % kTauSBufs;
         if (!mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status)) break;
-        if (kt >= 2 && !mbar_wait(&sm.s_empty[b], ((kt >> 1) - 1) & 1, abort, P.status)) break;
+        if (kt >= kTauSBufs &&
+            !mbar_wait(&sm.s_empty[b], ((kt / kTauSBufs) - 1) & 1, abort, P.status))
+          break;
         tc_fence_after();
         const uint32_t kbase = smem_u32(sm.k[s]);
         const uint32_t dcol = tmem + static_cast<uint32_t>(b * 128);
@@ -365,9 +369,10 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     RowCand rc;
     rc.init(1.f / P.c);
     for (int kt = 0; kt < nkt; ++kt) {
-      const int b = kt & 1;
+      const int b = kt % kTauSBufs;
       // the warp leaves together: feed_warp needs all 32 lanes
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (kt >> 1) & 1, abort, P.status)))
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&sm.s_full[b], (kt / kTauSBufs) & 1, abort, P.status)))
         break;
       tc_fence_after();
       const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 128 * kTauSBufs);
   if (*abort) return;  // status already records the timeout; outputs of this tile are void
   solve_rows<BK>(P, t, cs, tid, kTauThreads);
   __syncthreads();
