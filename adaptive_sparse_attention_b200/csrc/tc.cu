@@ -1,11 +1,13 @@
 // tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16, sm_100a.
 //
 // tau_tc_kernel (one CTA of 384 threads per 128-row query tile):
-//   warp 0      TMA producer: the query tile once, then the tile's key tiles through a
-//               kStages-deep shared-memory ring (128B-swizzled, K-major).
+//   warp 0      TMA producer: the tile's key tiles through a kTauStages-deep shared-memory ring
+//               (128B-swizzled, K-major).
 //   warp 1      allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
-//               K = d, fp32 accumulators) into one of four TMEM score buffers, so that the
-//               score warps can fall up to three tiles behind during a burst of insertions.
+//               K = d, fp32 accumulators) into one of three TMEM score buffers, so that the
+//               score warps can fall up to two tiles behind during a burst of insertions.  Q is
+//               the A operand from TMEM (the score warps store it there once), which halves the
+//               MMA's shared-memory reads; shared memory then carries only the K tiles.
 //   warps 4..11 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
 //               columns 64 s .. 64 s + 63 with s = (w - 4) / 4, i.e. one 64-key segment of every
 //               key tile, into the segment's running max and candidate buffer (common.cuh).
@@ -44,8 +46,11 @@ namespace {
 constexpr int kOutThreads = 384;
 constexpr int kTauThreads = 384;
 constexpr int kScoreWarp0 = 4;            // score / p warps start at warp 4 (lane quarter w % 4)
-constexpr int kTauStages = 4;             // key tiles in flight in the tau pass
-constexpr int kTauSBufs = 4;              // TMEM score buffers of the tau pass (128 columns each)
+constexpr int kTauStages = 5;             // key tiles in flight in the tau pass
+constexpr int kTauSBufs = 3;              // TMEM score buffers of the tau pass (128 columns each)
+constexpr uint32_t kTauColQ = 128 * kTauSBufs;  // TMEM columns of the query tile (A operand)
+constexpr uint32_t kTauTmemCols = 512;          // allocation (a power of two >= 32)
+static_assert(kTauColQ + 128 / 2 <= kTauTmemCols, "score buffers + Q (d <= 128) fit in TMEM");
 constexpr int kOutStages = 3;             // key tiles and value tiles in flight in the out pass
 constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every mbarrier wait
 constexpr int kTimeoutCode = 4;           // ENTMAX_ATTN_ETIMEOUT
@@ -253,7 +258,6 @@ __device__ __forceinline__ void tmem_row64(uint32_t ta, int j0, int jmax, float 
 
 template <int D>
 struct TauSmem {
-  alignas(1024) __nv_bfloat16 q[kTile * D];
   alignas(1024) __nv_bfloat16 k[kTauStages][kTile * D];
   CandSmem cand;
   uint64_t q_full;
@@ -268,8 +272,7 @@ struct TauSmem {
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kTauThreads, 1)
-    tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  Problem P) {
+    tau_tc_kernel(const __grid_constant__ CUtensorMap tmk, Problem P) {
   extern __shared__ unsigned char smem_raw[];
   TauSmem<D>& sm = *reinterpret_cast<TauSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   constexpr uint32_t kTileBytes = kTile * D * 2;
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_full, 8);  // one arrival per score warp once its part of Q is in TMEM
     for (int s = 0; s < kTauStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -301,7 +304,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
-  if (warp == 1) tmem_alloc(&sm.tmem_base, 128 * kTauSBufs);
+  if (warp == 1) tmem_alloc(&sm.tmem_base, kTauTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -310,10 +313,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
       const int krow0 = static_cast<int>(t.khead + t.seq_start);
-      mbar_expect_tx(&sm.q_full, kTileBytes);
-      for (int h = 0; h < D / 64; ++h) tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
       int issued = 0;
       for (int kt = 0; kt < nkt; ++kt) {
         const int s = kt % kTauStages;
@@ -330,12 +330,10 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         const int s = kt % kTauStages;
         mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status);
       }
-      mbar_wait(&sm.q_full, 0, abort, P.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
-      const uint32_t qbase = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
       int issued = 0;
       for (int kt = 0; ok && kt < nkt; ++kt) {
@@ -348,8 +346,8 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         const uint32_t kbase = smem_u32(sm.k[s]);
         const uint32_t dcol = tmem + static_cast<uint32_t>(b * 128);
 #pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16)
-          mma_ss(dcol, kmajor_desc(qbase, kTile, k16), kmajor_desc(kbase, kTile, k16), idesc,
+        for (int k16 = 0; k16 < D / 16; ++k16)  // A = Q from TMEM: 16 columns of d = 8 TMEM columns
+          mma_ts(dcol, tmem + kTauColQ + k16 * 8, kmajor_desc(kbase, kTile, k16), idesc,
                  k16 > 0 ? 1u : 0u);
         mma_commit(&sm.k_empty[s]);
         mma_commit(&sm.s_full[b]);
@@ -366,6 +364,39 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     const int r = quarter * 32 + lane;  // query row of the tile == TMEM lane
     const int col = seg * kTile + r;
     const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+    {  // this thread's half of its query row into TMEM (columns = packed bf16 pairs of d)
+      constexpr int kWords = D / 4;  // 32-bit columns per half row
+      uint32_t w[kWords];
+      if (r < t.nrows) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            static_cast<const __nv_bfloat16*>(P.q) + (t.qhead + t.seq_start + t.row0 + r) * D +
+            seg * (D / 2));
+#pragma unroll
+        for (int i = 0; i < kWords / 4; ++i) {
+          const uint4 u = src[i];
+          w[4 * i] = u.x;
+          w[4 * i + 1] = u.y;
+          w[4 * i + 2] = u.z;
+          w[4 * i + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) w[i] = 0u;
+      }
+      const uint32_t qa = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTauColQ +
+                          static_cast<uint32_t>(seg * kWords);
+#pragma unroll
+      for (int i = 0; i < kWords; i += 16) {
+        uint32_t part[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) part[e] = w[i + e];
+        tmem_st16(qa + i, part);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full);
+    }
     RowCand rc;
     rc.init(1.f / P.c);
     for (int kt = 0; kt < nkt; ++kt) {
@@ -389,7 +420,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 128 * kTauSBufs);
+  if (warp == 1) tmem_dealloc(tmem, kTauTmemCols);
   if (*abort) return;  // status already records the timeout; outputs of this tile are void
   solve_rows<BK>(P, t, cs, tid, kTauThreads);
   __syncthreads();
@@ -648,15 +679,14 @@ dim3 tile_grid(const Problem& P) { return dim3(P.slots, P.Hq, P.cu ? 1 : P.B); }
 
 template <int D, int BK>
 cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
-  CUtensorMap mq, mk;
-  cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
-  if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
+  CUtensorMap mk;
+  cudaError_t e = make_map(&mk, P.k, kv_rows(P), D);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(TauSmem<D>) + 1024;
   auto kern = tau_tc_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<tile_grid(P), kTauThreads, smem, s>>>(mq, mk, P);
+  kern<<<tile_grid(P), kTauThreads, smem, s>>>(mk, P);
   return cudaGetLastError();
 }
 
