@@ -192,6 +192,7 @@ struct Search {
 struct CandSmem {
   float s[kCand * kCols];
   uint16_t kt[kCand * kCols];
+  float rowmax[kTile];  // running max of the row over all segments (raw); see feed_warp
   float m[kCols];       // segment max of raw scores
   float floor_[kCols];  // pruning floor (raw); -inf when the segment was never pruned
   int cnt[kCols];
@@ -220,8 +221,9 @@ __device__ __forceinline__ float max16(const float (&x)[N], int o) {
 
 // Candidate state of one (row, segment), held in registers by the thread that owns it.
 struct RowCand {
-  float m;       // running max of raw scores
-  float thr;     // keep threshold: max(m - 1/c, floor)
+  float m;       // running max of this segment's raw scores
+  float mx;      // largest max known for the row: max(m, what other segments published)
+  float thr;     // keep threshold: max(mx - 1/c, floor)
   float floor_;  // pruning floor, -inf if never raised
   float inv_c;   // 1 / c
   int cnt;
@@ -229,6 +231,7 @@ struct RowCand {
 
   __device__ __forceinline__ void init(float inv_c_) {
     m = -INFINITY;
+    mx = -INFINITY;
     thr = -INFINITY;
     floor_ = -INFINITY;
     inv_c = inv_c_;
@@ -261,7 +264,7 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   const int c = __shfl_sync(full, rc.cnt, src);
   float th = __shfl_sync(full, rc.thr, src);
   float fl = __shfl_sync(full, rc.floor_, src);
-  const float mm = __shfl_sync(full, rc.m, src);
+  const float mm = __shfl_sync(full, rc.mx, src);
   const bool have = lane < c;
   const float vo = have ? cs.s[lane * kCols + col_src] : -INFINITY;
   const uint16_t ko = have ? cs.kt[lane * kCols + col_src] : static_cast<uint16_t>(0);
@@ -320,9 +323,12 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
 // (row, segment) columns of a warp; every lane of the warp must call it together.  The hot path
 // is the max of each 16-key block; only when a lane's block max passes its threshold does that
 // lane count and insert its passing values -- through the cooperative insertion above when its
-// buffer lacks room.
+// buffer lacks room.  The threshold uses the largest max any segment of the row has published
+// in cs.rowmax[row]: a lower bound of the row's max, so every key with z > (row max) - 1 is
+// still kept, while records of one segment's max no longer trigger insertions in the others.
+// A stale or overwritten rowmax value only loosens the threshold.
 template <int N>
-__device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, int lane,
+__device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, int row, int lane,
                                           const float (&x)[N], int kt) {
   static_assert(N % 16 == 0, "16-key blocks");
   constexpr int NB = N / 16;
@@ -333,13 +339,20 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, in
   float cmax = sub[0];
 #pragma unroll
   for (int k = 1; k < NB; ++k) cmax = fmaxf(cmax, sub[k]);
+  const float shared_max = *reinterpret_cast<volatile float*>(&cs.rowmax[row]);
+  if (shared_max > rc.mx) {
+    rc.mx = shared_max;
+    rc.thr = fmaxf(rc.mx - rc.inv_c, rc.floor_);
+  }
   bool pass = cmax > rc.thr;
   if (!__any_sync(full, pass)) return;
   int incoming = 0;
   if (pass) {
-    if (cmax > rc.m) {
-      rc.m = cmax;
-      rc.thr = fmaxf(rc.m - rc.inv_c, rc.floor_);
+    rc.m = fmaxf(rc.m, cmax);
+    if (cmax > rc.mx) {
+      rc.mx = cmax;
+      rc.thr = fmaxf(rc.mx - rc.inv_c, rc.floor_);
+      cs.rowmax[row] = cmax;  // publish to the row's other segments
     }
 #pragma unroll
     for (int k = 0; k < NB; ++k)

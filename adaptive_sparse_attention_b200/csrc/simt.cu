@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(kThreads) tau_simt_kernel(Problem P) {
     return;
   }
   for (int w = tid; w < kMaxWords; w += kThreads) cs.words[w] = 0u;
+  cs.rowmax[tid] = -INFINITY;  // kThreads == kTile: thread tid owns row tid
   if (tid == 0) cs.fallback = P.force_fallback;
   load_q_tile<T, D>(P, t, sm.qs, tid);
 
@@ -134,8 +135,8 @@ __global__ void __launch_bounds__(kThreads) tau_simt_kernel(Problem P) {
     float x[kChunk];
 #pragma unroll
     for (int jj = 0; jj < kChunk; ++jj) x[jj] = sm.xs[jj * kTile + tid];
-    if ((chunk++ & 2) == 0) feed_warp<kChunk>(rc0, cs, tid, tid & 31, x, kt);
-    else feed_warp<kChunk>(rc1, cs, kTile + tid, tid & 31, x, kt);
+    if ((chunk++ & 2) == 0) feed_warp<kChunk>(rc0, cs, tid, tid, tid & 31, x, kt);
+    else feed_warp<kChunk>(rc1, cs, kTile + tid, tid, tid & 31, x, kt);
   });
   rc0.publish(cs, tid);
   rc1.publish(cs, kTile + tid);

@@ -304,6 +304,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
+  for (int r = tid; r < kTile; r += kTauThreads) cs.rowmax[r] = -INFINITY;
   if (warp == 1) tmem_alloc(&sm.tmem_base, kTauTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -413,7 +414,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
-      feed_warp<64>(rc, cs, col, lane, x, kt);
+      feed_warp<64>(rc, cs, col, r, lane, x, kt);
     }
     rc.publish(cs, col);
   }
