@@ -19,9 +19,9 @@
 namespace ea {
 
 constexpr int kTile = 128;      // query-tile rows and key-tile keys (block-mask granularity)
-constexpr int kSeg = 2;         // key segments per row (keys 0-63 / 64-127 of every key tile),
+constexpr int kSeg = 4;         // key segments per row (keys 32 g .. 32 g + 31 of every key tile),
                                 // each with its own running max and candidate buffer
-constexpr int kCand = 32;       // candidate slots per (row, segment) held in shared memory
+constexpr int kCand = 16;       // candidate slots per (row, segment) held in shared memory
 constexpr int kCols = kSeg * kTile;  // (row, segment) columns of the candidate buffers
 constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
 
@@ -184,10 +184,9 @@ struct Search {
 
 // ---------------------------------------------------------------------------------------------
 // Candidate buffers: for every (row r, segment g) -- column c = g * 128 + r -- up to kCand
-// (raw score, key tile) pairs in shared memory, entry e at [e * 256 + c], so that the 32 rows of
-// a warp hit 32 distinct banks whatever their fill levels.  A segment owns the keys 64 g .. 64 g
-// + 63 of every key tile; its running max is a max over those keys only, which keeps a superset
-// of the row's candidates (its threshold is never above the row's).
+// (raw score, key tile) pairs in shared memory, entry e at [e * kCols + c], so that the 32 rows
+// of a warp hit 32 distinct banks whatever their fill levels.  A segment owns the keys 32 g ..
+// 32 g + 31 of every key tile.
 // ---------------------------------------------------------------------------------------------
 struct CandSmem {
   float s[kCand * kCols];
@@ -247,11 +246,11 @@ struct RowCand {
   }
 };
 
-static_assert(kCand == 32, "one candidate slot per lane in the warp-cooperative compaction");
+static_assert(kCand <= 32, "at most one candidate slot per lane in the cooperative insertion");
 
 // Warp-cooperative insertion for lane src (buffer column col_src) when its buffer cannot take
-// all of its passing values: lane e holds old entry e, and lanes e and e + 32 of src's chunk x
-// are spread over the warp by shuffles.  Old entries and new values at or below the threshold
+// all of its passing values: lane e < kCand holds old entry e, and values e and e + 32 of src's
+// chunk x are spread over the warp by shuffles.  Old entries and new values at or below the threshold
 // are dropped; while more than kCand survive, the floor is raised halfway to the running max
 // (entries below the floor can only matter if tau ends up at or below it, which the solve
 // checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
@@ -398,9 +397,14 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
   // whole warp); rows past the end of the tile run on an empty candidate list and store nothing.
   for (int r = tid >> 2; r < kTile; r += groups) {
     const bool valid = r < t.nrows;
-    const int cnt0 = valid ? cs.cnt[r] : 0;
-    const int cnt = valid ? cnt0 + cs.cnt[kTile + r] : 0;
-    const float mz = valid ? P.c * fmaxf(cs.m[r], cs.m[kTile + r]) : 0.f;
+    int cnt[kSeg];
+    float mraw = -INFINITY;
+#pragma unroll
+    for (int g = 0; g < kSeg; ++g) {
+      cnt[g] = valid ? cs.cnt[g * kTile + r] : 0;
+      mraw = fmaxf(mraw, cs.m[g * kTile + r]);
+    }
+    const float mz = valid ? P.c * mraw : 0.f;
     const int pos = t.row0 + r;
     const int n = valid ? (P.causal ? pos + 1 : t.seq_len) : 1;
     Search sr;
@@ -408,15 +412,17 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     for (int it = 0; it < P.n_iter; ++it) {
       const float tau = sr.tau;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f;
-      for (int e = lane4; e < cnt; e += 4) {
-        const int idx = (e < cnt0) ? e * kCols + r : (e - cnt0) * kCols + kTile + r;
-        const float x = P.c * cs.s[idx] - tau;
-        if (x > 0.f) {
-          float a, b, c2;
-          entmax_powers<BK>(x, P.beta, a, b, c2);
-          s0 += a;
-          s1 += b;
-          s2 += c2;
+#pragma unroll
+      for (int g = 0; g < kSeg; ++g) {
+        for (int e = lane4; e < cnt[g]; e += 4) {
+          const float x = P.c * cs.s[e * kCols + g * kTile + r] - tau;
+          if (x > 0.f) {
+            float a, b, c2;
+            entmax_powers<BK>(x, P.beta, a, b, c2);
+            s0 += a;
+            s1 += b;
+            s2 += c2;
+          }
         }
       }
 #pragma unroll
@@ -431,18 +437,21 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     const float tau = sr.tau;
     if (!valid) continue;
     if (lane4 == 0) P.tau[t.qhead + t.seq_start + pos] = tau;
-    bool bad = cs.lost[r] || cs.lost[kTile + r];
+    bool bad = false;
 #pragma unroll
     for (int g = 0; g < kSeg; ++g) {
       const float fl = cs.floor_[g * kTile + r];
-      if (fl > -INFINITY && !(tau > P.c * fl)) bad = true;
+      if (cs.lost[g * kTile + r] || (fl > -INFINITY && !(tau > P.c * fl))) bad = true;
     }
     if (bad) cs.fallback = 1;
-    for (int e = lane4; e < cnt; e += 4) {
-      const int idx = (e < cnt0) ? e * kCols + r : (e - cnt0) * kCols + kTile + r;
-      if (P.c * cs.s[idx] > tau) {
-        const int kt = cs.kt[idx];
-        atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
+#pragma unroll
+    for (int g = 0; g < kSeg; ++g) {
+      for (int e = lane4; e < cnt[g]; e += 4) {
+        const int idx = e * kCols + g * kTile + r;
+        if (P.c * cs.s[idx] > tau) {
+          const int kt = cs.kt[idx];
+          atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
+        }
       }
     }
   }

@@ -126,20 +126,29 @@ __global__ void __launch_bounds__(kThreads) tau_simt_kernel(Problem P) {
   if (tid == 0) cs.fallback = P.force_fallback;
   load_q_tile<T, D>(P, t, sm.qs, tid);
 
-  // chunks 0-1 of a key tile are keys 0-63 (segment 0), chunks 2-3 keys 64-127 (segment 1)
-  RowCand rc0, rc1;
+  // chunk g (keys 32 g .. 32 g + 31) of every key tile is segment g
+  static_assert(kSeg * kChunk == kTile, "one 32-key chunk per segment");
+  RowCand rc0, rc1, rc2, rc3;
   rc0.init(1.f / P.c);
   rc1.init(1.f / P.c);
+  rc2.init(1.f / P.c);
+  rc3.init(1.f / P.c);
   int chunk = 0;
   sweep_keys<T, D>(P, t, sm, tid, [&](int kt) {
     float x[kChunk];
 #pragma unroll
     for (int jj = 0; jj < kChunk; ++jj) x[jj] = sm.xs[jj * kTile + tid];
-    if ((chunk++ & 2) == 0) feed_warp<kChunk>(rc0, cs, tid, tid, tid & 31, x, kt);
-    else feed_warp<kChunk>(rc1, cs, kTile + tid, tid, tid & 31, x, kt);
+    switch (chunk++ & 3) {  // uniform across the block
+      case 0: feed_warp<kChunk>(rc0, cs, tid, tid, tid & 31, x, kt); break;
+      case 1: feed_warp<kChunk>(rc1, cs, kTile + tid, tid, tid & 31, x, kt); break;
+      case 2: feed_warp<kChunk>(rc2, cs, 2 * kTile + tid, tid, tid & 31, x, kt); break;
+      default: feed_warp<kChunk>(rc3, cs, 3 * kTile + tid, tid, tid & 31, x, kt); break;
+    }
   });
   rc0.publish(cs, tid);
   rc1.publish(cs, kTile + tid);
+  rc2.publish(cs, 2 * kTile + tid);
+  rc3.publish(cs, 3 * kTile + tid);
   __syncthreads();
   solve_rows<BK>(P, t, cs, tid, kThreads);
   __syncthreads();

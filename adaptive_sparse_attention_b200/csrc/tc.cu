@@ -1,17 +1,18 @@
 // tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16, sm_100a.
 //
-// tau_tc_kernel (one CTA of 384 threads per 128-row query tile):
-//   warp 0      TMA producer: the tile's key tiles through a kTauStages-deep shared-memory ring
+// tau_tc_kernel (one CTA of 576 threads per 128-row query tile):
+//   warp 16     TMA producer: the tile's key tiles through a kTauStages-deep shared-memory ring
 //               (128B-swizzled, K-major).
-//   warp 1      allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
+//   warp 17     allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
 //               K = d, fp32 accumulators) into one of three TMEM score buffers, so that the
 //               score warps can fall up to two tiles behind during a burst of insertions.  Q is
 //               the A operand from TMEM (the score warps store it there once), which halves the
 //               MMA's shared-memory reads; shared memory then carries only the K tiles.
-//   warps 4..11 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
-//               columns 64 s .. 64 s + 63 with s = (w - 4) / 4, i.e. one 64-key segment of every
-//               key tile, into the segment's running max and candidate buffer (common.cuh).
-//   then all 384 threads solve tau per row (4-lane groups) and warp 0 writes the block mask
+//   warps 0..15 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
+//               columns 32 g .. 32 g + 31 with g = w / 4, i.e. one 32-key segment of every key
+//               tile, into the segment's candidate buffer (common.cuh); the four segments of a
+//               row share its running max.
+//   then the score warps solve tau per row (4-lane groups) and warp 0 writes the block mask
 //   and the compact tile list.
 //
 // out_tc_kernel (one CTA of 384 threads per query tile, over the listed key tiles only):
@@ -44,8 +45,11 @@ namespace ea {
 namespace {
 
 constexpr int kOutThreads = 384;
-constexpr int kTauThreads = 384;
-constexpr int kScoreWarp0 = 4;            // score / p warps start at warp 4 (lane quarter w % 4)
+constexpr int kScoreWarp0 = 4;            // p warps of the out pass start at warp 4 (quarter w % 4)
+constexpr int kTauScoreWarps = 16;        // tau pass: warps 0..15 score, 16 TMA, 17 MMA
+constexpr int kTauTmaWarp = 16;
+constexpr int kTauMmaWarp = 17;
+constexpr int kTauThreads = 32 * (kTauScoreWarps + 2);
 constexpr int kTauStages = 5;             // key tiles in flight in the tau pass
 constexpr int kTauSBufs = 3;              // TMEM score buffers of the tau pass (128 columns each)
 constexpr uint32_t kTauColQ = 128 * kTauSBufs;  // TMEM columns of the query tile (A operand)
@@ -235,22 +239,33 @@ __device__ __forceinline__ uint64_t value_desc(uint32_t base, int k16) {
   return sw128_desc(base + static_cast<uint32_t>(k16) * 2048u, 128u * 128u, 1024u);
 }
 
-// 64 raw scores of this thread's row from TMEM columns [ta, ta + 64), keys j0 + i; keys at or
+// 32 raw scores of this thread's row from TMEM columns [ta, ta + 32), keys j0 + i; keys at or
 // past jmax (outside the row's causal / sequence range) read as -inf.
-__device__ __forceinline__ void tmem_row64(uint32_t ta, int j0, int jmax, float (&x)[64]) {
-  uint32_t u0[32], u1[32];
-  tmem_ld32(ta, u0);
-  tmem_ld32(ta + 32, u1);
+__device__ __forceinline__ void tmem_row32(uint32_t ta, int j0, int jmax, float (&x)[32]) {
+  uint32_t u[32];
+  tmem_ld32(ta, u);
   tmem_wait_ld();
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    x[i] = __uint_as_float(u0[i]);
-    x[32 + i] = __uint_as_float(u1[i]);
-  }
-  if (j0 + 64 > jmax) {  // diagonal or ragged tile
+  for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]);
+  if (j0 + 32 > jmax) {  // diagonal or ragged tile
 #pragma unroll
-    for (int i = 0; i < 64; ++i)
+    for (int i = 0; i < 32; ++i)
       if (j0 + i >= jmax) x[i] = -INFINITY;
+  }
+}
+
+// N (8 or 16) 32-bit words into N consecutive TMEM columns of this warp's lanes.
+template <int N>
+__device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&w)[N]) {
+  static_assert(N == 8 || N == 16, "8 or 16 columns");
+  if constexpr (N == 16) {
+    tmem_st16(taddr, w);
+  } else {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+            taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+        : "memory");
   }
 }
 
@@ -289,14 +304,14 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   constexpr uint32_t kTileBytes = kTile * D * 2;
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, 8);  // one arrival per score warp once its part of Q is in TMEM
+    mbar_init(&sm.q_full, kTauScoreWarps);  // each score warp stores its part of Q into TMEM
     for (int s = 0; s < kTauStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
     }
     for (int b = 0; b < kTauSBufs; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_empty[b], 8);  // one arrival per score warp
+      mbar_init(&sm.s_empty[b], kTauScoreWarps);  // one arrival per score warp
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -305,14 +320,14 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   }
   for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
   for (int r = tid; r < kTile; r += kTauThreads) cs.rowmax[r] = -INFINITY;
-  if (warp == 1) tmem_alloc(&sm.tmem_base, kTauTmemCols);
+  if (warp == kTauMmaWarp) tmem_alloc(&sm.tmem_base, kTauTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int nkt = t.nkt;
 
-  if (warp == 0) {
+  if (warp == kTauTmaWarp) {
     if (lane == 0) {
       const int krow0 = static_cast<int>(t.khead + t.seq_start);
       int issued = 0;
@@ -332,7 +347,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kTauMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
       bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
@@ -359,19 +374,19 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         mbar_wait(&sm.drain, 0, abort, P.status);
       }
     }
-  } else if (warp >= kScoreWarp0) {
+  } else {  // score warps 0..15
     const int quarter = warp & 3;
-    const int seg = (warp - kScoreWarp0) >> 2;
+    const int seg = warp >> 2;  // keys 32 seg .. 32 seg + 31 of every key tile
     const int r = quarter * 32 + lane;  // query row of the tile == TMEM lane
     const int col = seg * kTile + r;
     const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
-    {  // this thread's half of its query row into TMEM (columns = packed bf16 pairs of d)
-      constexpr int kWords = D / 4;  // 32-bit columns per half row
+    {  // this thread's quarter of its query row into TMEM (columns = packed bf16 pairs of d)
+      constexpr int kWords = D / 8;  // 32-bit columns per quarter row
       uint32_t w[kWords];
       if (r < t.nrows) {
         const uint4* src = reinterpret_cast<const uint4*>(
             static_cast<const __nv_bfloat16*>(P.q) + (t.qhead + t.seq_start + t.row0 + r) * D +
-            seg * (D / 2));
+            seg * (D / 4));
 #pragma unroll
         for (int i = 0; i < kWords / 4; ++i) {
           const uint4 u = src[i];
@@ -386,13 +401,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       }
       const uint32_t qa = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTauColQ +
                           static_cast<uint32_t>(seg * kWords);
-#pragma unroll
-      for (int i = 0; i < kWords; i += 16) {
-        uint32_t part[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) part[e] = w[i + e];
-        tmem_st16(qa + i, part);
-      }
+      tmem_st_words<kWords>(qa, w);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -408,22 +417,22 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         break;
       tc_fence_after();
       const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                          static_cast<uint32_t>(b * 128 + seg * 64);
-      float x[64];
-      tmem_row64(ta, kt * kTile + seg * 64, jmax, x);
+                          static_cast<uint32_t>(b * 128 + seg * 32);
+      float x[32];
+      tmem_row32(ta, kt * kTile + seg * 32, jmax, x);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
-      feed_warp<64>(rc, cs, col, r, lane, x, kt);
+      feed_warp<32>(rc, cs, col, r, lane, x, kt);
     }
     rc.publish(cs, col);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTauTmemCols);
+  if (warp == kTauMmaWarp) tmem_dealloc(tmem, kTauTmemCols);
   if (*abort) return;  // status already records the timeout; outputs of this tile are void
-  solve_rows<BK>(P, t, cs, tid, kTauThreads);
+  if (warp < kTauScoreWarps) solve_rows<BK>(P, t, cs, tid, 32 * kTauScoreWarps);
   __syncthreads();
   if (warp == 0) emit_tile(P, t, cs.words, cs.fallback, lane);
 }
