@@ -250,10 +250,10 @@ static_assert(kCand <= 32, "at most one candidate slot per lane in the cooperati
 
 // Warp-cooperative insertion for lane src (buffer column col_src) when its buffer cannot take
 // all of its passing values: lane e < kCand holds old entry e, and values e and e + 32 of src's
-// chunk x are spread over the warp by shuffles.  Old entries and new values at or below the threshold
-// are dropped; while more than kCand survive, the floor is raised halfway to the running max
-// (entries below the floor can only matter if tau ends up at or below it, which the solve
-// checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
+// chunk x are spread over the warp by shuffles.  Old entries and new values at or below the
+// threshold are dropped; if more than kCand survive, the floor is raised to the (kCand + 1)-th
+// largest value by bisection, so that the kCand largest survive (entries below the floor can
+// only matter if tau ends up at or below it, which the solve checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
 // of the buffer.  Call with the whole warp converged; x is read from lane src only.
 template <int N>
 __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, int col_src,
@@ -279,9 +279,25 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   unsigned bo = __ballot_sync(full, vo > th);
   unsigned b0 = __ballot_sync(full, vn0 > th);
   unsigned b1 = __ballot_sync(full, vn1 > th);
-  for (int guard = 0; guard < 12 && __popc(bo) + __popc(b0) + __popc(b1) > kCand; ++guard) {
-    fl = th + 0.5f * (mm - th);
-    th = fl;
+  if (__popc(bo) + __popc(b0) + __popc(b1) > kCand) {
+    // Raise the floor to (just above) the (kCand + 1)-th largest value: bisection on
+    // [th, mm] keeps "more than kCand above lo, at most kCand above hi".
+    float lo = th, hi = mm;
+    for (int it = 0; it < 24; ++it) {
+      const float mid = 0.5f * (lo + hi);
+      if (!(mid > lo && mid < hi)) break;  // the interval cannot shrink further in fp32
+      const int n = __popc(__ballot_sync(full, vo > mid)) +
+                    __popc(__ballot_sync(full, vn0 > mid)) +
+                    __popc(__ballot_sync(full, vn1 > mid));
+      if (n > kCand) {
+        lo = mid;
+      } else {
+        hi = mid;
+        if (n == kCand) break;  // exactly kCand survive: as high as the floor needs to go
+      }
+    }
+    fl = hi;
+    th = hi;
     bo = __ballot_sync(full, vo > th);
     b0 = __ballot_sync(full, vn0 > th);
     b1 = __ballot_sync(full, vn1 > th);
@@ -312,7 +328,7 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   if (lane == src) {
     const int total = no + n0 + n1;
     rc.cnt = min(total, kCand);
-    if (total > kCand) rc.lost = 1;  // only when 12 halvings could not separate the values
+    if (total > kCand) rc.lost = 1;  // only when ties at the floor could not be separated
     rc.thr = th;
     rc.floor_ = fl;
   }
