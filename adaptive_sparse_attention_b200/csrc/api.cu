@@ -219,8 +219,13 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
   e = use_tensor_cores(dtype, flags) ? ea::launch_tau_tc(P, stream)
                                      : ea::launch_tau_simt(P, dtype, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  const int64_t ctas = std::min<int64_t>(L.tiles, 2 * num_sms());
-  e = ea::launch_tau_fallback(P, dtype, static_cast<int>(ctas), stream);
+  if (use_tensor_cores(dtype, flags)) {
+    const int64_t ctas = std::min<int64_t>(L.tiles, num_sms());
+    e = ea::launch_tau_tc_fallback(P, static_cast<int>(ctas), stream);
+  } else {
+    const int64_t ctas = std::min<int64_t>(L.tiles, 2 * num_sms());
+    e = ea::launch_tau_fallback(P, dtype, static_cast<int>(ctas), stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e);
   return ENTMAX_ATTN_OK;
 }

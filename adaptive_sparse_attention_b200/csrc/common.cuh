@@ -251,9 +251,10 @@ static_assert(kCand <= 32, "at most one candidate slot per lane in the cooperati
 // Warp-cooperative insertion for lane src (buffer column col_src) when its buffer cannot take
 // all of its passing values: lane e < kCand holds old entry e, and values e and e + 32 of src's
 // chunk x are spread over the warp by shuffles.  Old entries and new values at or below the
-// threshold are dropped; if more than kCand survive, the floor is raised to the (kCand + 1)-th
-// largest value by bisection, so that the kCand largest survive (entries below the floor can
-// only matter if tau ends up at or below it, which the solve checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
+// threshold are dropped; if more than kCand survive, the floor is raised by bisection to just
+// above the (kCand/2 + 1)-th largest value, so that the kCand/2 largest survive and the buffer
+// has room again (entries below the floor can only matter if tau ends up at or below it, which
+// the solve checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
 // of the buffer.  Call with the whole warp converged; x is read from lane src only.
 template <int N>
 __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, int col_src,
@@ -280,8 +281,10 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   unsigned b0 = __ballot_sync(full, vn0 > th);
   unsigned b1 = __ballot_sync(full, vn1 > th);
   if (__popc(bo) + __popc(b0) + __popc(b1) > kCand) {
-    // Raise the floor to (just above) the (kCand + 1)-th largest value: bisection on
-    // [th, mm] keeps "more than kCand above lo, at most kCand above hi".
+    // Raise the floor to (just above) the (kKeep + 1)-th largest value, kKeep = kCand / 2, so
+    // that later passing values find room without another cooperative insertion: bisection on
+    // [th, mm] keeps "more than kKeep above lo, at most kKeep above hi".
+    constexpr int kKeep = kCand / 2;
     float lo = th, hi = mm;
     for (int it = 0; it < 24; ++it) {
       const float mid = 0.5f * (lo + hi);
@@ -289,11 +292,11 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
       const int n = __popc(__ballot_sync(full, vo > mid)) +
                     __popc(__ballot_sync(full, vn0 > mid)) +
                     __popc(__ballot_sync(full, vn1 > mid));
-      if (n > kCand) {
+      if (n > kKeep) {
         lo = mid;
       } else {
         hi = mid;
-        if (n == kCand) break;  // exactly kCand survive: as high as the floor needs to go
+        if (n == kKeep) break;  // exactly kKeep survive: as high as the floor needs to go
       }
     }
     fl = hi;
@@ -376,7 +379,23 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, in
         for (int i = 0; i < 16; ++i) incoming += (x[16 * k + i] > rc.thr) ? 1 : 0;
       }
   }
-  const unsigned need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
+  unsigned need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
+  if (need) {
+    // Entries pushed while the row max was lower go stale as it rises; every lane drops its
+    // stale entries (at or below its threshold) in parallel, and only lanes that still lack
+    // room take the cooperative insertion.
+    int n = 0;
+    for (int e = 0; e < rc.cnt; ++e) {
+      const float v = cs.s[e * kCols + col];
+      if (v > rc.thr) {
+        cs.s[n * kCols + col] = v;
+        cs.kt[n * kCols + col] = cs.kt[e * kCols + col];
+        ++n;
+      }
+    }
+    rc.cnt = n;
+    need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
+  }
   for (unsigned rest = need; rest; rest &= rest - 1u) {
     const int src = __ffs(rest) - 1;
     coop_insert<N>(cs, rc, src, col - lane + src, x, kt, lane);

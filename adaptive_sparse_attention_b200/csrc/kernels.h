@@ -14,6 +14,8 @@ cudaError_t launch_out_simt(const Problem& P, int dtype, cudaStream_t s);
 
 // Tensor-core (tcgen05) kernels, bf16 only, d in {64, 128}.
 cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s);
+// Multi-sweep tau search on the tensor cores for the overflow queue (one CTA per SM at most).
+cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t s);
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s);
 
 inline int beta_kind(float beta) {

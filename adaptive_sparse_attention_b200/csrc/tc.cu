@@ -437,6 +437,235 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   if (warp == 0) emit_tile(P, t, cs.words, cs.fallback, lane);
 }
 
+// ---------------------------------------------------------------------- tau overflow kernel --
+// tau_tc_sweep_kernel: the exact tau search for query tiles whose candidate buffers overflowed,
+// with no candidate buffers at all.  S = Q K^T is recomputed on the tensor cores for every sweep
+// over the tile's key range: one sweep for the row max, one per search step (the sums of
+// (z - tau)^beta, ^(beta - 1), ^(beta - 2) over all keys with z > tau), one for the mask bits.
+// Roles as in tau_tc_kernel; the four segment threads of a row combine their partial results
+// through shared memory after every sweep.  CTAs loop over the overflow queue.
+
+template <int D>
+struct SweepSmem {
+  alignas(1024) __nv_bfloat16 k[kTauStages][kTile * D];
+  float part[2][3][kSeg][kTile];  // per-sweep partials, double-buffered by sweep parity
+  uint32_t words[kMaxWords];
+  uint64_t q_full;
+  uint64_t k_full[kTauStages];
+  uint64_t k_empty[kTauStages];
+  uint64_t s_full[kTauSBufs];
+  uint64_t s_empty[kTauSBufs];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void score_warps_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kTauScoreWarps) : "memory");
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kTauThreads, 1)
+    tau_tc_sweep_kernel(const __grid_constant__ CUtensorMap tmk, Problem P) {
+  extern __shared__ unsigned char smem_raw[];
+  SweepSmem<D>& sm = *reinterpret_cast<SweepSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int ntiles = (P.cu ? 1 : P.B) * P.Hq * P.slots;
+  const int nq = min(*P.queue_count, ntiles);
+  if (static_cast<int>(blockIdx.x) >= nq) return;  // nothing queued for this CTA
+  volatile int* abort = &sm.abort;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+  const unsigned full = 0xffffffffu;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, kTauScoreWarps);
+    for (int s = 0; s < kTauStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int b = 0; b < kTauSBufs; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_empty[b], kTauScoreWarps);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int w = tid; w < kMaxWords; w += kTauThreads) sm.words[w] = 0u;
+  if (warp == kTauMmaWarp) tmem_alloc(&sm.tmem_base, kTauTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int nsweep = P.n_iter + 2;
+  int g = 0;       // key-tile steps so far in this CTA (identical in every role)
+  int tcount = 0;  // tiles so far (phase of q_full)
+  int issued_total = 0;
+
+  for (int i = blockIdx.x; i < nq; i += gridDim.x) {
+    const int id = P.queue[i];
+    if (id < 0 || id >= ntiles) continue;  // uniform across the block
+    const TileInfo t = map_tile(P, id % P.slots, (id / P.slots) % P.Hq, id / (P.slots * P.Hq));
+    const int nkt = t.nkt;
+    const int total = nsweep * nkt;
+    if (warp == kTauTmaWarp) {
+      if (lane == 0) {
+        const int krow0 = static_cast<int>(t.khead + t.seq_start);
+        for (int u = 0; u < total; ++u) {
+          const int gg = g + u, s = gg % kTauStages;
+          if (gg >= kTauStages &&
+              !mbar_wait(&sm.k_empty[s], ((gg / kTauStages) - 1) & 1, abort, P.status))
+            break;
+          mbar_expect_tx(&sm.k_full[s], kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
+                        krow0 + (u % nkt) * kTile);
+          issued_total = gg + 1;
+        }
+      }
+    } else if (warp == kTauMmaWarp) {
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+        bool ok = mbar_wait(&sm.q_full, tcount & 1, abort, P.status);
+        for (int u = 0; ok && u < total; ++u) {
+          const int gg = g + u, s = gg % kTauStages, b = gg % kTauSBufs;
+          if (!mbar_wait(&sm.k_full[s], (gg / kTauStages) & 1, abort, P.status)) break;
+          if (gg >= kTauSBufs &&
+              !mbar_wait(&sm.s_empty[b], ((gg / kTauSBufs) - 1) & 1, abort, P.status))
+            break;
+          tc_fence_after();
+          const uint32_t kbase = smem_u32(sm.k[s]);
+#pragma unroll
+          for (int k16 = 0; k16 < D / 16; ++k16)
+            mma_ts(tmem + static_cast<uint32_t>(b * 128), tmem + kTauColQ + k16 * 8,
+                   kmajor_desc(kbase, kTile, k16), idesc, k16 > 0 ? 1u : 0u);
+          mma_commit(&sm.k_empty[s]);
+          mma_commit(&sm.s_full[b]);
+          issued_total = gg + 1;
+        }
+      }
+    } else {  // score warps 0..15: every step of every sweep, even after an abort (barriers)
+      const int quarter = warp & 3;
+      const int seg = warp >> 2;
+      const int r = quarter * 32 + lane;
+      const bool valid = r < t.nrows;
+      const int jmax = valid ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+      {  // this thread's quarter of its query row into TMEM
+        constexpr int kWords = D / 8;
+        uint32_t w[kWords];
+        if (valid) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              static_cast<const __nv_bfloat16*>(P.q) + (t.qhead + t.seq_start + t.row0 + r) * D +
+              seg * (D / 4));
+#pragma unroll
+          for (int e = 0; e < kWords / 4; ++e) {
+            const uint4 u = src[e];
+            w[4 * e] = u.x;
+            w[4 * e + 1] = u.y;
+            w[4 * e + 2] = u.z;
+            w[4 * e + 3] = u.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < kWords; ++e) w[e] = 0u;
+        }
+        tmem_st_words<kWords>(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTauColQ +
+                                  static_cast<uint32_t>(seg * kWords),
+                              w);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.q_full);
+      }
+      Search sr;
+      sr.init(0.f, 1, P.alpha);
+      for (int sw = 0; sw < nsweep; ++sw) {
+        float a0 = (sw == 0) ? -INFINITY : 0.f, a1 = 0.f, a2 = 0.f;
+        const float tau = sr.tau;
+        for (int kt = 0; kt < nkt; ++kt) {
+          const int gg = g + sw * nkt + kt, b = gg % kTauSBufs;
+          const bool okw = __all_sync(
+              full, !*abort && mbar_wait(&sm.s_full[b], (gg / kTauSBufs) & 1, abort, P.status));
+          if (!okw) continue;
+          tc_fence_after();
+          float x[32];
+          tmem_row32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                         static_cast<uint32_t>(b * 128 + seg * 32),
+                     kt * kTile + seg * 32, jmax, x);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[b]);
+          if (sw == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) a0 = fmaxf(a0, x[e]);
+          } else if (sw <= P.n_iter) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float y = P.c * x[e] - tau;
+              if (y > 0.f) {
+                float p0, p1, p2;
+                entmax_powers<BK>(y, P.beta, p0, p1, p2);
+                a0 += p0;
+                a1 += p1;
+                a2 += p2;
+              }
+            }
+          } else {
+            bool any = false;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) any |= (P.c * x[e] > tau);
+            if (any) atomicOr(&sm.words[kt >> 5], 1u << (kt & 31));
+          }
+        }
+        if (sw == nsweep - 1) break;  // the mask sweep needs no combination
+        const int pb = sw & 1;
+        sm.part[pb][0][seg][r] = a0;
+        sm.part[pb][1][seg][r] = a1;
+        sm.part[pb][2][seg][r] = a2;
+        score_warps_sync();
+        float t0 = sm.part[pb][0][0][r], t1 = sm.part[pb][1][0][r], t2 = sm.part[pb][2][0][r];
+#pragma unroll
+        for (int q2 = 1; q2 < kSeg; ++q2) {
+          if (sw == 0) {
+            t0 = fmaxf(t0, sm.part[pb][0][q2][r]);
+          } else {
+            t0 += sm.part[pb][0][q2][r];
+            t1 += sm.part[pb][1][q2][r];
+            t2 += sm.part[pb][2][q2][r];
+          }
+        }
+        if (sw == 0) sr.init(valid ? P.c * t0 : 0.f, valid ? jmax : 1, P.alpha);
+        else sr.step<BK>(t0, t1, t2, P.beta);
+      }
+      if (seg == 0 && valid) P.tau[t.qhead + t.seq_start + t.row0 + r] = sr.tau;
+    }
+    g += total;
+    ++tcount;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (!*abort && warp == 0) emit_tile(P, t, sm.words, 0, lane);
+    __syncthreads();
+    for (int w = tid; w < kMaxWords; w += kTauThreads) sm.words[w] = 0u;
+  }
+  // drain: issued copies have landed and issued MMAs have completed before TMEM is released
+  if (warp == kTauTmaWarp && lane == 0) {
+    for (int gg = (issued_total > kTauStages ? issued_total - kTauStages : 0); gg < issued_total;
+         ++gg)
+      mbar_wait(&sm.k_full[gg % kTauStages], (gg / kTauStages) & 1, abort, P.status);
+  }
+  if (warp == kTauMmaWarp && lane == 0 && issued_total > 0) {
+    mma_commit(&sm.drain);
+    mbar_wait(&sm.drain, 0, abort, P.status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kTauMmaWarp) tmem_dealloc(tmem, kTauTmemCols);
+}
+
 // ------------------------------------------------------------------------------- out kernel --
 
 template <int D>
@@ -701,6 +930,19 @@ cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
 }
 
 template <int D, int BK>
+cudaError_t launch_sweep_t(const Problem& P, int num_ctas, cudaStream_t s) {
+  CUtensorMap mk;
+  cudaError_t e = make_map(&mk, P.k, kv_rows(P), D);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(SweepSmem<D>) + 1024;
+  auto kern = tau_tc_sweep_kernel<D, BK>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<num_ctas, kTauThreads, smem, s>>>(mk, P);
+  return cudaGetLastError();
+}
+
+template <int D, int BK>
 cudaError_t launch_out_t(const Problem& P, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
@@ -731,6 +973,18 @@ cudaError_t launch_out_t(const Problem& P, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s) { EA_TC_DISPATCH(launch_tau_t); }
+
+cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t s) {
+  const int bk = beta_kind(P.beta);
+  if (P.d == 64) {
+    if (bk == kBetaOne) return launch_sweep_t<64, kBetaOne>(P, num_ctas, s);
+    if (bk == kBetaTwo) return launch_sweep_t<64, kBetaTwo>(P, num_ctas, s);
+    return launch_sweep_t<64, kBetaGeneral>(P, num_ctas, s);
+  }
+  if (bk == kBetaOne) return launch_sweep_t<128, kBetaOne>(P, num_ctas, s);
+  if (bk == kBetaTwo) return launch_sweep_t<128, kBetaTwo>(P, num_ctas, s);
+  return launch_sweep_t<128, kBetaGeneral>(P, num_ctas, s);
+}
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) { EA_TC_DISPATCH(launch_out_t); }
 
 }  // namespace ea
