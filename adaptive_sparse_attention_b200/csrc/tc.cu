@@ -1,13 +1,11 @@
 // tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16, sm_100a.
 //
 // tau_tc_kernel (one CTA of 576 threads per 128-row query tile):
-//   warp 16     TMA producer: the tile's key tiles through a kTauStages-deep shared-memory ring
-//               (128B-swizzled, K-major).
+//   warp 16     TMA producer: the query tile, then the tile's key tiles through a 4-stage
+//               shared-memory ring (128B-swizzled, K-major).
 //   warp 17     allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
-//               K = d, fp32 accumulators) into one of three TMEM score buffers, so that the
-//               score warps can fall up to two tiles behind during a burst of insertions.  Q is
-//               the A operand from TMEM (the score warps store it there once), which halves the
-//               MMA's shared-memory reads; shared memory then carries only the K tiles.
+//               K = d, fp32 accumulators) into one of four TMEM score buffers, so that the score
+//               warps can fall up to three tiles behind during a burst of insertions.
 //   warps 0..15 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
 //               columns 32 g .. 32 g + 31 with g = w / 4, i.e. one 32-key segment of every key
 //               tile, into the segment's candidate buffer (common.cuh); the four segments of a
@@ -271,15 +269,21 @@ __device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&w
 
 // ------------------------------------------------------------------------------- tau kernel --
 
+// The tau kernel keeps Q in shared memory so that TMEM holds four 128-column score buffers: the
+// score warps may fall three key tiles behind the MMA during a burst of insertions.
+constexpr int kMainStages = 4;  // key tiles in flight
+constexpr int kMainSBufs = 4;   // TMEM score buffers
+
 template <int D>
 struct TauSmem {
-  alignas(1024) __nv_bfloat16 k[kTauStages][kTile * D];
+  alignas(1024) __nv_bfloat16 q[kTile * D];
+  alignas(1024) __nv_bfloat16 k[kMainStages][kTile * D];
   CandSmem cand;
   uint64_t q_full;
-  uint64_t k_full[kTauStages];
-  uint64_t k_empty[kTauStages];
-  uint64_t s_full[kTauSBufs];
-  uint64_t s_empty[kTauSBufs];
+  uint64_t k_full[kMainStages];
+  uint64_t k_empty[kMainStages];
+  uint64_t s_full[kMainSBufs];
+  uint64_t s_empty[kMainSBufs];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -287,7 +291,8 @@ struct TauSmem {
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kTauThreads, 1)
-    tau_tc_kernel(const __grid_constant__ CUtensorMap tmk, Problem P) {
+    tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  Problem P) {
   extern __shared__ unsigned char smem_raw[];
   TauSmem<D>& sm = *reinterpret_cast<TauSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -304,12 +309,12 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   constexpr uint32_t kTileBytes = kTile * D * 2;
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, kTauScoreWarps);  // each score warp stores its part of Q into TMEM
-    for (int s = 0; s < kTauStages; ++s) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kMainStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
     }
-    for (int b = 0; b < kTauSBufs; ++b) {
+    for (int b = 0; b < kMainSBufs; ++b) {
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.s_empty[b], kTauScoreWarps);  // one arrival per score warp
     }
@@ -329,12 +334,16 @@ __global__ void __launch_bounds__(kTauThreads, 1)
 
   if (warp == kTauTmaWarp) {
     if (lane == 0) {
+      const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
       const int krow0 = static_cast<int>(t.khead + t.seq_start);
+      mbar_expect_tx(&sm.q_full, kTileBytes);
+      for (int h = 0; h < D / 64; ++h)
+        tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
       int issued = 0;
       for (int kt = 0; kt < nkt; ++kt) {
-        const int s = kt % kTauStages;
-        if (kt >= kTauStages &&
-            !mbar_wait(&sm.k_empty[s], ((kt / kTauStages) - 1) & 1, abort, P.status))
+        const int s = kt % kMainStages;
+        if (kt >= kMainStages &&
+            !mbar_wait(&sm.k_empty[s], ((kt / kMainStages) - 1) & 1, abort, P.status))
           break;
         mbar_expect_tx(&sm.k_full[s], kTileBytes);
         for (int h = 0; h < D / 64; ++h)
@@ -342,28 +351,30 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         issued = kt + 1;
       }
       // drain: every issued copy has landed before the CTA may exit
-      for (int kt = (issued > kTauStages ? issued - kTauStages : 0); kt < issued; ++kt) {
-        const int s = kt % kTauStages;
-        mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status);
+      for (int kt = (issued > kMainStages ? issued - kMainStages : 0); kt < issued; ++kt) {
+        const int s = kt % kMainStages;
+        mbar_wait(&sm.k_full[s], (kt / kMainStages) & 1, abort, P.status);
       }
+      mbar_wait(&sm.q_full, 0, abort, P.status);
     }
   } else if (warp == kTauMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      const uint32_t qbase = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
       int issued = 0;
       for (int kt = 0; ok && kt < nkt; ++kt) {
-        const int s = kt % kTauStages, b = kt % kTauSBufs;
-        if (!mbar_wait(&sm.k_full[s], (kt / kTauStages) & 1, abort, P.status)) break;
-        if (kt >= kTauSBufs &&
-            !mbar_wait(&sm.s_empty[b], ((kt / kTauSBufs) - 1) & 1, abort, P.status))
+        const int s = kt % kMainStages, b = kt % kMainSBufs;
+        if (!mbar_wait(&sm.k_full[s], (kt / kMainStages) & 1, abort, P.status)) break;
+        if (kt >= kMainSBufs &&
+            !mbar_wait(&sm.s_empty[b], ((kt / kMainSBufs) - 1) & 1, abort, P.status))
           break;
         tc_fence_after();
         const uint32_t kbase = smem_u32(sm.k[s]);
         const uint32_t dcol = tmem + static_cast<uint32_t>(b * 128);
 #pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16)  // A = Q from TMEM: 16 columns of d = 8 TMEM columns
-          mma_ts(dcol, tmem + kTauColQ + k16 * 8, kmajor_desc(kbase, kTile, k16), idesc,
+        for (int k16 = 0; k16 < D / 16; ++k16)
+          mma_ss(dcol, kmajor_desc(qbase, kTile, k16), kmajor_desc(kbase, kTile, k16), idesc,
                  k16 > 0 ? 1u : 0u);
         mma_commit(&sm.k_empty[s]);
         mma_commit(&sm.s_full[b]);
@@ -380,40 +391,13 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     const int r = quarter * 32 + lane;  // query row of the tile == TMEM lane
     const int col = seg * kTile + r;
     const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
-    {  // this thread's quarter of its query row into TMEM (columns = packed bf16 pairs of d)
-      constexpr int kWords = D / 8;  // 32-bit columns per quarter row
-      uint32_t w[kWords];
-      if (r < t.nrows) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(P.q) + (t.qhead + t.seq_start + t.row0 + r) * D +
-            seg * (D / 4));
-#pragma unroll
-        for (int i = 0; i < kWords / 4; ++i) {
-          const uint4 u = src[i];
-          w[4 * i] = u.x;
-          w[4 * i + 1] = u.y;
-          w[4 * i + 2] = u.z;
-          w[4 * i + 3] = u.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < kWords; ++i) w[i] = 0u;
-      }
-      const uint32_t qa = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTauColQ +
-                          static_cast<uint32_t>(seg * kWords);
-      tmem_st_words<kWords>(qa, w);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.q_full);
-    }
     RowCand rc;
     rc.init(1.f / P.c);
     for (int kt = 0; kt < nkt; ++kt) {
-      const int b = kt % kTauSBufs;
+      const int b = kt % kMainSBufs;
       // the warp leaves together: feed_warp needs all 32 lanes
       if (!__all_sync(0xffffffffu,
-                      mbar_wait(&sm.s_full[b], (kt / kTauSBufs) & 1, abort, P.status)))
+                      mbar_wait(&sm.s_full[b], (kt / kMainSBufs) & 1, abort, P.status)))
         break;
       tc_fence_after();
       const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -918,14 +902,15 @@ dim3 tile_grid(const Problem& P) { return dim3(P.slots, P.Hq, P.cu ? 1 : P.B); }
 
 template <int D, int BK>
 cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
-  CUtensorMap mk;
-  cudaError_t e = make_map(&mk, P.k, kv_rows(P), D);
+  CUtensorMap mq, mk;
+  cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(TauSmem<D>) + 1024;
   auto kern = tau_tc_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<tile_grid(P), kTauThreads, smem, s>>>(mk, P);
+  kern<<<tile_grid(P), kTauThreads, smem, s>>>(mq, mk, P);
   return cudaGetLastError();
 }
 
