@@ -218,6 +218,23 @@ __device__ __forceinline__ float max16(const float (&x)[N], int o) {
   return max3f(max3f(a, b, c), max3f(d, e, x[o + 15]), -INFINITY);
 }
 
+// Shared-memory stores under a predicate, issued without a branch (the insertion loops below
+// would otherwise compile to one divergent branch per key).
+__device__ __forceinline__ void st_shared_if(bool p, float* addr, float v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q st.shared.f32 [%1], %2;\n}" ::"r"(
+          static_cast<int>(p)),
+      "r"(static_cast<uint32_t>(__cvta_generic_to_shared(addr))), "f"(v)
+      : "memory");
+}
+__device__ __forceinline__ void st_shared_if(bool p, uint16_t* addr, uint16_t v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q st.shared.u16 [%1], %2;\n}" ::"r"(
+          static_cast<int>(p)),
+      "r"(static_cast<uint32_t>(__cvta_generic_to_shared(addr))), "h"(v)
+      : "memory");
+}
+
 // Candidate state of one (row, segment), held in registers by the thread that owns it.
 struct RowCand {
   float m;       // running max of this segment's raw scores
@@ -373,25 +390,22 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, in
       cs.rowmax[row] = cmax;  // publish to the row's other segments
     }
 #pragma unroll
-    for (int k = 0; k < NB; ++k)
-      if (sub[k] > rc.thr) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) incoming += (x[16 * k + i] > rc.thr) ? 1 : 0;
-      }
+    for (int i = 0; i < N; ++i) incoming += (x[i] > rc.thr) ? 1 : 0;  // branch-free count
   }
   unsigned need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
   if (need) {
     // Entries pushed while the row max was lower go stale as it rises; every lane drops its
     // stale entries (at or below its threshold) in parallel, and only lanes that still lack
-    // room take the cooperative insertion.
+    // room take the cooperative insertion.  Fixed trip count, predicated stores: no branches.
     int n = 0;
-    for (int e = 0; e < rc.cnt; ++e) {
+#pragma unroll
+    for (int e = 0; e < kCand; ++e) {
       const float v = cs.s[e * kCols + col];
-      if (v > rc.thr) {
-        cs.s[n * kCols + col] = v;
-        cs.kt[n * kCols + col] = cs.kt[e * kCols + col];
-        ++n;
-      }
+      const uint16_t kk = cs.kt[e * kCols + col];
+      const bool keep = e < rc.cnt && v > rc.thr;
+      st_shared_if(keep, &cs.s[n * kCols + col], v);
+      st_shared_if(keep, &cs.kt[n * kCols + col], kk);
+      n += keep ? 1 : 0;
     }
     rc.cnt = n;
     need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
@@ -401,20 +415,17 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, in
     coop_insert<N>(cs, rc, src, col - lane + src, x, kt, lane);
   }
   if (pass && !((need >> lane) & 1u)) {
+    // room for every passing value is guaranteed here; predicated stores, no branches
+    int c = rc.cnt;
+    const uint16_t kt16 = static_cast<uint16_t>(kt);
 #pragma unroll
-    for (int k = 0; k < NB; ++k) {
-      if (sub[k] > rc.thr) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float v = x[16 * k + i];
-          if (v > rc.thr) {
-            cs.s[rc.cnt * kCols + col] = v;
-            cs.kt[rc.cnt * kCols + col] = static_cast<uint16_t>(kt);
-            ++rc.cnt;
-          }
-        }
-      }
+    for (int i = 0; i < N; ++i) {
+      const bool take = x[i] > rc.thr;
+      st_shared_if(take, &cs.s[c * kCols + col], x[i]);
+      st_shared_if(take, &cs.kt[c * kCols + col], kt16);
+      c += take ? 1 : 0;
     }
+    rc.cnt = c;
   }
 }
 
