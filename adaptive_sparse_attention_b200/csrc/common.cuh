@@ -23,6 +23,9 @@ constexpr int kSeg = 4;         // key segments per row (keys 32 g .. 32 g + 31 
                                 // each with its own running max and candidate buffer
 constexpr int kCand = 16;       // candidate slots per (row, segment) held in shared memory
 constexpr int kCols = kSeg * kTile;  // (row, segment) columns of the candidate buffers
+static_assert(kCand % 4 == 0, "the solve splits a buffer over 4 lanes");
+constexpr int kXchWarps = 16;  // warps feeding candidates per CTA (one exchange row each)
+constexpr int kExchangeMax = 2;  // up to this many passing rows of a warp go through the exchange row
 constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
 
 enum BetaKind { kBetaOne = 0, kBetaTwo = 1, kBetaGeneral = 2 };
@@ -188,7 +191,8 @@ struct Search {
 // of a warp hit 32 distinct banks whatever their fill levels.  A segment owns the keys 32 g ..
 // 32 g + 31 of every key tile.
 // ---------------------------------------------------------------------------------------------
-struct CandSmem {
+struct alignas(16) CandSmem {
+  float xrow[kXchWarps][32];  // per-warp exchange rows of feed_warp (first: 16-byte aligned)
   float s[kCand * kCols];
   uint16_t kt[kCand * kCols];
   float rowmax[kTile];  // running max of the row over all segments (raw); see feed_warp
@@ -265,50 +269,32 @@ struct RowCand {
 
 static_assert(kCand <= 32, "at most one candidate slot per lane in the cooperative insertion");
 
-// Warp-cooperative insertion for lane src (buffer column col_src) when its buffer cannot take
-// all of its passing values: lane e < kCand holds old entry e, and values e and e + 32 of src's
-// chunk x are spread over the warp by shuffles.  Old entries and new values at or below the
-// threshold are dropped; if more than kCand survive, the floor is raised by bisection to just
-// above the (kCand/2 + 1)-th largest value, so that the kCand/2 largest survive and the buffer
-// has room again (entries below the floor can only matter if tau ends up at or below it, which
-// the solve checks).  Survivors -- old ones first, then new ones in key order -- are written to the front
-// of the buffer.  Call with the whole warp converged; x is read from lane src only.
-template <int N>
+// Insertion of the passing values of one lane (src, buffer column col_src) when they do not fit
+// into its buffer.  Lane e < c0 holds old entry e, lane j holds value j of src's chunk (v).
+// Old entries and new values at or below the threshold th are dropped; if more than kCand
+// survive, the floor is raised by bisection to just above the (kCand/2 + 1)-th largest value,
+// so that the kCand/2 largest survive and the buffer has room again (entries below the floor
+// can only matter if tau ends up at or below it, which the solve checks).  Survivors -- old ones
+// first, then new ones in key order -- are written to the front of the buffer.  Warp-uniform
+// arguments; call with the whole warp converged.
 __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, int col_src,
-                                            const float (&x)[N], int kt, int lane) {
-  static_assert(N == 32 || N == 64, "chunks of 32 or 64 keys");
+                                            float v, float th, int c0, int kt, int lane) {
   const unsigned full = 0xffffffffu;
-  const int c = __shfl_sync(full, rc.cnt, src);
-  float th = __shfl_sync(full, rc.thr, src);
   float fl = __shfl_sync(full, rc.floor_, src);
   const float mm = __shfl_sync(full, rc.mx, src);
-  const bool have = lane < c;
+  const bool have = lane < c0;
   const float vo = have ? cs.s[lane * kCols + col_src] : -INFINITY;
   const uint16_t ko = have ? cs.kt[lane * kCols + col_src] : static_cast<uint16_t>(0);
-  float vn0 = -INFINITY, vn1 = -INFINITY;  // src's values lane and 32 + lane
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const float t = __shfl_sync(full, x[i], src);
-    if (lane == (i & 31)) {
-      if (i < 32) vn0 = t;
-      else vn1 = t;
-    }
-  }
   unsigned bo = __ballot_sync(full, vo > th);
-  unsigned b0 = __ballot_sync(full, vn0 > th);
-  unsigned b1 = __ballot_sync(full, vn1 > th);
-  if (__popc(bo) + __popc(b0) + __popc(b1) > kCand) {
-    // Raise the floor to (just above) the (kKeep + 1)-th largest value, kKeep = kCand / 2, so
-    // that later passing values find room without another cooperative insertion: bisection on
-    // [th, mm] keeps "more than kKeep above lo, at most kKeep above hi".
+  unsigned bn = __ballot_sync(full, v > th);
+  if (__popc(bo) + __popc(bn) > kCand) {
+    // Bisection on [th, mm] keeps "more than kKeep above lo, at most kKeep above hi".
     constexpr int kKeep = kCand / 2;
     float lo = th, hi = mm;
     for (int it = 0; it < 24; ++it) {
       const float mid = 0.5f * (lo + hi);
       if (!(mid > lo && mid < hi)) break;  // the interval cannot shrink further in fp32
-      const int n = __popc(__ballot_sync(full, vo > mid)) +
-                    __popc(__ballot_sync(full, vn0 > mid)) +
-                    __popc(__ballot_sync(full, vn1 > mid));
+      const int n = __popc(__ballot_sync(full, vo > mid)) + __popc(__ballot_sync(full, v > mid));
       if (n > kKeep) {
         lo = mid;
       } else {
@@ -319,34 +305,25 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
     fl = hi;
     th = hi;
     bo = __ballot_sync(full, vo > th);
-    b0 = __ballot_sync(full, vn0 > th);
-    b1 = __ballot_sync(full, vn1 > th);
+    bn = __ballot_sync(full, v > th);
   }
   const unsigned below = (1u << lane) - 1u;
-  const int no = __popc(bo), n0 = __popc(b0), n1 = __popc(b1);
-  __syncwarp();
+  const int no = __popc(bo), nn = __popc(bn);
+  __syncwarp();  // every old entry is in registers before the buffer is rewritten
   if ((bo >> lane) & 1u) {
     const int at = __popc(bo & below);
     cs.s[at * kCols + col_src] = vo;
     cs.kt[at * kCols + col_src] = ko;
   }
-  if ((b0 >> lane) & 1u) {
-    const int at = no + __popc(b0 & below);
+  if ((bn >> lane) & 1u) {
+    const int at = no + __popc(bn & below);
     if (at < kCand) {
-      cs.s[at * kCols + col_src] = vn0;
+      cs.s[at * kCols + col_src] = v;
       cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
     }
   }
-  if ((b1 >> lane) & 1u) {
-    const int at = no + n0 + __popc(b1 & below);
-    if (at < kCand) {
-      cs.s[at * kCols + col_src] = vn1;
-      cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
-    }
-  }
-  __syncwarp();
   if (lane == src) {
-    const int total = no + n0 + n1;
+    const int total = no + nn;
     rc.cnt = min(total, kCand);
     if (total > kCand) rc.lost = 1;  // only when ties at the floor could not be separated
     rc.thr = th;
@@ -354,34 +331,31 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   }
 }
 
-// Feeds N raw scores of key tile kt (keys outside the row's range already -inf) for the 32
+// Feeds 32 raw scores of key tile kt (keys outside the row's range already -inf) for the 32
 // (row, segment) columns of a warp; every lane of the warp must call it together.  The hot path
-// is the max of each 16-key block; only when a lane's block max passes its threshold does that
-// lane count and insert its passing values -- through the cooperative insertion above when its
-// buffer lacks room.  The threshold uses the largest max any segment of the row has published
-// in cs.rowmax[row]: a lower bound of the row's max, so every key with z > (row max) - 1 is
-// still kept, while records of one segment's max no longer trigger insertions in the others.
-// A stale or overwritten rowmax value only loosens the threshold.
+// is the max of each 16-key block.  A row whose chunk max passes its threshold is, when few rows
+// of the warp pass, handled by the whole warp: its lane writes the chunk to the warp's exchange
+// row xrow (32 floats, 16-byte aligned, private to the warp), every lane compares one value, and
+// a ballot gives each passing value its slot -- one compare per lane instead of 32 per passing
+// row.  When many rows pass (more than kExchangeMax), each lane stores its own values and only
+// rows without room take the exchange path.  The threshold uses the largest max any segment of
+// the row has published in cs.rowmax[row]: a lower bound of the row's max, so every key with
+// z > (row max) - 1 is still kept, while records of one segment's max no longer trigger
+// insertions in the others.  A stale or overwritten rowmax value only loosens the threshold.
 template <int N>
-__device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, int row, int lane,
-                                          const float (&x)[N], int kt) {
-  static_assert(N % 16 == 0, "16-key blocks");
-  constexpr int NB = N / 16;
+__device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, float* xrow, int col,
+                                          int row, int lane, const float (&x)[N], int kt) {
+  static_assert(N == 32, "one value per lane in the exchange row");
   const unsigned full = 0xffffffffu;
-  float sub[NB];
-#pragma unroll
-  for (int k = 0; k < NB; ++k) sub[k] = max16(x, 16 * k);
-  float cmax = sub[0];
-#pragma unroll
-  for (int k = 1; k < NB; ++k) cmax = fmaxf(cmax, sub[k]);
+  const float cmax = fmaxf(max16(x, 0), max16(x, 16));
   const float shared_max = *reinterpret_cast<volatile float*>(&cs.rowmax[row]);
   if (shared_max > rc.mx) {
     rc.mx = shared_max;
     rc.thr = fmaxf(rc.mx - rc.inv_c, rc.floor_);
   }
-  bool pass = cmax > rc.thr;
-  if (!__any_sync(full, pass)) return;
-  int incoming = 0;
+  const bool pass = cmax > rc.thr;
+  const unsigned passing = __ballot_sync(full, pass);
+  if (!passing) return;
   if (pass) {
     rc.m = fmaxf(rc.m, cmax);
     if (cmax > rc.mx) {
@@ -389,44 +363,75 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, int col, in
       rc.thr = fmaxf(rc.mx - rc.inv_c, rc.floor_);
       cs.rowmax[row] = cmax;  // publish to the row's other segments
     }
+  }
+  unsigned serial = passing;
+  if (__popc(passing) > kExchangeMax) {
+    // Many rows pass (the first key tiles of a row, before its max settles): each lane counts
+    // and stores its own passing values, all lanes at once; rows without room go on below.
+    int incoming = 0;
 #pragma unroll
     for (int i = 0; i < N; ++i) incoming += (x[i] > rc.thr) ? 1 : 0;  // branch-free count
-  }
-  unsigned need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
-  if (need) {
-    // Entries pushed while the row max was lower go stale as it rises; every lane drops its
-    // stale entries (at or below its threshold) in parallel, and only lanes that still lack
-    // room take the cooperative insertion.  Fixed trip count, predicated stores: no branches.
-    int n = 0;
+    const bool fits = pass && rc.cnt + incoming <= kCand;
+    if (fits) {
+      int c = rc.cnt;
+      const uint16_t kt16 = static_cast<uint16_t>(kt);
 #pragma unroll
-    for (int e = 0; e < kCand; ++e) {
-      const float v = cs.s[e * kCols + col];
-      const uint16_t kk = cs.kt[e * kCols + col];
-      const bool keep = e < rc.cnt && v > rc.thr;
-      st_shared_if(keep, &cs.s[n * kCols + col], v);
-      st_shared_if(keep, &cs.kt[n * kCols + col], kk);
-      n += keep ? 1 : 0;
+      for (int i = 0; i < N; ++i) {  // fixed trip count, predicated stores: no branches
+        const bool take = x[i] > rc.thr;
+        st_shared_if(take, &cs.s[c * kCols + col], x[i]);
+        st_shared_if(take, &cs.kt[c * kCols + col], kt16);
+        c += take ? 1 : 0;
+      }
+      rc.cnt = c;
     }
-    rc.cnt = n;
-    need = __ballot_sync(full, pass && rc.cnt + incoming > kCand);
+    serial = __ballot_sync(full, pass && !fits);
+    __syncwarp();  // these stores are visible to the lanes that read the buffers below
   }
-  for (unsigned rest = need; rest; rest &= rest - 1u) {
+  const unsigned below = (1u << lane) - 1u;
+  for (unsigned rest = serial; rest; rest &= rest - 1u) {
     const int src = __ffs(rest) - 1;
-    coop_insert<N>(cs, rc, src, col - lane + src, x, kt, lane);
-  }
-  if (pass && !((need >> lane) & 1u)) {
-    // room for every passing value is guaranteed here; predicated stores, no branches
-    int c = rc.cnt;
-    const uint16_t kt16 = static_cast<uint16_t>(kt);
+    if (lane == src) {
+      float4* d = reinterpret_cast<float4*>(xrow);
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const bool take = x[i] > rc.thr;
-      st_shared_if(take, &cs.s[c * kCols + col], x[i]);
-      st_shared_if(take, &cs.kt[c * kCols + col], kt16);
-      c += take ? 1 : 0;
+      for (int i = 0; i < 8; ++i) d[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
     }
-    rc.cnt = c;
+    __syncwarp();
+    const float v = xrow[lane];
+    const float th = __shfl_sync(full, rc.thr, src);
+    const int c0 = __shfl_sync(full, rc.cnt, src);
+    const int col_src = col - lane + src;
+    const unsigned take = __ballot_sync(full, v > th);
+    const int n = __popc(take);
+    if (c0 + n <= kCand) {
+      if ((take >> lane) & 1u) {
+        const int at = c0 + __popc(take & below);
+        cs.s[at * kCols + col_src] = v;
+        cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
+      }
+      if (lane == src) rc.cnt = c0 + n;
+    } else {
+      coop_insert(cs, rc, src, col_src, v, th, c0, kt, lane);
+    }
+    __syncwarp();  // the exchange row is read by every lane before the next row overwrites it
   }
+}
+
+// Takes 32 raw scores of a key tile into the row's running max without inserting candidates
+// (the keys are fed again later): raises the segment max, the row max shared with the other
+// segments and the threshold.
+template <int N>
+__device__ __forceinline__ void observe_max(RowCand& rc, CandSmem& cs, int row,
+                                            const float (&x)[N]) {
+  static_assert(N == 32, "32-key chunks");
+  const float cmax = fmaxf(max16(x, 0), max16(x, 16));
+  rc.m = fmaxf(rc.m, cmax);
+  const float shared_max = *reinterpret_cast<volatile float*>(&cs.rowmax[row]);
+  const float mx = fmaxf(shared_max, cmax);
+  if (mx > rc.mx) {
+    rc.mx = mx;
+    rc.thr = fmaxf(rc.mx - rc.inv_c, rc.floor_);
+  }
+  if (cmax > shared_max) cs.rowmax[row] = cmax;
 }
 
 // Solves tau for every row of the tile from the published candidate buffers of both segments,
@@ -453,6 +458,17 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     const float mz = valid ? P.c * mraw : 0.f;
     const int pos = t.row0 + r;
     const int n = valid ? (P.causal ? pos + 1 : t.seq_len) : 1;
+    // this lane's share of the row's candidates (raw scores; -inf in empty slots), held in
+    // registers for all search steps
+    float raw[kSeg][kCand / 4];
+#pragma unroll
+    for (int g = 0; g < kSeg; ++g) {
+#pragma unroll
+      for (int i = 0; i < kCand / 4; ++i) {
+        const int e = lane4 + 4 * i;
+        raw[g][i] = (e < cnt[g]) ? cs.s[e * kCols + g * kTile + r] : -INFINITY;
+      }
+    }
     Search sr;
     sr.init(mz, n, P.alpha);
     for (int it = 0; it < P.n_iter; ++it) {
@@ -460,8 +476,9 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
       float s0 = 0.f, s1 = 0.f, s2 = 0.f;
 #pragma unroll
       for (int g = 0; g < kSeg; ++g) {
-        for (int e = lane4; e < cnt[g]; e += 4) {
-          const float x = P.c * cs.s[e * kCols + g * kTile + r] - tau;
+#pragma unroll
+        for (int i = 0; i < kCand / 4; ++i) {
+          const float x = P.c * raw[g][i] - tau;
           if (x > 0.f) {
             float a, b, c2;
             entmax_powers<BK>(x, P.beta, a, b, c2);
@@ -492,10 +509,10 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     if (bad) cs.fallback = 1;
 #pragma unroll
     for (int g = 0; g < kSeg; ++g) {
-      for (int e = lane4; e < cnt[g]; e += 4) {
-        const int idx = e * kCols + g * kTile + r;
-        if (P.c * cs.s[idx] > tau) {
-          const int kt = cs.kt[idx];
+#pragma unroll
+      for (int i = 0; i < kCand / 4; ++i) {
+        if (P.c * raw[g][i] > tau) {
+          const int kt = cs.kt[(lane4 + 4 * i) * kCols + g * kTile + r];
           atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
         }
       }

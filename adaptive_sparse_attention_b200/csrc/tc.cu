@@ -45,6 +45,7 @@ namespace {
 constexpr int kOutThreads = 384;
 constexpr int kScoreWarp0 = 4;            // p warps of the out pass start at warp 4 (quarter w % 4)
 constexpr int kTauScoreWarps = 16;        // tau pass: warps 0..15 score, 16 TMA, 17 MMA
+static_assert(kTauScoreWarps <= kXchWarps, "one exchange row per score warp");
 constexpr int kTauTmaWarp = 16;
 constexpr int kTauMmaWarp = 17;
 constexpr int kTauThreads = 32 * (kTauScoreWarps + 2);
@@ -187,22 +188,23 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (lane = thread).
+// 32 consecutive TMEM columns of this warp's lanes into registers, waiting for the load in the
+// same asm statement: the registers are defined only once the data has arrived, so the compiler
+// cannot move a use of them ahead of the wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
+      "%28, %29, %30, %31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
         "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      : "r"(taddr)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -242,7 +244,6 @@ __device__ __forceinline__ uint64_t value_desc(uint32_t base, int k16) {
 __device__ __forceinline__ void tmem_row32(uint32_t ta, int j0, int jmax, float (&x)[32]) {
   uint32_t u[32];
   tmem_ld32(ta, u);
-  tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]);
   if (j0 + 32 > jmax) {  // diagonal or ragged tile
@@ -273,6 +274,14 @@ __device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&w
 // score warps may fall three key tiles behind the MMA during a burst of insertions.
 constexpr int kMainStages = 4;  // key tiles in flight
 constexpr int kMainSBufs = 4;   // TMEM score buffers
+
+// Key-tile order of the tau pass.  Until a row's running max has seen a few hundred keys, its
+// threshold is low and most scores are inserted as candidates, only to be dropped again later.
+// So the first w key tiles are first swept for the row max alone and fed as candidates once more
+// after the last tile; step i of the sweep handles key tile i (i < nkt) or i - nkt.  Costs w
+// extra Q K^T tiles; used when a row spans enough tiles for them to pay off.
+__device__ __forceinline__ int warm_tiles(int nkt) { return nkt >= 32 ? 8 : (nkt >= 16 ? 4 : 0); }
+__device__ __forceinline__ int step_tile(int i, int nkt) { return i < nkt ? i : i - nkt; }
 
 template <int D>
 struct TauSmem {
@@ -331,6 +340,8 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int nkt = t.nkt;
+  const int warm = warm_tiles(nkt);
+  const int nsteps = nkt + warm;
 
   if (warp == kTauTmaWarp) {
     if (lane == 0) {
@@ -340,20 +351,21 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       for (int h = 0; h < D / 64; ++h)
         tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
       int issued = 0;
-      for (int kt = 0; kt < nkt; ++kt) {
-        const int s = kt % kMainStages;
-        if (kt >= kMainStages &&
-            !mbar_wait(&sm.k_empty[s], ((kt / kMainStages) - 1) & 1, abort, P.status))
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % kMainStages;
+        const int kt = step_tile(i, nkt);
+        if (i >= kMainStages &&
+            !mbar_wait(&sm.k_empty[s], ((i / kMainStages) - 1) & 1, abort, P.status))
           break;
         mbar_expect_tx(&sm.k_full[s], kTileBytes);
         for (int h = 0; h < D / 64; ++h)
           tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64, krow0 + kt * kTile);
-        issued = kt + 1;
+        issued = i + 1;
       }
       // drain: every issued copy has landed before the CTA may exit
-      for (int kt = (issued > kMainStages ? issued - kMainStages : 0); kt < issued; ++kt) {
-        const int s = kt % kMainStages;
-        mbar_wait(&sm.k_full[s], (kt / kMainStages) & 1, abort, P.status);
+      for (int i = (issued > kMainStages ? issued - kMainStages : 0); i < issued; ++i) {
+        const int s = i % kMainStages;
+        mbar_wait(&sm.k_full[s], (i / kMainStages) & 1, abort, P.status);
       }
       mbar_wait(&sm.q_full, 0, abort, P.status);
     }
@@ -363,11 +375,11 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       const uint32_t qbase = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
       int issued = 0;
-      for (int kt = 0; ok && kt < nkt; ++kt) {
-        const int s = kt % kMainStages, b = kt % kMainSBufs;
-        if (!mbar_wait(&sm.k_full[s], (kt / kMainStages) & 1, abort, P.status)) break;
-        if (kt >= kMainSBufs &&
-            !mbar_wait(&sm.s_empty[b], ((kt / kMainSBufs) - 1) & 1, abort, P.status))
+      for (int i = 0; ok && i < nsteps; ++i) {
+        const int s = i % kMainStages, b = i % kMainSBufs;
+        if (!mbar_wait(&sm.k_full[s], (i / kMainStages) & 1, abort, P.status)) break;
+        if (i >= kMainSBufs &&
+            !mbar_wait(&sm.s_empty[b], ((i / kMainSBufs) - 1) & 1, abort, P.status))
           break;
         tc_fence_after();
         const uint32_t kbase = smem_u32(sm.k[s]);
@@ -378,7 +390,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
                  k16 > 0 ? 1u : 0u);
         mma_commit(&sm.k_empty[s]);
         mma_commit(&sm.s_full[b]);
-        issued = kt + 1;
+        issued = i + 1;
       }
       if (issued > 0) {  // all issued MMAs complete before tensor memory is released
         mma_commit(&sm.drain);
@@ -393,11 +405,12 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
     RowCand rc;
     rc.init(1.f / P.c);
-    for (int kt = 0; kt < nkt; ++kt) {
-      const int b = kt % kMainSBufs;
+    for (int i = 0; i < nsteps; ++i) {
+      const int b = i % kMainSBufs;
+      const int kt = step_tile(i, nkt);
       // the warp leaves together: feed_warp needs all 32 lanes
       if (!__all_sync(0xffffffffu,
-                      mbar_wait(&sm.s_full[b], (kt / kMainSBufs) & 1, abort, P.status)))
+                      mbar_wait(&sm.s_full[b], (i / kMainSBufs) & 1, abort, P.status)))
         break;
       tc_fence_after();
       const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -407,7 +420,10 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
-      feed_warp<32>(rc, cs, col, r, lane, x, kt);
+      if (i < warm)
+        observe_max(rc, cs, r, x);
+      else
+        feed_warp<32>(rc, cs, cs.xrow[warp], col, r, lane, x, kt);
     }
     rc.publish(cs, col);
   }
@@ -812,7 +828,6 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         const int c0 = half * 64 + q2 * 32;  // S column == key offset in the tile
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + kColS + b * 128 + c0, u);
-        tmem_wait_ld();
         uint32_t pk[16];
         const int j0 = kt * kTile + c0;
 #pragma unroll
@@ -843,7 +858,6 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       for (int c0 = 0; c0 < kHalfD; c0 += 32) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + kColO + half * kHalfD + c0, u);
-        tmem_wait_ld();
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(op + c0);
 #pragma unroll
