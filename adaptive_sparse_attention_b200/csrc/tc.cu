@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdint>
 #include <mutex>
 
@@ -879,6 +880,305 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------------------------- paired-head out kernel --
+// out_pair_kernel: the output pass for two query heads of one GQA group (same key/value head,
+// same query tile), so that every key and value tile is loaded once for both.  The tile walks
+// the union of the two heads' compact lists; each head computes S and O only on its own listed
+// tiles.  TMEM holds S_A, S_B (128 columns each) and O_A, O_B; P is written back over the S
+// columns its warp has already read (keys 64 h + 32 q of the tile -> columns 64 h + 16 q), so
+// the PV product of head X on a tile and the next S of head X are issued back to back and the
+// tensor pipe always holds the other head's work while one head's p warps run:
+//   ... PV_A(u), S_A(u+1), PV_B(u), S_B(u+1), PV_A(u+1), ...
+// tcgen05.mma instructions of a CTA execute in issue order, so S_X(u+1) overwrites the columns
+// PV_X(u) reads only after PV_X(u) has read them.
+//   warp 0       TMA producer of both query tiles and the key tiles (kPairKStages-stage ring)
+//   warp 1       tcgen05.mma issue (one thread)
+//   warp 2       TMA producer of the value tiles (kPairVStages-stage ring)
+//   warps 4..11  p warps of head A, warps 12..19 of head B (quarter w % 4, 64-key half)
+constexpr int kPairThreads = 640;
+constexpr int kPairKStages = 3;
+constexpr int kPairVStages = 2;
+constexpr uint32_t kPairColO = 256;  // O_A at 256, O_B at 384 (d <= 128 columns each)
+
+template <int D>
+struct PairSmem {
+  alignas(1024) __nv_bfloat16 q[2][kTile * D];
+  alignas(1024) __nv_bfloat16 k[kPairKStages][kTile * D];
+  alignas(1024) __nv_bfloat16 v[kPairVStages][kTile * D];
+  uint64_t q_full;
+  uint64_t k_full[kPairKStages];
+  uint64_t k_empty[kPairKStages];
+  uint64_t v_full[kPairVStages];
+  uint64_t v_empty[kPairVStages];
+  uint64_t s_full[2];  // per head: S_X of its next listed tile is in TMEM
+  uint64_t p_full[2];  // per head: its p warps have read S_X and stored P_X (8 arrivals)
+  uint64_t o_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Merged walk over two ascending compact lists (entries clamped to the tile's key range): each
+// step yields the next key tile and whether either list holds it.  Advances at least one list
+// per step, so it ends after at most na + nb steps whatever the lists hold.
+struct UnionWalk {
+  const int* la;
+  const int* lb;
+  int na, nb, ia, ib, nkt;
+  __device__ __forceinline__ bool next(int& kt, bool& in_a, bool& in_b) {
+    if (ia >= na && ib >= nb) return false;
+    const int a = ia < na ? clamp_kt(la[ia], nkt) : INT_MAX;
+    const int b = ib < nb ? clamp_kt(lb[ib], nkt) : INT_MAX;
+    kt = min(a, b);
+    in_a = a == kt;
+    in_b = b == kt;
+    ia += in_a ? 1 : 0;
+    ib += in_b ? 1 : 0;
+    return true;
+  }
+};
+
+// A shared-memory descriptor moved by a byte offset (the start address field holds address / 16
+// in 14 bits; every shared-memory address here is below 256 KB, so the field cannot overflow).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    out_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv, Problem P) {
+  extern __shared__ unsigned char smem_raw[];
+  PairSmem<D>& sm = *reinterpret_cast<PairSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int slot = gridDim.x - 1 - blockIdx.x;
+  const TileInfo ta = map_tile(P, slot, 2 * blockIdx.y, blockIdx.z);
+  if (!ta.valid) return;
+  const TileInfo tb = map_tile(P, slot, 2 * blockIdx.y + 1, blockIdx.z);
+  // Lists from the tau pass, clamped so that no workspace content sends a read outside them.
+  const int cnt_a = min(max(P.count[ta.tile_id], 0), ta.nkt);
+  const int cnt_b = min(max(P.count[tb.tile_id], 0), tb.nkt);
+  const int* list_a = P.list + ta.tile_id * P.nkt_max;
+  const int* list_b = P.list + tb.tile_id * P.nkt_max;
+  volatile int* abort = &sm.abort;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kPairKStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kPairVStages; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], 8);  // one arrival per p warp of the head
+    }
+    mbar_init(&sm.o_full, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0 || warp == 2) {
+    if (lane == 0) {
+      // warp 0 streams both query tiles and the key tiles, warp 2 the value tiles
+      const bool keys = warp == 0;
+      const CUtensorMap* map = keys ? &tmk : &tmv;
+      const int stages = keys ? kPairKStages : kPairVStages;
+      __nv_bfloat16* ring = keys ? sm.k[0] : sm.v[0];
+      uint64_t* full = keys ? sm.k_full : sm.v_full;
+      uint64_t* empty = keys ? sm.k_empty : sm.v_empty;
+      const int krow0 = static_cast<int>(ta.khead + ta.seq_start);
+      if (keys) {
+        mbar_expect_tx(&sm.q_full, 2 * kTileBytes);
+        const int qa = static_cast<int>(ta.qhead + ta.seq_start + ta.row0);
+        const int qb = static_cast<int>(tb.qhead + tb.seq_start + tb.row0);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(sm.q[0] + h * kTile * 64, &tmq, &sm.q_full, h * 64, qa);
+          tma_load_2d(sm.q[1] + h * kTile * 64, &tmq, &sm.q_full, h * 64, qb);
+        }
+      }
+      UnionWalk walk{list_a, list_b, cnt_a, cnt_b, 0, 0, ta.nkt};
+      int kt;
+      bool in_a, in_b;
+      int issued = 0;
+      for (int u = 0; walk.next(kt, in_a, in_b); ++u) {
+        const int s = u % stages;
+        if (u >= stages && !mbar_wait(&empty[s], ((u / stages) - 1) & 1, abort, P.status)) break;
+        mbar_expect_tx(&full[s], kTileBytes);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_2d(ring + s * kTile * D + h * kTile * 64, map, &full[s], h * 64,
+                      krow0 + kt * kTile);
+        issued = u + 1;
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int u = (issued > stages ? issued - stages : 0); u < issued; ++u)
+        mbar_wait(&full[u % stages], (u / stages) & 1, abort, P.status);
+      if (keys) mbar_wait(&sm.q_full, 0, abort, P.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(128, D, false, true);
+      // descriptors of both query tiles for every 16-wide slice of d, and the per-slice byte
+      // offsets inside a key tile (K-major) and a value tile (MN-major)
+      uint64_t qdesc[2][D / 16];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int k16 = 0; k16 < D / 16; ++k16) qdesc[x][k16] = kmajor_desc(smem_u32(sm.q[x]), kTile, k16);
+      const uint64_t kdesc0 = kmajor_desc(smem_u32(sm.k[0]), kTile, 0);
+      const uint64_t vdesc0 = value_desc(smem_u32(sm.v[0]), 0);
+      auto issue_s = [&](int x, int ks) {  // S_X = Q_X K^T from key stage ks
+        const uint64_t kd = desc_add(kdesc0, static_cast<uint32_t>(ks) * kTileBytes);
+#pragma unroll
+        for (int k16 = 0; k16 < D / 16; ++k16)
+          mma_ss(tmem + static_cast<uint32_t>(x * 128), qdesc[x][k16],
+                 desc_add(kd, static_cast<uint32_t>((k16 >> 2) * kTile * 128 + (k16 & 3) * 32)),
+                 idesc_s, k16 > 0 ? 1u : 0u);
+        mma_commit(&sm.s_full[x]);
+      };
+      auto issue_pv = [&](int x, int vs, bool first) {  // O_X += P_X V from value stage vs
+        const uint64_t vd = desc_add(vdesc0, static_cast<uint32_t>(vs) * kTileBytes);
+        const uint32_t sx = tmem + static_cast<uint32_t>(x * 128);
+#pragma unroll
+        for (int k16 = 0; k16 < kTile / 16; ++k16)
+          mma_ts(tmem + kPairColO + static_cast<uint32_t>(x * 128),
+                 sx + static_cast<uint32_t>(64 * (k16 >> 2) + 8 * (k16 & 3)),
+                 desc_add(vd, static_cast<uint32_t>(k16) * 2048u), idesc_o,
+                 (first && k16 == 0) ? 0u : 1u);
+      };
+      bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
+      UnionWalk walk{list_a, list_b, cnt_a, cnt_b, 0, 0, ta.nkt};
+      int kt;
+      bool cur_a = false, cur_b = false;
+      bool more = walk.next(kt, cur_a, cur_b);
+      int done_a = 0, done_b = 0;  // PV products issued per head
+      if (ok && more) {
+        ok = mbar_wait(&sm.k_full[0], 0, abort, P.status);
+        if (ok) {
+          tc_fence_after();
+          if (cur_a) issue_s(0, 0);
+          if (cur_b) issue_s(1, 0);
+          mma_commit(&sm.k_empty[0]);
+        }
+      }
+      for (int u = 0; ok && more; ++u) {
+        bool nx_a = false, nx_b = false;
+        const bool more_nx = walk.next(kt, nx_a, nx_b);
+        const int ks = (u + 1) % kPairKStages, vs = u % kPairVStages;
+        if (more_nx &&
+            !mbar_wait(&sm.k_full[ks], ((u + 1) / kPairKStages) & 1, abort, P.status))
+          break;
+        if (!mbar_wait(&sm.v_full[vs], (u / kPairVStages) & 1, abort, P.status)) break;
+        if (cur_a) {
+          if (!mbar_wait(&sm.p_full[0], done_a & 1, abort, P.status)) break;
+          tc_fence_after();
+          issue_pv(0, vs, done_a == 0);
+          ++done_a;
+        }
+        tc_fence_after();
+        if (nx_a) issue_s(0, ks);
+        if (cur_b) {
+          if (!mbar_wait(&sm.p_full[1], done_b & 1, abort, P.status)) break;
+          tc_fence_after();
+          issue_pv(1, vs, done_b == 0);
+          ++done_b;
+        }
+        if (nx_b) issue_s(1, ks);
+        mma_commit(&sm.v_empty[vs]);
+        if (more_nx) mma_commit(&sm.k_empty[ks]);
+        cur_a = nx_a;
+        cur_b = nx_b;
+        more = more_nx;
+      }
+      mma_commit(&sm.o_full);  // arrives once every MMA issued so far has completed
+    }
+  } else if (warp >= kScoreWarp0) {
+    const int x = (warp - kScoreWarp0) >> 3;  // head A or B
+    const TileInfo& t = x ? tb : ta;
+    const int cnt = x ? cnt_b : cnt_a;
+    const int* list = x ? list_b : list_a;
+    const int quarter = warp & 3;
+    const int half = ((warp - kScoreWarp0) >> 2) & 1;  // keys 64 half .. 64 half + 63
+    const int r = quarter * 32 + lane;
+    const bool row_ok = r < t.nrows;
+    const int pos = t.row0 + r;
+    const int jmax = row_ok ? (P.causal ? pos + 1 : t.seq_len) : 0;
+    const float tau = row_ok ? P.tau[t.qhead + t.seq_start + pos] : INFINITY;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t sx = tmem + lane_off + static_cast<uint32_t>(x * 128);
+    for (int i = 0; i < cnt; ++i) {
+      const int kt = clamp_kt(list[i], t.nkt);
+      if (!mbar_wait(&sm.s_full[x], i & 1, abort, P.status)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int c0 = half * 64 + q2 * 32;  // S column == key offset in the tile
+        uint32_t u[32];
+        tmem_ld32(sx + static_cast<uint32_t>(c0), u);
+        uint32_t pk[16];
+        const int j0 = kt * kTile + c0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float s0 = __uint_as_float(u[2 * e]), s1 = __uint_as_float(u[2 * e + 1]);
+          const float p0 = (j0 + 2 * e < jmax) ? entmax_p<BK>(P.c * s0 - tau, P.beta) : 0.f;
+          const float p1 = (j0 + 2 * e + 1 < jmax) ? entmax_p<BK>(P.c * s1 - tau, P.beta) : 0.f;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        // keys c0 .. c0 + 31 as 16 packed columns over S columns this warp has already read
+        tmem_st16(sx + static_cast<uint32_t>(half * 64 + q2 * 16), pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[x]);
+    }
+    // epilogue: this warp's half of O_X's columns, from TMEM to global memory
+    const bool o_ok = mbar_wait(&sm.o_full, 0, abort, P.status);
+    tc_fence_after();
+    constexpr int kHalfD = D / 2;
+    __nv_bfloat16* op =
+        static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D + half * kHalfD;
+    if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (only after a failed tau pass)
+      uint4* dst = reinterpret_cast<uint4*>(op);
+      for (int e = 0; e < kHalfD / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+    } else if (o_ok && !*abort) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < kHalfD; c0 += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + kPairColO + static_cast<uint32_t>(x * 128 + half * kHalfD + c0),
+                  u);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(op + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(u[8 * e + 0]), __uint_as_float(u[8 * e + 1]));
+            w.y = pack_bf16x2(__uint_as_float(u[8 * e + 2]), __uint_as_float(u[8 * e + 3]));
+            w.z = pack_bf16x2(__uint_as_float(u[8 * e + 4]), __uint_as_float(u[8 * e + 5]));
+            w.w = pack_bf16x2(__uint_as_float(u[8 * e + 6]), __uint_as_float(u[8 * e + 7]));
+            dst[e] = w;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 // ------------------------------------------------------------------------------ host side --
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
@@ -956,6 +1256,21 @@ cudaError_t launch_out_t(const Problem& P, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int D, int BK>
+cudaError_t launch_out_pair_t(const Problem& P, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mv, P.v, kv_rows(P), D);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(PairSmem<D>) + 1024;
+  auto kern = out_pair_kernel<D, BK>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(P.slots, P.Hq / 2, P.cu ? 1 : P.B), kPairThreads, smem, s>>>(mq, mk, mv, P);
+  return cudaGetLastError();
+}
+
 #define EA_TC_DISPATCH(FN)                                          \
   do {                                                              \
     const int bk = beta_kind(P.beta);                               \
@@ -984,6 +1299,10 @@ cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t 
   if (bk == kBetaTwo) return launch_sweep_t<128, kBetaTwo>(P, num_ctas, s);
   return launch_sweep_t<128, kBetaGeneral>(P, num_ctas, s);
 }
-cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) { EA_TC_DISPATCH(launch_out_t); }
+cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) {
+  // heads 2 j and 2 j + 1 share their key/value head when the group size is even
+  if (P.G % 2 == 0) EA_TC_DISPATCH(launch_out_pair_t);
+  EA_TC_DISPATCH(launch_out_t);
+}
 
 }  // namespace ea
