@@ -14,6 +14,7 @@ OK, EINVAL, EALIGN, ECUDA, ETIMEOUT, ENOMEM = 0, 1, 2, 3, 4, 5
 FP32, BF16 = 0, 1
 FLAG_CUDA_CORES = 1
 FLAG_ALL_FALLBACK = 2
+FLAG_TEST_STALL = 4  # test hook of the bounded device waits (ENTMAX_ATTN_FLAG_TEST_STALL)
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES
 
 _c_int, _c_float, _c_size_t, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p

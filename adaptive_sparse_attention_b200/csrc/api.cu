@@ -213,6 +213,7 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
   P.mask = block_mask;
   attach_workspace(&P, v);
   P.force_fallback = (flags & ENTMAX_ATTN_FLAG_ALL_FALLBACK) ? 1 : 0;
+  P.test_stall = (flags & ENTMAX_ATTN_FLAG_TEST_STALL) ? 1 : 0;
 
   cudaError_t e = cudaMemsetAsync(v.queue_count, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -55,6 +55,7 @@ struct Problem {
   int* queue_count;    // 1 int
   int* status;         // per-device status word
   int force_fallback;  // every tile takes the overflow path
+  int test_stall;      // test hook: the tensor-core tau kernel never requests its query tile
 };
 
 struct TileInfo {

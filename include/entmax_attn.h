@@ -75,6 +75,12 @@ extern "C" {
 #define ENTMAX_ATTN_FLAG_CUDA_CORES 1u    /* run BF16 products on the CUDA cores too */
 #define ENTMAX_ATTN_FLAG_ALL_FALLBACK 2u  /* send every query tile through the multi-sweep tau
                                              search that handles candidate-buffer overflow */
+#define ENTMAX_ATTN_FLAG_TEST_STALL 4u    /* test hook of the bounded waits: the tensor-core tau
+                                             pass never requests its query tiles, so each of its
+                                             CTAs gives up after one wait limit (about 2 s) and
+                                             the pass ends with ENTMAX_ATTN_ETIMEOUT in the
+                                             status word; its outputs are void.  Use it on a
+                                             problem of a few query tiles only. */
 
 /* Full forward pass: tau search + block mask, then the output pass over active tiles.
  * Writes out, tau and every word of block_mask.  Scratch memory (compact tile lists, overflow
