@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <mutex>
@@ -240,6 +241,12 @@ __device__ __forceinline__ uint64_t value_desc(uint32_t base, int k16) {
   return sw128_desc(base + static_cast<uint32_t>(k16) * 2048u, 128u * 128u, 1024u);
 }
 
+// A shared-memory descriptor moved by a byte offset (the start address field holds address / 16
+// in 14 bits; every shared-memory address here is below 256 KB, so the field cannot overflow).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // 32 raw scores of this thread's row from TMEM columns [ta, ta + 32), keys j0 + i; keys at or
 // past jmax (outside the row's causal / sequence range) read as -inf.
 __device__ __forceinline__ void tmem_row32(uint32_t ta, int j0, int jmax, float (&x)[32]) {
@@ -290,6 +297,7 @@ struct TauSmem {
   alignas(1024) __nv_bfloat16 k[kMainStages][kTile * D];
   CandSmem cand;
   uint64_t q_full;
+  uint64_t q_empty;
   uint64_t k_full[kMainStages];
   uint64_t k_empty[kMainStages];
   uint64_t s_full[kMainSBufs];
@@ -298,6 +306,30 @@ struct TauSmem {
   uint32_t tmem_base;
   int abort;
 };
+
+// Score warps only (named barrier 1): a barrier, and a barrier that also returns whether any
+// score thread passed a true flag (the same answer in every thread).
+__device__ __forceinline__ void score_warps_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kTauScoreWarps) : "memory");
+}
+__device__ __forceinline__ bool score_warps_any(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.b32 p, %1, 0;\n"
+      " barrier.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"(static_cast<int>(flag)), "n"(32 * kTauScoreWarps)
+      : "memory");
+  return r != 0;
+}
+
+// Query tile L of the tau pass's tile order: the longest tiles (highest slot) of every head
+// first, so that the tiles a persistent CTA takes in turn shrink as the pass runs out.
+__device__ __forceinline__ TileInfo tau_tile(const Problem& P, int L, int per_slot) {
+  const int slot = P.slots - 1 - L / per_slot;
+  const int hb = L % per_slot;
+  return map_tile(P, slot, hb % P.Hq, hb / P.Hq);
+}
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kTauThreads, 1)
@@ -309,17 +341,14 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   CandSmem& cs = sm.cand;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int slot = gridDim.x - 1 - blockIdx.x;  // longest query tiles first
-  const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
-  if (!t.valid) {
-    emit_empty(P, t, tid, kTauThreads);
-    return;
-  }
+  const int per_slot = P.Hq * (P.cu ? 1 : P.B);
+  const int ntiles = P.slots * per_slot;
   volatile int* abort = &sm.abort;
   constexpr uint32_t kTileBytes = kTile * D * 2;
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kMainStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -334,68 +363,88 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
-  for (int r = tid; r < kTile; r += kTauThreads) cs.rowmax[r] = -INFINITY;
   if (warp == kTauMmaWarp) tmem_alloc(&sm.tmem_base, kTauTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const int nkt = t.nkt;
-  const int warm = warm_tiles(nkt);
-  const int nsteps = nkt + warm;
 
+  // Every role walks the same tiles L = blockIdx.x, blockIdx.x + gridDim.x, ...; the rings
+  // (key stages, score buffers) and the query buffer's phases run on across tiles, so the
+  // producer and the MMA thread start on the next tile while the score warps finish this one.
   if (warp == kTauTmaWarp) {
     if (lane == 0) {
-      const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
-      const int krow0 = static_cast<int>(t.khead + t.seq_start);
-      if (!P.test_stall) {  // the test hook leaves q_full incomplete: every wait runs out
-        mbar_expect_tx(&sm.q_full, kTileBytes);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
-      }
-      int issued = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i % kMainStages;
-        const int kt = step_tile(i, nkt);
-        if (i >= kMainStages &&
-            !mbar_wait(&sm.k_empty[s], ((i / kMainStages) - 1) & 1, abort, P.status))
-          break;
-        mbar_expect_tx(&sm.k_full[s], kTileBytes);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64, krow0 + kt * kTile);
-        issued = i + 1;
+      int it = 0, gk = 0;  // tiles and key tiles issued so far
+      bool ok = true;
+      for (int L = blockIdx.x; ok && L < ntiles; L += gridDim.x) {
+        const TileInfo t = tau_tile(P, L, per_slot);
+        if (!t.valid) continue;
+        // the query buffer is free once every S product of the previous tile has completed
+        if (it > 0 && !mbar_wait(&sm.q_empty, (it - 1) & 1, abort, P.status)) break;
+        const int qrow = static_cast<int>(t.qhead + t.seq_start + t.row0);
+        const int krow0 = static_cast<int>(t.khead + t.seq_start);
+        if (!P.test_stall) {  // the test hook leaves q_full incomplete: every wait runs out
+          mbar_expect_tx(&sm.q_full, kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
+        }
+        ++it;
+        const int nkt = t.nkt, nsteps = nkt + warm_tiles(nkt);
+        for (int i = 0; i < nsteps; ++i, ++gk) {
+          const int s = gk % kMainStages;
+          if (gk >= kMainStages &&
+              !mbar_wait(&sm.k_empty[s], ((gk / kMainStages) - 1) & 1, abort, P.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&sm.k_full[s], kTileBytes);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
+                        krow0 + step_tile(i, nkt) * kTile);
+        }
       }
       // drain: every issued copy has landed before the CTA may exit
-      for (int i = (issued > kMainStages ? issued - kMainStages : 0); i < issued; ++i) {
-        const int s = i % kMainStages;
-        mbar_wait(&sm.k_full[s], (i / kMainStages) & 1, abort, P.status);
-      }
-      mbar_wait(&sm.q_full, 0, abort, P.status);
+      for (int g = (gk > kMainStages ? gk - kMainStages : 0); g < gk; ++g)
+        mbar_wait(&sm.k_full[g % kMainStages], (g / kMainStages) & 1, abort, P.status);
+      if (it > 0) mbar_wait(&sm.q_full, (it - 1) & 1, abort, P.status);
     }
   } else if (warp == kTauMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
-      const uint32_t qbase = smem_u32(sm.q);
-      bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
-      int issued = 0;
-      for (int i = 0; ok && i < nsteps; ++i) {
-        const int s = i % kMainStages, b = i % kMainSBufs;
-        if (!mbar_wait(&sm.k_full[s], (i / kMainStages) & 1, abort, P.status)) break;
-        if (i >= kMainSBufs &&
-            !mbar_wait(&sm.s_empty[b], ((i / kMainSBufs) - 1) & 1, abort, P.status))
-          break;
-        tc_fence_after();
-        const uint32_t kbase = smem_u32(sm.k[s]);
-        const uint32_t dcol = tmem + static_cast<uint32_t>(b * 128);
+      uint64_t qdesc[D / 16];
 #pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16)
-          mma_ss(dcol, kmajor_desc(qbase, kTile, k16), kmajor_desc(kbase, kTile, k16), idesc,
-                 k16 > 0 ? 1u : 0u);
-        mma_commit(&sm.k_empty[s]);
-        mma_commit(&sm.s_full[b]);
-        issued = i + 1;
+      for (int k16 = 0; k16 < D / 16; ++k16) qdesc[k16] = kmajor_desc(smem_u32(sm.q), kTile, k16);
+      const uint64_t kdesc0 = kmajor_desc(smem_u32(sm.k[0]), kTile, 0);
+      int it = 0, gk = 0;  // tiles and key tiles consumed so far (one S buffer per key tile)
+      bool ok = true;
+      for (int L = blockIdx.x; ok && L < ntiles; L += gridDim.x) {
+        const TileInfo t = tau_tile(P, L, per_slot);
+        if (!t.valid) continue;
+        if (!mbar_wait(&sm.q_full, it & 1, abort, P.status)) break;
+        ++it;
+        const int nsteps = t.nkt + warm_tiles(t.nkt);
+        for (int i = 0; i < nsteps; ++i, ++gk) {
+          const int s = gk % kMainStages, b = gk % kMainSBufs;
+          if (!mbar_wait(&sm.k_full[s], (gk / kMainStages) & 1, abort, P.status) ||
+              (gk >= kMainSBufs &&
+               !mbar_wait(&sm.s_empty[b], ((gk / kMainSBufs) - 1) & 1, abort, P.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = desc_add(kdesc0, static_cast<uint32_t>(s) * kTileBytes);
+          const uint32_t dcol = tmem + static_cast<uint32_t>(b * 128);
+#pragma unroll
+          for (int k16 = 0; k16 < D / 16; ++k16)
+            mma_ss(dcol, qdesc[k16],
+                   desc_add(kd, static_cast<uint32_t>((k16 >> 2) * kTile * 128 + (k16 & 3) * 32)),
+                   idesc, k16 > 0 ? 1u : 0u);
+          mma_commit(&sm.k_empty[s]);
+          mma_commit(&sm.s_full[b]);
+        }
+        if (ok) mma_commit(&sm.q_empty);  // the tile's S products have read Q
       }
-      if (issued > 0) {  // all issued MMAs complete before tensor memory is released
+      if (gk > 0) {  // all issued MMAs complete before tensor memory is released
         mma_commit(&sm.drain);
         mbar_wait(&sm.drain, 0, abort, P.status);
       }
@@ -405,39 +454,57 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     const int seg = warp >> 2;  // keys 32 seg .. 32 seg + 31 of every key tile
     const int r = quarter * 32 + lane;  // query row of the tile == TMEM lane
     const int col = seg * kTile + r;
-    const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
-    RowCand rc;
-    rc.init(1.f / P.c);
-    for (int i = 0; i < nsteps; ++i) {
-      const int b = i % kMainSBufs;
-      const int kt = step_tile(i, nkt);
-      // the warp leaves together: feed_warp needs all 32 lanes
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(&sm.s_full[b], (i / kMainSBufs) & 1, abort, P.status)))
-        break;
-      tc_fence_after();
-      const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                          static_cast<uint32_t>(b * 128 + seg * 32);
-      float x[32];
-      tmem_row32(ta, kt * kTile + seg * 32, jmax, x);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
-      if (i < warm)
-        observe_max(rc, cs, r, x);
-      else
-        feed_warp<32>(rc, cs, cs.xrow[warp], col, r, lane, x, kt);
+    constexpr int kScoreThreads = 32 * kTauScoreWarps;
+    int gs = 0;  // score buffers consumed so far
+    for (int L = blockIdx.x; L < ntiles; L += gridDim.x) {
+      const TileInfo t = tau_tile(P, L, per_slot);
+      if (!t.valid) {
+        emit_empty(P, t, tid, kScoreThreads);
+        continue;
+      }
+      // per-tile shared state; warp 0 cleared the mask words and the flag after its last emit
+      if (tid < kTile) cs.rowmax[tid] = -INFINITY;  // warps 0..3: thread tid owns row tid
+      score_warps_sync();
+      const int nkt = t.nkt, warm = warm_tiles(nkt), nsteps = nkt + warm;
+      const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+      RowCand rc;
+      rc.init(1.f / P.c);
+      for (int i = 0; i < nsteps; ++i, ++gs) {
+        const int b = gs % kMainSBufs;
+        const int kt = step_tile(i, nkt);
+        // the warp leaves together: feed_warp needs all 32 lanes
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&sm.s_full[b], (gs / kMainSBufs) & 1, abort, P.status)))
+          break;
+        tc_fence_after();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            static_cast<uint32_t>(b * 128 + seg * 32);
+        float x[32];
+        tmem_row32(ta, kt * kTile + seg * 32, jmax, x);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
+        if (i < warm)
+          observe_max(rc, cs, r, x);
+        else
+          feed_warp<32>(rc, cs, cs.xrow[warp], col, r, lane, x, kt);
+      }
+      rc.publish(cs, col);
+      if (score_warps_any(*abort != 0)) break;  // status already records the timeout
+      solve_rows<BK>(P, t, cs, tid, kScoreThreads);
+      score_warps_sync();
+      if (warp == 0) {
+        emit_tile(P, t, cs.words, cs.fallback, lane);
+        __syncwarp();
+        for (int w = lane; w < kMaxWords; w += 32) cs.words[w] = 0u;
+        if (lane == 0) cs.fallback = P.force_fallback;
+      }
     }
-    rc.publish(cs, col);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kTauMmaWarp) tmem_dealloc(tmem, kTauTmemCols);
-  if (*abort) return;  // status already records the timeout; outputs of this tile are void
-  if (warp < kTauScoreWarps) solve_rows<BK>(P, t, cs, tid, 32 * kTauScoreWarps);
-  __syncthreads();
-  if (warp == 0) emit_tile(P, t, cs.words, cs.fallback, lane);
 }
 
 // ---------------------------------------------------------------------- tau overflow kernel --
@@ -462,10 +529,6 @@ struct SweepSmem {
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ void score_warps_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(32 * kTauScoreWarps) : "memory");
-}
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kTauThreads, 1)
@@ -939,12 +1002,6 @@ struct UnionWalk {
   }
 };
 
-// A shared-memory descriptor moved by a byte offset (the start address field holds address / 16
-// in 14 bits; every shared-memory address here is below 256 KB, so the field cannot overflow).
-__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
-  return desc + static_cast<uint64_t>(bytes >> 4);
-}
-
 template <int D, int BK>
 __global__ void __launch_bounds__(kPairThreads, 1)
     out_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -1216,6 +1273,14 @@ int64_t kv_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) 
 
 dim3 tile_grid(const Problem& P) { return dim3(P.slots, P.Hq, P.cu ? 1 : P.B); }
 
+// Streaming multiprocessors of the current device (one persistent CTA each).
+cudaError_t device_sms(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  return e;
+}
+
 template <int D, int BK>
 cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
   CUtensorMap mq, mk;
@@ -1226,7 +1291,11 @@ cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
   auto kern = tau_tc_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<tile_grid(P), kTauThreads, smem, s>>>(mq, mk, P);
+  int sms = 0;
+  e = device_sms(&sms);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = static_cast<int64_t>(P.slots) * P.Hq * (P.cu ? 1 : P.B);
+  kern<<<static_cast<unsigned>(std::min<int64_t>(ntiles, sms)), kTauThreads, smem, s>>>(mq, mk, P);
   return cudaGetLastError();
 }
 
