@@ -1135,9 +1135,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         bool nx_a = false, nx_b = false;
         const bool more_nx = walk.next(kt, nx_a, nx_b);
         const int ks = (u + 1) % kPairKStages, vs = u % kPairVStages;
-        if (more_nx &&
-            !mbar_wait(&sm.k_full[ks], ((u + 1) / kPairKStages) & 1, abort, P.status))
-          break;
+        // each resource is awaited just before its first use, so that whatever is ready
+        // reaches the tensor pipe first
         if (!mbar_wait(&sm.v_full[vs], (u / kPairVStages) & 1, abort, P.status)) break;
         if (cur_a) {
           if (!mbar_wait(&sm.p_full[0], done_a & 1, abort, P.status)) break;
@@ -1145,6 +1144,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           issue_pv(0, vs, done_a == 0);
           ++done_a;
         }
+        if (more_nx &&
+            !mbar_wait(&sm.k_full[ks], ((u + 1) / kPairKStages) & 1, abort, P.status))
+          break;
         tc_fence_after();
         if (nx_a) issue_s(0, ks);
         if (cur_b) {
