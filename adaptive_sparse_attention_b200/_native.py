@@ -14,6 +14,7 @@ OK, EINVAL, EALIGN, ECUDA, ETIMEOUT, ENOMEM = 0, 1, 2, 3, 4, 5
 FP32, BF16 = 0, 1
 FLAG_CUDA_CORES = 1
 FLAG_ALL_FALLBACK = 2
+FLAG_NO_BLOCK_MASK = 8  # ENTMAX_ATTN_FLAG_NO_BLOCK_MASK
 FLAG_TEST_STALL = 4  # test hook of the bounded device waits (ENTMAX_ATTN_FLAG_TEST_STALL)
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES
 
@@ -24,6 +25,9 @@ _c_uint = ctypes.c_uint
 SIGNATURES = {
     "entmax_attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                  _c_int, _c_float, _c_int, _c_int, _vp, _c_int, _vp]),
+    "entmax_attn_fwd_no_block_mask": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                               _c_int, _c_int, _c_float, _c_int, _c_int, _vp,
+                                               _c_int, _vp]),
     "entmax_attn_mask_words": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "entmax_attn_mask_layout": (_c_int, [_c_int, _c_int, _c_int, _c_int,
                                          ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),

@@ -110,6 +110,24 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool 
     return out, tau, block_mask
 
 
+def entmax_attn_fwd_no_block_mask(q, k, v, alpha: float = 1.5, n_iter: int = 10,
+                                  causal: bool = True, cu_seqlens=None, out=None, tau=None,
+                                  stream=None):
+    """Forward pass without the block mask (the output pass visits every causally valid key
+    tile).  Returns (out, tau)."""
+    _check_inputs(q, k, v, cu_seqlens)
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    o2, t2, _ = alloc_outputs(q, k, cu_seqlens) if None in (out, tau) else (None,) * 3
+    out = o2 if out is None else out
+    tau = t2 if tau is None else tau
+    rc = N.lib().entmax_attn_fwd_no_block_mask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(tau),
+                                               B, Hq, Hkv, T, d, float(alpha), int(n_iter),
+                                               int(bool(causal)), _ptr(cu_seqlens), _DT[q.dtype],
+                                               _stream(stream))
+    N.check(rc, "entmax_attn_fwd_no_block_mask")
+    return out, tau
+
+
 def entmax_attn_fwd_noalloc(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool = True,
                             cu_seqlens=None, out=None, tau=None, block_mask=None, stream=None):
     """Forward pass through the allocation-free entry point: the library's scratch is a fixed

@@ -200,8 +200,9 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
   int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
                               &L, &P);
   if (rc != ENTMAX_ATTN_OK) return rc;
-  if (!tau || !block_mask || !workspace) return ENTMAX_ATTN_EINVAL;
-  if (!aligned16(tau) || !aligned16(block_mask) ||
+  const bool no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) != 0;
+  if (!tau || (!block_mask && !no_mask) || !workspace) return ENTMAX_ATTN_EINVAL;
+  if (!aligned16(tau) || (block_mask && !aligned16(block_mask)) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return ENTMAX_ATTN_EALIGN;
   const WsView v = ws_view(workspace, L);
@@ -214,6 +215,7 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
   attach_workspace(&P, v);
   P.force_fallback = (flags & ENTMAX_ATTN_FLAG_ALL_FALLBACK) ? 1 : 0;
   P.test_stall = (flags & ENTMAX_ATTN_FLAG_TEST_STALL) ? 1 : 0;
+  P.no_mask = no_mask ? 1 : 0;
 
   cudaError_t e = cudaMemsetAsync(v.queue_count, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -254,22 +256,26 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
   P.out = out;
   P.tau = const_cast<float*>(tau);
   attach_workspace(&P, wv);
+  P.no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) ? 1 : 0;
   cudaError_t e = use_tensor_cores(dtype, flags) ? ea::launch_out_tc(P, stream)
                                                  : ea::launch_out_simt(P, dtype, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return ENTMAX_ATTN_OK;
 }
 
-int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
-                    uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
-                    int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
-                    cudaStream_t stream) {
+namespace {
+
+// Both passes on the library's cached workspace of (device, stream); flags as the two-pass form.
+int fwd_cached(const void* q, const void* k, const void* v, void* out, float* tau,
+               uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
+               int n_iter, int causal, const int32_t* cu_seqlens, int dtype, unsigned flags,
+               cudaStream_t stream) {
   Layout L;
   ea::Problem P;
   int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
                               &L, &P);
   if (rc != ENTMAX_ATTN_OK) return rc;
-  if (!v || !out || !tau || !block_mask) return ENTMAX_ATTN_EINVAL;
+  if (!v || !out || !tau) return ENTMAX_ATTN_EINVAL;
   const size_t need = ws_view(nullptr, L).bytes;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -295,10 +301,29 @@ int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, floa
     ws = c.ptr;
   }
   rc = entmax_attn_tau_pass(q, k, tau, block_mask, ws, need, B, Hq, Hkv, T, d, alpha, n_iter,
-                            causal, cu_seqlens, dtype, 0u, stream);
+                            causal, cu_seqlens, dtype, flags, stream);
   if (rc != ENTMAX_ATTN_OK) return rc;
   return entmax_attn_out_pass(q, k, v, tau, ws, need, out, B, Hq, Hkv, T, d, alpha, causal,
-                              cu_seqlens, dtype, 0u, stream);
+                              cu_seqlens, dtype, flags, stream);
+}
+
+}  // namespace
+
+int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
+                    uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
+                    int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                    cudaStream_t stream) {
+  if (!block_mask) return ENTMAX_ATTN_EINVAL;
+  return fwd_cached(q, k, v, out, tau, block_mask, B, Hq, Hkv, T, d, alpha, n_iter, causal,
+                    cu_seqlens, dtype, 0u, stream);
+}
+
+int entmax_attn_fwd_no_block_mask(const void* q, const void* k, const void* v, void* out,
+                                  float* tau, int B, int Hq, int Hkv, int T, int d, float alpha,
+                                  int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                                  cudaStream_t stream) {
+  return fwd_cached(q, k, v, out, tau, nullptr, B, Hq, Hkv, T, d, alpha, n_iter, causal,
+                    cu_seqlens, dtype, ENTMAX_ATTN_FLAG_NO_BLOCK_MASK, stream);
 }
 
 int entmax_attn_fallback_tiles(const void* workspace, cudaStream_t stream) {

@@ -56,6 +56,8 @@ struct Problem {
   int* status;         // per-device status word
   int force_fallback;  // every tile takes the overflow path
   int test_stall;      // test hook: the tensor-core tau kernel never requests its query tile
+  int no_mask;         // no block mask: the tau pass writes neither mask nor lists, and the
+                       // output pass visits every causally valid key tile
 };
 
 struct TileInfo {
@@ -532,6 +534,7 @@ __device__ __forceinline__ void emit_tile(const Problem& P, const TileInfo& t,
     }
     return;
   }
+  if (P.no_mask) return;
   uint32_t* mw = P.mask + t.tile_id * P.W;
   int* list = P.list + t.tile_id * P.nkt_max;
   int base = 0;
@@ -564,9 +567,21 @@ __device__ __forceinline__ int clamp_kt(int kt, int nkt) {
   return (kt >= 0 && kt < nkt) ? kt : 0;
 }
 
+// Number of key tiles the output pass visits for a query tile: its compact list's count, clamped
+// to the tile's key range, or every causally valid key tile without the block mask.
+__device__ __forceinline__ int list_count(const Problem& P, const TileInfo& t) {
+  return P.no_mask ? t.nkt : min(max(P.count[t.tile_id], 0), t.nkt);
+}
+
+// Key tile of entry i of that sequence (list points at the query tile's compact list).
+__device__ __forceinline__ int list_tile(const Problem& P, const int* list, int i, int nkt) {
+  return P.no_mask ? i : clamp_kt(list[i], nkt);
+}
+
 // Unused slot of a packed batch: zero mask words, empty list.
 __device__ __forceinline__ void emit_empty(const Problem& P, const TileInfo& t, int tid,
                                            int nthreads) {
+  if (P.no_mask) return;
   for (int w = tid; w < P.W; w += nthreads) P.mask[t.tile_id * P.W + w] = 0u;
   if (tid == 0) P.count[t.tile_id] = 0;
 }

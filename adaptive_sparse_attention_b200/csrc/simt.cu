@@ -232,10 +232,10 @@ __global__ void __launch_bounds__(kThreads) out_simt_kernel(Problem P) {
 #pragma unroll
   for (int c = 0; c < D; ++c) o[c] = 0.f;
 
-  const int cnt = min(max(P.count[t.tile_id], 0), t.nkt);  // see clamp_kt
+  const int cnt = list_count(P, t);  // see clamp_kt
   const int* list = P.list + t.tile_id * P.nkt_max;
   for (int i = 0; i < cnt; ++i) {
-    const int kt = clamp_kt(list[i], t.nkt);
+    const int kt = list_tile(P, list, i, t.nkt);
     for (int ch = 0; ch < kTile / kChunk; ++ch) {
       const int j0 = kt * kTile + ch * kChunk;
       if (j0 >= t.seq_len) break;

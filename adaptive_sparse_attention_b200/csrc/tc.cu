@@ -770,7 +770,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   if (!t.valid) return;
   // The list comes from the tau pass; clamping keeps every read inside this tile's list and key
   // range even if the workspace was never filled.
-  const int cnt = min(max(P.count[t.tile_id], 0), t.nkt);
+  const int cnt = list_count(P, t);
   const int* list = P.list + t.tile_id * P.nkt_max;
   volatile int* abort = &sm.abort;
   constexpr uint32_t kTileBytes = kTile * D * 2;
@@ -819,7 +819,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         if (i >= kOutStages &&
             !mbar_wait(&empty[s], ((i / kOutStages) - 1) & 1, abort, P.status))
           break;
-        const int row = krow0 + clamp_kt(list[i], t.nkt) * kTile;
+        const int row = krow0 + list_tile(P, list, i, t.nkt) * kTile;
         mbar_expect_tx(&full[s], kTileBytes);
         for (int h = 0; h < D / 64; ++h)
           tma_load_2d(ring[s] + h * kTile * 64, map, &full[s], h * 64, row);
@@ -884,7 +884,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     for (int i = 0; i < cnt; ++i) {
       const int b = i & 1;
-      const int kt = clamp_kt(list[i], t.nkt);
+      const int kt = list_tile(P, list, i, t.nkt);
       if (!mbar_wait(&sm.s_full[b], (i >> 1) & 1, abort, P.status)) break;
       // P[b] is free once the PV product of step i-2 has completed
       if (i >= 2 && !mbar_wait(&sm.p_free[b], ((i >> 1) - 1) & 1, abort, P.status)) break;
@@ -989,10 +989,11 @@ struct UnionWalk {
   const int* la;
   const int* lb;
   int na, nb, ia, ib, nkt;
+  int all;  // no block mask: both lists are 0, 1, ..., nkt - 1
   __device__ __forceinline__ bool next(int& kt, bool& in_a, bool& in_b) {
     if (ia >= na && ib >= nb) return false;
-    const int a = ia < na ? clamp_kt(la[ia], nkt) : INT_MAX;
-    const int b = ib < nb ? clamp_kt(lb[ib], nkt) : INT_MAX;
+    const int a = ia < na ? (all ? ia : clamp_kt(la[ia], nkt)) : INT_MAX;
+    const int b = ib < nb ? (all ? ib : clamp_kt(lb[ib], nkt)) : INT_MAX;
     kt = min(a, b);
     in_a = a == kt;
     in_b = b == kt;
@@ -1016,8 +1017,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (!ta.valid) return;
   const TileInfo tb = map_tile(P, slot, 2 * blockIdx.y + 1, blockIdx.z);
   // Lists from the tau pass, clamped so that no workspace content sends a read outside them.
-  const int cnt_a = min(max(P.count[ta.tile_id], 0), ta.nkt);
-  const int cnt_b = min(max(P.count[tb.tile_id], 0), tb.nkt);
+  const int cnt_a = list_count(P, ta);
+  const int cnt_b = list_count(P, tb);
   const int* list_a = P.list + ta.tile_id * P.nkt_max;
   const int* list_b = P.list + tb.tile_id * P.nkt_max;
   volatile int* abort = &sm.abort;
@@ -1066,7 +1067,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tma_load_2d(sm.q[1] + h * kTile * 64, &tmq, &sm.q_full, h * 64, qb);
         }
       }
-      UnionWalk walk{list_a, list_b, cnt_a, cnt_b, 0, 0, ta.nkt};
+      UnionWalk walk{list_a, list_b, cnt_a, cnt_b, 0, 0, ta.nkt, P.no_mask};
       int kt;
       bool in_a, in_b;
       int issued = 0;
@@ -1117,7 +1118,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                  (first && k16 == 0) ? 0u : 1u);
       };
       bool ok = mbar_wait(&sm.q_full, 0, abort, P.status);
-      UnionWalk walk{list_a, list_b, cnt_a, cnt_b, 0, 0, ta.nkt};
+      UnionWalk walk{list_a, list_b, cnt_a, cnt_b, 0, 0, ta.nkt, P.no_mask};
       int kt;
       bool cur_a = false, cur_b = false;
       bool more = walk.next(kt, cur_a, cur_b);
@@ -1179,7 +1180,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t sx = tmem + lane_off + static_cast<uint32_t>(x * 128);
     for (int i = 0; i < cnt; ++i) {
-      const int kt = clamp_kt(list[i], t.nkt);
+      const int kt = list_tile(P, list, i, t.nkt);
       if (!mbar_wait(&sm.s_full[x], i & 1, abort, P.status)) break;
       tc_fence_after();
 #pragma unroll

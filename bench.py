@@ -301,13 +301,18 @@ def run_native(args, rank, world, local):
     out, tau, mask = ea.alloc_outputs(qd, kd, cud)
     ws = ea.alloc_workspace(qd, kd, cud)
 
+    from adaptive_sparse_attention_b200 import _native
+    nm = args.no_block_mask
+    flags = _native.FLAG_NO_BLOCK_MASK if nm else 0
+
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, stream=stream)
+        ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, flags=flags,
+                    stream=stream)
         if ev:
             ev[1].record(stream)
-        ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, stream=stream)
+        ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, flags=flags, stream=stream)
         if ev:
             ev[2].record(stream)
 
@@ -335,11 +340,14 @@ def run_native(args, rank, world, local):
     st = ea.status(stream)
     assert st == 0, f"device status {st}"
 
+    if nm:  # the mask, for the effective FLOP count only: one masked tau pass, not timed
+        ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, stream=stream)
+        torch.cuda.synchronize()
     bits = ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, cu)
     act_pairs, dense_pairs = count_pairs(w, bits, cu)
     eff_flops = 4 * w.d * act_pairs
     tau_flops = 2 * w.d * dense_pairs
-    out_flops = 4 * w.d * act_pairs
+    out_flops = 4 * w.d * (dense_pairs if nm else act_pairs)  # the work the output pass does
     tokens = w.B * w.T * w.Hq if cu is None else w.T * w.Hq  # query rows (token x head)
     tokens_seq = w.B * w.T if cu is None else w.T
     value = world * eff_flops / (ms_step * 1e-3) / 1e12
@@ -347,12 +355,20 @@ def run_native(args, rank, world, local):
     # end to end through the C ABI entry point: H2D of q, k, v from pinned host memory, the
     # forward pass, D2H of out, every step
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+
+    def fwd():
+        if nm:
+            ea.entmax_attn_fwd_no_block_mask(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau,
+                                             stream=stream)
+        else:
+            ea.entmax_attn_fwd(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau, mask,
+                               stream=stream)
+
     outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e2e_steps = max(2, min(args.steps, 5))
     for _ in range(1):
         qd.copy_(qh, non_blocking=True)
-        ea.entmax_attn_fwd(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau, mask,
-                           stream=stream)
+        fwd()
         outh.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
@@ -362,8 +378,7 @@ def run_native(args, rank, world, local):
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        ea.entmax_attn_fwd(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau, mask,
-                           stream=stream)
+        fwd()
         outh.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -394,7 +409,8 @@ def run_native(args, rank, world, local):
                 "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "peak_source": peak_note,
                 "algorithmic": ("2 d flops per causally valid pair (dense scores)" if dom_tau
-                                else "4 d flops per valid pair inside active tiles")}
+                                else ("4 d flops per causally valid pair (every tile)" if nm
+                                      else "4 d flops per valid pair inside active tiles"))}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -410,6 +426,7 @@ def run_native(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": dict(workload_config(w, world),
+                       variant="no_block_mask" if nm else "block_mask",
                        l2=f"inputs {in_bytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB L2; "
                           f"no flush" if in_bytes > L2_BYTES else "inputs fit in L2; no flush"),
         "tokens_per_s": world * tokens_seq / (ms_step * 1e-3),
@@ -443,6 +460,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline figure")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-block-mask", action="store_true",
+                    help="time the variant without block mask (output pass over every causal "
+                         "tile); the effective FLOPs keep counting active tiles only")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -75,6 +75,11 @@ extern "C" {
 #define ENTMAX_ATTN_FLAG_CUDA_CORES 1u    /* run BF16 products on the CUDA cores too */
 #define ENTMAX_ATTN_FLAG_ALL_FALLBACK 2u  /* send every query tile through the multi-sweep tau
                                              search that handles candidate-buffer overflow */
+#define ENTMAX_ATTN_FLAG_NO_BLOCK_MASK 8u /* the variant without block mask (AdaSplash page,
+                                             "adasplash_no_block_mask"): the tau pass writes no
+                                             mask and no tile lists (block_mask may be NULL), and
+                                             the output pass visits every causally valid key tile.
+                                             Give it to both passes. */
 #define ENTMAX_ATTN_FLAG_TEST_STALL 4u    /* test hook of the bounded waits: the tensor-core tau
                                              pass never requests its query tiles, so each of its
                                              CTAs gives up after one wait limit (about 2 s) and
@@ -99,6 +104,15 @@ size_t entmax_attn_mask_words(int B, int Hq, int T, int has_cu_seqlens);
  * Returns ENTMAX_ATTN_OK or ENTMAX_ATTN_EINVAL. */
 int entmax_attn_mask_layout(int B, int Hq, int T, int has_cu_seqlens, int* tiles_per_head,
                             int* words_per_tile);
+
+/* The full forward pass without the block mask: tau search, then the output pass over every
+ * causally valid key tile (the pages' "adasplash_no_block_mask" variant).  The same out and tau as
+ * entmax_attn_fwd (key tiles whose p are all zero add nothing), no mask written, workspace
+ * handled as in entmax_attn_fwd.  Returns ENTMAX_ATTN_OK or an error code. */
+int entmax_attn_fwd_no_block_mask(const void* q, const void* k, const void* v, void* out,
+                                  float* tau, int B, int Hq, int Hkv, int T, int d, float alpha,
+                                  int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                                  cudaStream_t stream);
 
 /* Two-pass form, for callers that own the scratch memory or time the passes apart.
  * workspace: device memory of at least entmax_attn_workspace_bytes(...) bytes, 256-byte

@@ -129,6 +129,29 @@ def test_argument_errors_are_reported_before_any_launch(native, case):
                              a["Hkv"], a["T"], a["d"], a["alpha"], a["n_iter"], a["causal"],
                              None, a["dtype"], None)
     assert rc == native.EINVAL
+    rc = lib.entmax_attn_fwd_no_block_mask(_fake(a["q"]) if a["q"] else None, _fake(0x2000),
+                                           _fake(0x3000), _fake(0x5000), _fake(0x6000), a["B"],
+                                           a["Hq"], a["Hkv"], a["T"], a["d"], a["alpha"],
+                                           a["n_iter"], a["causal"], None, a["dtype"], None)
+    assert rc == native.EINVAL
+
+
+def test_block_mask_is_required_unless_the_variant_says_otherwise(native):
+    """A NULL block_mask is an argument error of the masked passes; with
+    ENTMAX_ATTN_FLAG_NO_BLOCK_MASK the same call passes the argument checks (it then needs a
+    device, so only the misaligned workspace below is seen)."""
+    lib = native.lib()
+    rc = lib.entmax_attn_tau_pass(_fake(0x1000), _fake(0x2000), _fake(0x3000), None,
+                                  _fake(0x10000), 1 << 40, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
+                                  0, None)
+    assert rc == native.EINVAL
+    rc = lib.entmax_attn_fwd(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x5000),
+                             _fake(0x6000), None, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1, None)
+    assert rc == native.EINVAL
+    rc = lib.entmax_attn_tau_pass(_fake(0x1000), _fake(0x2000), _fake(0x3000), None,
+                                  _fake(0x10010), 1 << 40, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
+                                  native.FLAG_NO_BLOCK_MASK, None)
+    assert rc == native.EALIGN
 
 
 def test_misaligned_pointers_are_rejected(native):
