@@ -528,6 +528,7 @@ struct SweepSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int kind;  // what the current round over the tile does (row max, search step, mask bits)
 };
 
 template <int D, int BK>
@@ -557,6 +558,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
+    sm.kind = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int w = tid; w < kMaxWords; w += kTauThreads) sm.words[w] = 0u;
@@ -565,7 +567,6 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const int nsweep = P.n_iter + 2;
   int g = 0;       // key-tile steps so far in this CTA (identical in every role)
   int tcount = 0;  // tiles so far (phase of q_full)
   int issued_total = 0;
@@ -575,83 +576,88 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     if (id < 0 || id >= ntiles) continue;  // uniform across the block
     const TileInfo t = map_tile(P, id % P.slots, (id / P.slots) % P.Hq, id / (P.slots * P.Hq));
     const int nkt = t.nkt;
-    const int total = nsweep * nkt;
-    if (warp == kTauTmaWarp) {
-      if (lane == 0) {
-        const int krow0 = static_cast<int>(t.khead + t.seq_start);
-        for (int u = 0; u < total; ++u) {
-          const int gg = g + u, s = gg % kTauStages;
-          if (gg >= kTauStages &&
-              !mbar_wait(&sm.k_empty[s], ((gg / kTauStages) - 1) & 1, abort, P.status))
-            break;
-          mbar_expect_tx(&sm.k_full[s], kTileBytes);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
-                        krow0 + (u % nkt) * kTile);
-          issued_total = gg + 1;
-        }
-      }
-    } else if (warp == kTauMmaWarp) {
-      if (lane == 0) {
-        constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
-        bool ok = mbar_wait(&sm.q_full, tcount & 1, abort, P.status);
-        for (int u = 0; ok && u < total; ++u) {
-          const int gg = g + u, s = gg % kTauStages, b = gg % kTauSBufs;
-          if (!mbar_wait(&sm.k_full[s], (gg / kTauStages) & 1, abort, P.status)) break;
-          if (gg >= kTauSBufs &&
-              !mbar_wait(&sm.s_empty[b], ((gg / kTauSBufs) - 1) & 1, abort, P.status))
-            break;
-          tc_fence_after();
-          const uint32_t kbase = smem_u32(sm.k[s]);
+    const int quarter = warp & 3;
+    const int seg = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const bool valid = r < t.nrows;
+    const int jmax = valid ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+    Search sr;  // score warps: the row's search
+    int steps_done = 0;
+    if (warp < kTauScoreWarps) {  // this thread's quarter of its query row into TMEM
+      constexpr int kWords = D / 8;
+      uint32_t w[kWords];
+      if (valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            static_cast<const __nv_bfloat16*>(P.q) + (t.qhead + t.seq_start + t.row0 + r) * D +
+            seg * (D / 4));
 #pragma unroll
-          for (int k16 = 0; k16 < D / 16; ++k16)
-            mma_ts(tmem + static_cast<uint32_t>(b * 128), tmem + kTauColQ + k16 * 8,
-                   kmajor_desc(kbase, kTile, k16), idesc, k16 > 0 ? 1u : 0u);
-          mma_commit(&sm.k_empty[s]);
-          mma_commit(&sm.s_full[b]);
-          issued_total = gg + 1;
+        for (int e = 0; e < kWords / 4; ++e) {
+          const uint4 u = src[e];
+          w[4 * e] = u.x;
+          w[4 * e + 1] = u.y;
+          w[4 * e + 2] = u.z;
+          w[4 * e + 3] = u.w;
         }
-      }
-    } else {  // score warps 0..15: every step of every sweep, even after an abort (barriers)
-      const int quarter = warp & 3;
-      const int seg = warp >> 2;
-      const int r = quarter * 32 + lane;
-      const bool valid = r < t.nrows;
-      const int jmax = valid ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
-      {  // this thread's quarter of its query row into TMEM
-        constexpr int kWords = D / 8;
-        uint32_t w[kWords];
-        if (valid) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              static_cast<const __nv_bfloat16*>(P.q) + (t.qhead + t.seq_start + t.row0 + r) * D +
-              seg * (D / 4));
+      } else {
 #pragma unroll
-          for (int e = 0; e < kWords / 4; ++e) {
-            const uint4 u = src[e];
-            w[4 * e] = u.x;
-            w[4 * e + 1] = u.y;
-            w[4 * e + 2] = u.z;
-            w[4 * e + 3] = u.w;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < kWords; ++e) w[e] = 0u;
-        }
-        tmem_st_words<kWords>(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTauColQ +
-                                  static_cast<uint32_t>(seg * kWords),
-                              w);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.q_full);
+        for (int e = 0; e < kWords; ++e) w[e] = 0u;
       }
-      Search sr;
+      tmem_st_words<kWords>(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kTauColQ +
+                                static_cast<uint32_t>(seg * kWords),
+                            w);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full);
       sr.init(0.f, 1, P.alpha);
-      for (int sw = 0; sw < nsweep; ++sw) {
-        float a0 = (sw == 0) ? -INFINITY : 0.f, a1 = 0.f, a2 = 0.f;
+    }
+    // One sweep of S over the tile's key range per round; what a round does (row max, one
+    // search step, mask bits) is decided by the score warps at the end of the round before and
+    // published in sm.kind behind a CTA barrier, so that every role runs the same rounds.  The
+    // search stops as soon as every row of the tile has settled (at most n_iter steps).
+    for (;;) {
+      const int kind = sm.kind;  // 0 row max, 1 search step, 2 mask bits
+      if (warp == kTauTmaWarp) {
+        if (lane == 0) {
+          const int krow0 = static_cast<int>(t.khead + t.seq_start);
+          for (int kt = 0; kt < nkt; ++kt) {
+            const int gg = g + kt, s = gg % kTauStages;
+            if (gg >= kTauStages &&
+                !mbar_wait(&sm.k_empty[s], ((gg / kTauStages) - 1) & 1, abort, P.status))
+              break;
+            mbar_expect_tx(&sm.k_full[s], kTileBytes);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
+                          krow0 + kt * kTile);
+            issued_total = gg + 1;
+          }
+        }
+      } else if (warp == kTauMmaWarp) {
+        if (lane == 0) {
+          constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+          bool ok = kind != 0 || mbar_wait(&sm.q_full, tcount & 1, abort, P.status);
+          for (int kt = 0; ok && kt < nkt; ++kt) {
+            const int gg = g + kt, s = gg % kTauStages, b = gg % kTauSBufs;
+            if (!mbar_wait(&sm.k_full[s], (gg / kTauStages) & 1, abort, P.status)) break;
+            if (gg >= kTauSBufs &&
+                !mbar_wait(&sm.s_empty[b], ((gg / kTauSBufs) - 1) & 1, abort, P.status))
+              break;
+            tc_fence_after();
+            const uint32_t kbase = smem_u32(sm.k[s]);
+#pragma unroll
+            for (int k16 = 0; k16 < D / 16; ++k16)
+              mma_ts(tmem + static_cast<uint32_t>(b * 128), tmem + kTauColQ + k16 * 8,
+                     kmajor_desc(kbase, kTile, k16), idesc, k16 > 0 ? 1u : 0u);
+            mma_commit(&sm.k_empty[s]);
+            mma_commit(&sm.s_full[b]);
+            issued_total = gg + 1;
+          }
+        }
+      } else {  // score warps 0..15: every step of the round, even after an abort (barriers)
+        float a0 = (kind == 0) ? -INFINITY : 0.f, a1 = 0.f, a2 = 0.f;
         const float tau = sr.tau;
         for (int kt = 0; kt < nkt; ++kt) {
-          const int gg = g + sw * nkt + kt, b = gg % kTauSBufs;
+          const int gg = g + kt, b = gg % kTauSBufs;
           const bool okw = __all_sync(
               full, !*abort && mbar_wait(&sm.s_full[b], (gg / kTauSBufs) & 1, abort, P.status));
           if (!okw) continue;
@@ -663,10 +669,10 @@ __global__ void __launch_bounds__(kTauThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.s_empty[b]);
-          if (sw == 0) {
+          if (kind == 0) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) a0 = fmaxf(a0, x[e]);
-          } else if (sw <= P.n_iter) {
+          } else if (kind == 1) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float y = P.c * x[e] - tau;
@@ -685,29 +691,50 @@ __global__ void __launch_bounds__(kTauThreads, 1)
             if (any) atomicOr(&sm.words[kt >> 5], 1u << (kt & 31));
           }
         }
-        if (sw == nsweep - 1) break;  // the mask sweep needs no combination
-        const int pb = sw & 1;
-        sm.part[pb][0][seg][r] = a0;
-        sm.part[pb][1][seg][r] = a1;
-        sm.part[pb][2][seg][r] = a2;
-        score_warps_sync();
-        float t0 = sm.part[pb][0][0][r], t1 = sm.part[pb][1][0][r], t2 = sm.part[pb][2][0][r];
+        int next = 3;  // done
+        if (kind != 2) {
+          const int pb = steps_done & 1;
+          sm.part[pb][0][seg][r] = a0;
+          sm.part[pb][1][seg][r] = a1;
+          sm.part[pb][2][seg][r] = a2;
+          score_warps_sync();
+          float t0 = sm.part[pb][0][0][r], t1 = sm.part[pb][1][0][r], t2 = sm.part[pb][2][0][r];
 #pragma unroll
-        for (int q2 = 1; q2 < kSeg; ++q2) {
-          if (sw == 0) {
-            t0 = fmaxf(t0, sm.part[pb][0][q2][r]);
+          for (int q2 = 1; q2 < kSeg; ++q2) {
+            if (kind == 0) {
+              t0 = fmaxf(t0, sm.part[pb][0][q2][r]);
+            } else {
+              t0 += sm.part[pb][0][q2][r];
+              t1 += sm.part[pb][1][q2][r];
+              t2 += sm.part[pb][2][q2][r];
+            }
+          }
+          if (kind == 0) {
+            sr.init(valid ? P.c * t0 : 0.f, valid ? jmax : 1, P.alpha);
+            // start from the tau the main pass found on the candidates it kept: a lower bound
+            // of the row's tau when finite, and inside the bracket either way
+            const float t_kept = valid ? P.tau[t.qhead + t.seq_start + t.row0 + r] : sr.lo;
+            if (t_kept > sr.lo && t_kept < sr.hi) sr.tau = t_kept;
+            next = 1;
           } else {
-            t0 += sm.part[pb][0][q2][r];
-            t1 += sm.part[pb][1][q2][r];
-            t2 += sm.part[pb][2][q2][r];
+            sr.step<BK>(t0, t1, t2, P.beta);
+            ++steps_done;
+            const bool busy = valid && !sr.settled();
+            next = (steps_done < P.n_iter && score_warps_any(busy)) ? 1 : 2;
           }
         }
-        if (sw == 0) sr.init(valid ? P.c * t0 : 0.f, valid ? jmax : 1, P.alpha);
-        else sr.step<BK>(t0, t1, t2, P.beta);
+        if (*abort) next = 3;
+        score_warps_sync();  // every score thread has read sm.kind of this round
+        if (tid == 0) sm.kind = next;
       }
-      if (seg == 0 && valid) P.tau[t.qhead + t.seq_start + t.row0 + r] = sr.tau;
+      g += nkt;
+      tc_fence_before();
+      __syncthreads();  // the next round's kind is published
+      tc_fence_after();
+      if (sm.kind == 3) break;
     }
-    g += total;
+    if (warp < kTauScoreWarps && seg == 0 && valid)
+      P.tau[t.qhead + t.seq_start + t.row0 + r] = sr.tau;
     ++tcount;
     tc_fence_before();
     __syncthreads();
@@ -715,6 +742,8 @@ __global__ void __launch_bounds__(kTauThreads, 1)
     if (!*abort && warp == 0) emit_tile(P, t, sm.words, 0, lane);
     __syncthreads();
     for (int w = tid; w < kMaxWords; w += kTauThreads) sm.words[w] = 0u;
+    if (tid == 0) sm.kind = 0;
+    __syncthreads();
   }
   // drain: issued copies have landed and issued MMAs have completed before TMEM is released
   if (warp == kTauTmaWarp && lane == 0) {
