@@ -5,7 +5,8 @@
 //                        list.  The path for fp32 inputs.
 //   tau_fallback_kernel  the multi-sweep search for query tiles whose candidate buffers
 //                        overflowed: one sweep for the row max, one per search step over all
-//                        valid keys, one for the mask bits.  Any dtype.
+//                        valid keys (from the main pass's tau, until every row has settled),
+//                        one for the mask bits.  Any dtype.
 //   out_simt_kernel      output pass on the CUDA cores over the listed key tiles.
 //
 // One CTA of 128 threads per query tile, thread r owning row r of the tile.  The query tile
@@ -184,7 +185,13 @@ __global__ void __launch_bounds__(kThreads) tau_fallback_kernel(Problem P) {
     const int n = row_ok ? (P.causal ? pos + 1 : t.seq_len) : 1;
     Search sr;
     sr.init(mz, n, P.alpha);
+    {  // start from the tau the main pass found on the candidates it kept (inside the bracket)
+      const float t_kept = row_ok ? P.tau[t.qhead + t.seq_start + pos] : sr.lo;
+      if (t_kept > sr.lo && t_kept < sr.hi) sr.tau = t_kept;
+    }
     for (int it = 0; it < P.n_iter; ++it) {
+      // stop once every row of the tile has settled (uniform across the block)
+      if (it > 0 && !__syncthreads_or(row_ok && !sr.settled())) break;
       const float tau = sr.tau;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f;
       sweep_keys<T, D>(P, t, sm, tid, [&](int) {
