@@ -128,6 +128,27 @@ def entmax_attn_fwd_no_block_mask(q, k, v, alpha: float = 1.5, n_iter: int = 10,
     return out, tau
 
 
+def entmax_rows(x, alpha: float = 1.5, n_iter: int = 10, out=None, tau=None, stream=None):
+    """Row-wise alpha-entmax over the last dimension of x (fp32 or bf16, contiguous rows).
+    Returns (p, tau): p like x, tau fp32 with x's leading shape."""
+    if x.dtype not in _DT:
+        raise TypeError("x must be float32 or bfloat16")
+    if x.dim() < 1 or x.numel() == 0 or x.stride(-1) != 1:
+        raise ValueError("x needs a non-empty, unit-stride last dimension")
+    n = x.shape[-1]
+    x2 = x.reshape(-1, n)  # a view when the rows have one stride, else a contiguous copy
+    rows = x2.shape[0]
+    p = (torch.empty((rows, n), dtype=x.dtype, device=x.device) if out is None
+         else out.view(rows, n))
+    if p.stride(1) != 1 or p.dtype != x.dtype:
+        raise ValueError("out must have x's dtype and unit-stride rows")
+    t = torch.empty(rows, dtype=torch.float32, device=x.device) if tau is None else tau.view(rows)
+    rc = N.lib().entmax_attn_rows(_ptr(x2), x2.stride(0), _ptr(p), p.stride(0), _ptr(t), rows, n,
+                                  float(alpha), int(n_iter), _DT[x.dtype], _stream(stream))
+    N.check(rc, "entmax_attn_rows")
+    return p.reshape(x.shape), t.reshape(x.shape[:-1])
+
+
 def entmax_attn_fwd_noalloc(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool = True,
                             cu_seqlens=None, out=None, tau=None, block_mask=None, stream=None):
     """Forward pass through the allocation-free entry point: the library's scratch is a fixed

@@ -309,6 +309,23 @@ int fwd_cached(const void* q, const void* k, const void* v, void* out, float* ta
 
 }  // namespace
 
+int entmax_attn_rows(const void* x, long long ldx, void* p, long long ldp, float* tau, int rows,
+                     int n, float alpha, int n_iter, int dtype, cudaStream_t stream) {
+  if (!x || !p || rows < 1 || n < 1 || ldx < n || ldp < n || !(alpha > 1.f) ||
+      !std::isfinite(alpha) ||
+      n_iter < 1 || (dtype != ENTMAX_ATTN_FP32 && dtype != ENTMAX_ATTN_BF16))
+    return ENTMAX_ATTN_EINVAL;
+  const uintptr_t esz = dtype == ENTMAX_ATTN_FP32 ? 4u : 2u;
+  if ((reinterpret_cast<uintptr_t>(x) % esz) || (reinterpret_cast<uintptr_t>(p) % esz) ||
+      (reinterpret_cast<uintptr_t>(tau) & 3u))
+    return ENTMAX_ATTN_EALIGN;
+  cudaError_t e = ea::launch_entmax_rows(x, static_cast<int64_t>(ldx), p,
+                                         static_cast<int64_t>(ldp), tau, rows, n, alpha, n_iter,
+                                         dtype, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ENTMAX_ATTN_OK;
+}
+
 int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
                     uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
                     int n_iter, int causal, const int32_t* cu_seqlens, int dtype,

@@ -145,20 +145,23 @@ __device__ __forceinline__ float entmax_p(float x, float beta) {
 // State of the bracketed Halley + bisection search for one row: the iterate, the bracket, and
 // the lengths of the last two steps.
 struct Search {
-  float tau, lo, hi, dx, dxold;
+  float tau, lo, hi, dx, dxold, m;
 
   // p_max <= 1 gives tau >= m - 1; n keys all at most m give tau <= m - n^(1 - alpha).
-  __device__ __forceinline__ void init(float m, int n, float alpha) {
+  __device__ __forceinline__ void init(float m_, int n, float alpha) {
+    m = m_;
     lo = m - 1.f;
     hi = m - exp2f((1.f - alpha) * __log2f((float)n));
     tau = lo;
     dx = dxold = hi - lo;
   }
 
-  // True once the last step moved tau by no more than rounding: later steps can then only move
+  // True once the last step moved tau by no more than rounding, measured against the larger of
+  // |tau| (what fp32 can resolve) and m - tau (the size of the differences z - tau that p is
+  // made of, small for long near-uniform rows when alpha > 2): later steps can then only move
   // it by a few ulps.
   __device__ __forceinline__ bool settled() const {
-    return dx <= 4.f * FLT_EPSILON * fmaxf(1.f, fabsf(tau));
+    return dx <= 4.f * FLT_EPSILON * fmaxf(fabsf(tau), m - tau);
   }
 
   // One step, given the sums over the keys with z > tau of (z - tau)^beta, ^(beta-1) and

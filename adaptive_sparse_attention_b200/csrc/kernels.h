@@ -18,6 +18,12 @@ cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s);
 cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t s);
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s);
 
+// Row-wise alpha-entmax of a [rows, n] matrix x (row stride ldx elements) into p (row stride
+// ldp); dtype 0 = fp32, 1 = bf16 for both x and p; tau may be null.
+cudaError_t launch_entmax_rows(const void* x, int64_t ldx, void* p, int64_t ldp, float* tau,
+                               int rows, int n, float alpha, int n_iter, int dtype,
+                               cudaStream_t s);
+
 inline int beta_kind(float beta) {
   return beta == 1.f ? kBetaOne : (beta == 2.f ? kBetaTwo : kBetaGeneral);
 }

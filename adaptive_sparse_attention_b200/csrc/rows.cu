@@ -1,0 +1,99 @@
+// rows.cu -- standalone row-wise alpha-entmax (AdaSplash page, "Triton Entmax (Optimized Entmax
+// Activation)"): for every row x of a matrix, p = [(alpha - 1) x - tau]_+^(1/(alpha - 1)) with
+// tau such that sum(p) = 1, found by the same bracketed Halley + bisection search as the
+// attention kernels' tau pass (Search in common.cuh), stopping early once tau has settled.
+// One warp per row; the row is re-read from global memory (L1) at every search step, so any
+// row length works.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ea {
+namespace {
+
+constexpr int kRowsPerCta = 8;
+
+template <typename T, int BK>
+__global__ void __launch_bounds__(32 * kRowsPerCta)
+    entmax_rows_kernel(const T* __restrict__ x, int64_t ldx, T* __restrict__ p, int64_t ldp,
+                       float* __restrict__ tau, int rows, int n, float alpha, float beta,
+                       int n_iter) {
+  const int row = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;  // whole warps leave together
+  const T* xr = x + row * ldx;
+  T* pr = p + row * ldp;
+  const float am1 = alpha - 1.f;
+  const unsigned full = 0xffffffffu;
+  float m = -INFINITY;
+  for (int j = lane; j < n; j += 32) m = fmaxf(m, load_elem(xr, j));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(full, m, o));
+  Search sr;
+  sr.init(am1 * m, n, alpha);
+  for (int it = 0; it < n_iter; ++it) {
+    const float t = sr.tau;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+    for (int j = lane; j < n; j += 32) {
+      const float y = am1 * load_elem(xr, j) - t;
+      if (y > 0.f) {
+        float a, b, c;
+        entmax_powers<BK>(y, beta, a, b, c);
+        s0 += a;
+        s1 += b;
+        s2 += c;
+      }
+    }
+    // butterfly sums: every lane ends with the same bits (fp32 addition commutes), so every
+    // lane takes the same step and the loop exit below is uniform
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s0 += __shfl_xor_sync(full, s0, o);
+      s1 += __shfl_xor_sync(full, s1, o);
+      s2 += __shfl_xor_sync(full, s2, o);
+    }
+    sr.step<BK>(s0, s1, s2, beta);
+    if (sr.settled()) break;
+  }
+  const float t = sr.tau;
+  for (int j = lane; j < n; j += 32)
+    store_elem(pr, j, entmax_p<BK>(am1 * load_elem(xr, j) - t, beta));
+  if (tau && lane == 0) tau[row] = t;
+}
+
+template <typename T>
+cudaError_t launch_rows_t(const void* x, int64_t ldx, void* p, int64_t ldp, float* tau, int rows,
+                          int n, float alpha, int n_iter, cudaStream_t s) {
+  const float beta = 1.f / (alpha - 1.f);
+  const dim3 grid((rows + kRowsPerCta - 1) / kRowsPerCta);
+  const dim3 block(32 * kRowsPerCta);
+  const T* xp = static_cast<const T*>(x);
+  T* pp = static_cast<T*>(p);
+  switch (beta_kind(beta)) {
+    case kBetaOne:
+      entmax_rows_kernel<T, kBetaOne><<<grid, block, 0, s>>>(xp, ldx, pp, ldp, tau, rows, n,
+                                                             alpha, beta, n_iter);
+      break;
+    case kBetaTwo:
+      entmax_rows_kernel<T, kBetaTwo><<<grid, block, 0, s>>>(xp, ldx, pp, ldp, tau, rows, n,
+                                                             alpha, beta, n_iter);
+      break;
+    default:
+      entmax_rows_kernel<T, kBetaGeneral><<<grid, block, 0, s>>>(xp, ldx, pp, ldp, tau, rows,
+                                                                 n, alpha, beta, n_iter);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_entmax_rows(const void* x, int64_t ldx, void* p, int64_t ldp, float* tau,
+                               int rows, int n, float alpha, int n_iter, int dtype,
+                               cudaStream_t s) {
+  return dtype == 0
+             ? launch_rows_t<float>(x, ldx, p, ldp, tau, rows, n, alpha, n_iter, s)
+             : launch_rows_t<__nv_bfloat16>(x, ldx, p, ldp, tau, rows, n, alpha, n_iter, s);
+}
+
+}  // namespace ea

@@ -138,6 +138,18 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
  * overflow path.  Synchronises `stream`.  Returns -1 on a CUDA error. */
 int entmax_attn_fallback_tiles(const void* workspace, cudaStream_t stream);
 
+/* Row-wise alpha-entmax (AdaSplash page, "Triton Entmax (Optimized Entmax Activation)"): for every
+ * row x of the [rows, n] matrix at `x` (row stride `ldx` elements, ldx >= n),
+ *   p = [(alpha - 1) x - tau]_+^(1/(alpha - 1)),  tau such that sum(p) = 1,
+ * written to the [rows, n] matrix at `p` (row stride `ldp` >= n), tau found by n_iter steps
+ * (fewer once it has settled) of the bracketed Halley + bisection search of the attention passes.
+ * x and p have the same dtype (ENTMAX_ATTN_FP32 or ENTMAX_ATTN_BF16) and may not overlap; tau
+ * (fp32 [rows]) may be NULL.  Device pointers, aligned to their element size; asynchronous on
+ * `stream`.  Returns ENTMAX_ATTN_OK, ENTMAX_ATTN_EINVAL (rows or n < 1, ldx or ldp < n, alpha <= 1
+ * or not finite, n_iter < 1, bad dtype, null x or p), ENTMAX_ATTN_EALIGN or ENTMAX_ATTN_ECUDA. */
+int entmax_attn_rows(const void* x, long long ldx, void* p, long long ldp, float* tau, int rows,
+                     int n, float alpha, int n_iter, int dtype, cudaStream_t stream);
+
 /* Synchronises `stream`, returns the device status word of the current device
  * (ENTMAX_ATTN_OK or ENTMAX_ATTN_ETIMEOUT) and clears it. */
 int entmax_attn_status(cudaStream_t stream);

@@ -154,6 +154,38 @@ def test_block_mask_is_required_unless_the_variant_says_otherwise(native):
     assert rc == native.EALIGN
 
 
+@pytest.mark.parametrize("case", ["rows0", "n0", "ldx_small", "ldp_small", "alpha1", "niter0",
+                                  "dtype", "null_x", "misaligned"])
+def test_rows_argument_errors(native, case):
+    lib = native.lib()
+    a = dict(x=0x1000, p=0x2000, tau=0x3000, rows=4, n=8, ldx=8, ldp=8, alpha=1.5, n_iter=10,
+             dtype=0)
+    want = native.EINVAL
+    if case == "rows0":
+        a["rows"] = 0
+    elif case == "n0":
+        a["n"] = 0
+    elif case == "ldx_small":
+        a["ldx"] = 7
+    elif case == "ldp_small":
+        a["ldp"] = 7
+    elif case == "alpha1":
+        a["alpha"] = 1.0
+    elif case == "niter0":
+        a["n_iter"] = 0
+    elif case == "dtype":
+        a["dtype"] = 5
+    elif case == "null_x":
+        a["x"] = 0
+    elif case == "misaligned":
+        a["p"] = 0x2002
+        want = native.EALIGN
+    rc = lib.entmax_attn_rows(_fake(a["x"]) if a["x"] else None, a["ldx"], _fake(a["p"]), a["ldp"],
+                              _fake(a["tau"]), a["rows"], a["n"], a["alpha"], a["n_iter"],
+                              a["dtype"], None)
+    assert rc == want
+
+
 def test_misaligned_pointers_are_rejected(native):
     lib = native.lib()
     rc = lib.entmax_attn_tau_pass(_fake(0x1008), _fake(0x2000), _fake(0x3000), _fake(0x4000),
