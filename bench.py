@@ -183,13 +183,31 @@ def dist_setup(args):
     return rank, world, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op: str, device: str) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest of the ranks' x (times: the job ends with its slowest rank)."""
+    return _reduce(x, world, "max", device)
+
+
+def sum_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The sum of the ranks' x (work: each rank solves its own problem)."""
+    return _reduce(x, world, "sum", device)
+
+
+def job_rate(units_per_rank: float, ms_per_rank: float, world: int, device: str = "cuda") -> float:
+    """Whole-job throughput in units per second: the units of all ranks over the slowest rank's
+    time (weak scaling: every rank runs a full problem of its own)."""
+    units = sum_over_ranks(units_per_rank, world, device)
+    ms = max_over_ranks(ms_per_rank, world, device)
+    return units / (ms * 1e-3)
 
 
 def barrier(world):
@@ -350,7 +368,7 @@ def run_native(args, rank, world, local):
     out_flops = 4 * w.d * (dense_pairs if nm else act_pairs)  # the work the output pass does
     tokens = w.B * w.T * w.Hq if cu is None else w.T * w.Hq  # query rows (token x head)
     tokens_seq = w.B * w.T if cu is None else w.T
-    value = world * eff_flops / (ms_step * 1e-3) / 1e12
+    value = job_rate(eff_flops, total_ms / args.steps, world) / 1e12
 
     # end to end through the C ABI entry point: H2D of q, k, v from pinned host memory, the
     # forward pass, D2H of out, every step
@@ -382,7 +400,10 @@ def run_native(args, rank, world, local):
         outh.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_one = e0.elapsed_time(e1) / e2e_steps
+    e2e_ms = max_over_ranks(e2e_one, world)
+    e2e_rate = job_rate(eff_flops, e2e_one, world)
+    dense_rate = job_rate(4 * w.d * dense_pairs, total_ms / args.steps, world)
     assert ea.status(stream) == 0
 
     if rank != 0:
@@ -432,7 +453,7 @@ def run_native(args, rank, world, local):
         "tokens_per_s": world * tokens_seq / (ms_step * 1e-3),
         "query_rows_per_s": world * tokens / (ms_step * 1e-3),
         "frac_of_bf16_peak": value / world / bf16_peak,
-        "dense_equiv_tflops": world * 4 * w.d * dense_pairs / (ms_step * 1e-3) / 1e12,
+        "dense_equiv_tflops": dense_rate / 1e12,
         "active_tile_pair_fraction": act_pairs / dense_pairs,
         "ms_tau_pass": mean_tau, "ms_out_pass": mean_out,
         "tau_pass_hbm_gbs": (q.numel() * q.element_size() + k.numel() * k.element_size()
@@ -440,7 +461,7 @@ def run_native(args, rank, world, local):
         "overflow_tiles": nfb,
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * eff_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": e2e_rate / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": out.numel() * out.element_size()},
         "gpu_launches": 3 * args.steps,
