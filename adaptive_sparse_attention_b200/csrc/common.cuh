@@ -207,6 +207,7 @@ struct alignas(16) CandSmem {
   int cnt[kCols];
   int lost[kCols];
   uint32_t words[kMaxWords];
+  int wbase[kMaxWords];  // list position of each mask word's first active key tile
   int fallback;         // some row of the tile needs the overflow path
 };
 
@@ -562,6 +563,47 @@ __device__ __forceinline__ void emit_tile(const Problem& P, const TileInfo& t,
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (lane == 0) P.count[t.tile_id] = base;
+}
+
+// emit_tile split over many threads, in two phases with a barrier of those threads between:
+// phase 1 (one warp): the overflow queue or the list position of every mask word and the count;
+// phase 2 (all nthreads threads): the mask words and one list entry per set bit.
+__device__ __forceinline__ void emit_tile_prefix(const Problem& P, const TileInfo& t,
+                                                 CandSmem& cs, int lane) {
+  if (cs.fallback) {
+    if (lane == 0) {
+      const int i = atomicAdd(P.queue_count, 1);
+      P.queue[i] = (int)t.tile_id;
+    }
+    return;
+  }
+  if (P.no_mask) return;
+  int base = 0;
+  for (int w0 = 0; w0 < P.W; w0 += 32) {
+    const int w = w0 + lane;
+    const int c = (w < P.W) ? __popc(cs.words[w]) : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (w < P.W) cs.wbase[w] = base + incl - c;
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) P.count[t.tile_id] = base;
+}
+__device__ __forceinline__ void emit_tile_entries(const Problem& P, const TileInfo& t,
+                                                  const CandSmem& cs, int tid, int nthreads) {
+  if (cs.fallback || P.no_mask) return;
+  uint32_t* mw = P.mask + t.tile_id * P.W;
+  int* list = P.list + t.tile_id * P.nkt_max;
+  for (int w = tid; w < P.W; w += nthreads) mw[w] = cs.words[w];
+  for (int i = tid; i < P.W * 32; i += nthreads) {
+    const uint32_t bits = cs.words[i >> 5];
+    const uint32_t bit = 1u << (i & 31);
+    if (bits & bit) list[cs.wbase[i >> 5] + __popc(bits & (bit - 1u))] = i;
+  }
 }
 
 // A compact-list entry forced into [0, nkt): out-of-range values (an unfilled workspace) read

@@ -462,9 +462,12 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         emit_empty(P, t, tid, kScoreThreads);
         continue;
       }
-      // per-tile shared state; warp 0 cleared the mask words and the flag after its last emit
+      // per-tile shared state: the row max now; the mask words and the overflow flag, which the
+      // previous tile's emit read, once every score thread has passed the barrier below
       if (tid < kTile) cs.rowmax[tid] = -INFINITY;  // warps 0..3: thread tid owns row tid
       score_warps_sync();
+      if (tid < kMaxWords) cs.words[tid] = 0u;
+      if (tid == 0) cs.fallback = P.force_fallback;
       const int nkt = t.nkt, warm = warm_tiles(nkt), nsteps = nkt + warm;
       const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
       RowCand rc;
@@ -493,12 +496,9 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       if (score_warps_any(*abort != 0)) break;  // status already records the timeout
       solve_rows<BK>(P, t, cs, tid, kScoreThreads);
       score_warps_sync();
-      if (warp == 0) {
-        emit_tile(P, t, cs.words, cs.fallback, lane);
-        __syncwarp();
-        for (int w = lane; w < kMaxWords; w += 32) cs.words[w] = 0u;
-        if (lane == 0) cs.fallback = P.force_fallback;
-      }
+      if (warp == 0) emit_tile_prefix(P, t, cs, lane);
+      score_warps_sync();
+      emit_tile_entries(P, t, cs, tid, kScoreThreads);
     }
   }
   tc_fence_before();
