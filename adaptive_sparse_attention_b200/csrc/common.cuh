@@ -21,9 +21,9 @@ namespace ea {
 constexpr int kTile = 128;      // query-tile rows and key-tile keys (block-mask granularity)
 constexpr int kSeg = 4;         // key segments per row (keys 32 g .. 32 g + 31 of every key tile),
                                 // each with its own running max and candidate buffer
-constexpr int kCand = 16;       // candidate slots per (row, segment) held in shared memory
+constexpr int kCand = 16;       // candidate slots per (row, segment) held in shared memory: the
+                                // default; kernels with shared memory to spare take more
 constexpr int kCols = kSeg * kTile;  // (row, segment) columns of the candidate buffers
-static_assert(kCand % 4 == 0, "the solve splits a buffer over 4 lanes");
 constexpr int kXchWarps = 16;  // warps feeding candidates per CTA (one exchange row each)
 constexpr int kExchangeMax = 2;  // up to this many passing rows of a warp go through the exchange row
 constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
@@ -192,15 +192,19 @@ struct Search {
 };
 
 // ---------------------------------------------------------------------------------------------
-// Candidate buffers: for every (row r, segment g) -- column c = g * 128 + r -- up to kCand
+// Candidate buffers: for every (row r, segment g) -- column c = g * 128 + r -- up to NC
 // (raw score, key tile) pairs in shared memory, entry e at [e * kCols + c], so that the 32 rows
 // of a warp hit 32 distinct banks whatever their fill levels.  A segment owns the keys 32 g ..
 // 32 g + 31 of every key tile.
 // ---------------------------------------------------------------------------------------------
-struct alignas(16) CandSmem {
+template <int NC>
+struct alignas(16) CandSmemT {
+  static_assert(NC % 4 == 0, "the solve splits a buffer over 4 lanes");
+  static_assert(NC <= 32, "at most one candidate slot per lane in the cooperative insertion");
+  static constexpr int kSlots = NC;
   float xrow[kXchWarps][32];  // per-warp exchange rows of feed_warp (first: 16-byte aligned)
-  float s[kCand * kCols];
-  uint16_t kt[kCand * kCols];
+  float s[NC * kCols];
+  uint16_t kt[NC * kCols];
   float rowmax[kTile];  // running max of the row over all segments (raw); see feed_warp
   float m[kCols];       // segment max of raw scores
   float floor_[kCols];  // pruning floor (raw); -inf when the segment was never pruned
@@ -210,6 +214,7 @@ struct alignas(16) CandSmem {
   int wbase[kMaxWords];  // list position of each mask word's first active key tile
   int fallback;         // some row of the tile needs the overflow path
 };
+using CandSmem = CandSmemT<kCand>;
 
 // max of three floats in one instruction
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -266,7 +271,8 @@ struct RowCand {
     lost = 0;
   }
 
-  __device__ __forceinline__ void publish(CandSmem& cs, int col) const {
+  template <class CS>
+  __device__ __forceinline__ void publish(CS& cs, int col) const {
     cs.m[col] = m;
     cs.floor_[col] = floor_;
     cs.cnt[col] = cnt;
@@ -274,17 +280,17 @@ struct RowCand {
   }
 };
 
-static_assert(kCand <= 32, "at most one candidate slot per lane in the cooperative insertion");
 
 // Insertion of the passing values of one lane (src, buffer column col_src) when they do not fit
 // into its buffer.  Lane e < c0 holds old entry e, lane j holds value j of src's chunk (v).
-// Old entries and new values at or below the threshold th are dropped; if more than kCand
-// survive, the floor is raised by bisection to just above the (kCand/2 + 1)-th largest value,
-// so that the kCand/2 largest survive and the buffer has room again (entries below the floor
+// Old entries and new values at or below the threshold th are dropped; if more than the buffer's
+// slots survive, the floor is raised by bisection to just above the (slots/2 + 1)-th largest
+// value, so that the slots/2 largest survive and the buffer has room again (entries below the floor
 // can only matter if tau ends up at or below it, which the solve checks).  Survivors -- old ones
 // first, then new ones in key order -- are written to the front of the buffer.  Warp-uniform
 // arguments; call with the whole warp converged.
-__device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, int col_src,
+template <class CS>
+__device__ __forceinline__ void coop_insert(CS& cs, RowCand& rc, int src, int col_src,
                                             float v, float th, int c0, int kt, int lane) {
   const unsigned full = 0xffffffffu;
   float fl = __shfl_sync(full, rc.floor_, src);
@@ -294,9 +300,9 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   const uint16_t ko = have ? cs.kt[lane * kCols + col_src] : static_cast<uint16_t>(0);
   unsigned bo = __ballot_sync(full, vo > th);
   unsigned bn = __ballot_sync(full, v > th);
-  if (__popc(bo) + __popc(bn) > kCand) {
+  if (__popc(bo) + __popc(bn) > CS::kSlots) {
     // Bisection on [th, mm] keeps "more than kKeep above lo, at most kKeep above hi".
-    constexpr int kKeep = kCand / 2;
+    constexpr int kKeep = CS::kSlots / 2;
     float lo = th, hi = mm;
     for (int it = 0; it < 24; ++it) {
       const float mid = 0.5f * (lo + hi);
@@ -324,15 +330,15 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
   }
   if ((bn >> lane) & 1u) {
     const int at = no + __popc(bn & below);
-    if (at < kCand) {
+    if (at < CS::kSlots) {
       cs.s[at * kCols + col_src] = v;
       cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
     }
   }
   if (lane == src) {
     const int total = no + nn;
-    rc.cnt = min(total, kCand);
-    if (total > kCand) rc.lost = 1;  // only when ties at the floor could not be separated
+    rc.cnt = min(total, CS::kSlots);
+    if (total > CS::kSlots) rc.lost = 1;  // only when ties at the floor could not be separated
     rc.thr = th;
     rc.floor_ = fl;
   }
@@ -349,8 +355,8 @@ __device__ __forceinline__ void coop_insert(CandSmem& cs, RowCand& rc, int src, 
 // the row has published in cs.rowmax[row]: a lower bound of the row's max, so every key with
 // z > (row max) - 1 is still kept, while records of one segment's max no longer trigger
 // insertions in the others.  A stale or overwritten rowmax value only loosens the threshold.
-template <int N>
-__device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, float* xrow, int col,
+template <int N, class CS>
+__device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int col,
                                           int row, int lane, const float (&x)[N], int kt) {
   static_assert(N == 32, "one value per lane in the exchange row");
   const unsigned full = 0xffffffffu;
@@ -378,7 +384,7 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, float* xrow
     int incoming = 0;
 #pragma unroll
     for (int i = 0; i < N; ++i) incoming += (x[i] > rc.thr) ? 1 : 0;  // branch-free count
-    const bool fits = pass && rc.cnt + incoming <= kCand;
+    const bool fits = pass && rc.cnt + incoming <= CS::kSlots;
     if (fits) {
       int c = rc.cnt;
       const uint16_t kt16 = static_cast<uint16_t>(kt);
@@ -409,7 +415,7 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, float* xrow
     const int col_src = col - lane + src;
     const unsigned take = __ballot_sync(full, v > th);
     const int n = __popc(take);
-    if (c0 + n <= kCand) {
+    if (c0 + n <= CS::kSlots) {
       if ((take >> lane) & 1u) {
         const int at = c0 + __popc(take & below);
         cs.s[at * kCols + col_src] = v;
@@ -426,8 +432,8 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CandSmem& cs, float* xrow
 // Takes 32 raw scores of a key tile into the row's running max without inserting candidates
 // (the keys are fed again later): raises the segment max, the row max shared with the other
 // segments and the threshold.
-template <int N>
-__device__ __forceinline__ void observe_max(RowCand& rc, CandSmem& cs, int row,
+template <int N, class CS>
+__device__ __forceinline__ void observe_max(RowCand& rc, CS& cs, int row,
                                             const float (&x)[N]) {
   static_assert(N == 32, "32-key chunks");
   const float cmax = fmaxf(max16(x, 0), max16(x, 16));
@@ -446,8 +452,8 @@ __device__ __forceinline__ void observe_max(RowCand& rc, CandSmem& cs, int row,
 // lanes that split a row's candidates and combine their partial sums with warp shuffles.
 // nthreads must be a multiple of 32; call from all threads of the block after a
 // __syncthreads() that follows publish().
-template <int BK>
-__device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, int tid,
+template <int BK, class CS>
+__device__ void solve_rows(const Problem& P, const TileInfo& t, CS& cs, int tid,
                            int nthreads) {
   const int lane4 = tid & 3;
   const int groups = nthreads >> 2;
@@ -467,11 +473,11 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
     const int n = valid ? (P.causal ? pos + 1 : t.seq_len) : 1;
     // this lane's share of the row's candidates (raw scores; -inf in empty slots), held in
     // registers for all search steps
-    float raw[kSeg][kCand / 4];
+    float raw[kSeg][CS::kSlots / 4];
 #pragma unroll
     for (int g = 0; g < kSeg; ++g) {
 #pragma unroll
-      for (int i = 0; i < kCand / 4; ++i) {
+      for (int i = 0; i < CS::kSlots / 4; ++i) {
         const int e = lane4 + 4 * i;
         raw[g][i] = (e < cnt[g]) ? cs.s[e * kCols + g * kTile + r] : -INFINITY;
       }
@@ -484,7 +490,7 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
 #pragma unroll
       for (int g = 0; g < kSeg; ++g) {
 #pragma unroll
-        for (int i = 0; i < kCand / 4; ++i) {
+        for (int i = 0; i < CS::kSlots / 4; ++i) {
           const float x = P.c * raw[g][i] - tau;
           if (x > 0.f) {
             float a, b, c2;
@@ -517,7 +523,7 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CandSmem& cs, in
 #pragma unroll
     for (int g = 0; g < kSeg; ++g) {
 #pragma unroll
-      for (int i = 0; i < kCand / 4; ++i) {
+      for (int i = 0; i < CS::kSlots / 4; ++i) {
         if (P.c * raw[g][i] > tau) {
           const int kt = cs.kt[(lane4 + 4 * i) * kCols + g * kTile + r];
           atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
@@ -568,8 +574,9 @@ __device__ __forceinline__ void emit_tile(const Problem& P, const TileInfo& t,
 // emit_tile split over many threads, in two phases with a barrier of those threads between:
 // phase 1 (one warp): the overflow queue or the list position of every mask word and the count;
 // phase 2 (all nthreads threads): the mask words and one list entry per set bit.
-__device__ __forceinline__ void emit_tile_prefix(const Problem& P, const TileInfo& t,
-                                                 CandSmem& cs, int lane) {
+template <class CS>
+__device__ __forceinline__ void emit_tile_prefix(const Problem& P, const TileInfo& t, CS& cs,
+                                                 int lane) {
   if (cs.fallback) {
     if (lane == 0) {
       const int i = atomicAdd(P.queue_count, 1);
@@ -593,8 +600,9 @@ __device__ __forceinline__ void emit_tile_prefix(const Problem& P, const TileInf
   }
   if (lane == 0) P.count[t.tile_id] = base;
 }
+template <class CS>
 __device__ __forceinline__ void emit_tile_entries(const Problem& P, const TileInfo& t,
-                                                  const CandSmem& cs, int tid, int nthreads) {
+                                                  const CS& cs, int tid, int nthreads) {
   if (cs.fallback || P.no_mask) return;
   uint32_t* mw = P.mask + t.tile_id * P.W;
   int* list = P.list + t.tile_id * P.nkt_max;

@@ -295,7 +295,7 @@ template <int D>
 struct TauSmem {
   alignas(1024) __nv_bfloat16 q[kTile * D];
   alignas(1024) __nv_bfloat16 k[kMainStages][kTile * D];
-  CandSmem cand;
+  CandSmemT<(D == 64 ? 32 : kCand)> cand;  // d = 64 leaves room for twice the candidates
   uint64_t q_full;
   uint64_t q_empty;
   uint64_t k_full[kMainStages];
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   TauSmem<D>& sm = *reinterpret_cast<TauSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  CandSmem& cs = sm.cand;
+  auto& cs = sm.cand;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int per_slot = P.Hq * (P.cu ? 1 : P.B);
