@@ -280,7 +280,16 @@ __device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&w
 
 // The tau kernel keeps Q in shared memory so that TMEM holds four 128-column score buffers: the
 // score warps may fall three key tiles behind the MMA during a burst of insertions.
-constexpr int kMainStages = 4;  // key tiles in flight
+// Candidate slots and key stages of the tau kernel.  d = 64 leaves shared memory for 32 slots
+// beside four key stages.  At d = 128, alpha other than 1.5 and 2 (the general power, e.g. 1.333)
+// keeps hundreds of keys within 1 of a row's max, so its rows take 28 slots at the price of one
+// key stage; alpha 1.5 and 2 keep 16 slots and four stages.
+__host__ __device__ constexpr int tau_slots(int d, int bk) {
+  return d == 64 ? 32 : (bk == kBetaGeneral ? 28 : kCand);
+}
+__host__ __device__ constexpr int tau_stages(int d, int bk) {
+  return (d == 128 && bk == kBetaGeneral) ? 3 : 4;
+}
 constexpr int kMainSBufs = 4;   // TMEM score buffers
 
 // Key-tile order of the tau pass.  Until a row's running max has seen a few hundred keys, its
@@ -291,15 +300,16 @@ constexpr int kMainSBufs = 4;   // TMEM score buffers
 __device__ __forceinline__ int warm_tiles(int nkt) { return nkt >= 32 ? 8 : (nkt >= 16 ? 4 : 0); }
 __device__ __forceinline__ int step_tile(int i, int nkt) { return i < nkt ? i : i - nkt; }
 
-template <int D>
+template <int D, int BK>
 struct TauSmem {
+  static constexpr int kStages = tau_stages(D, BK);
   alignas(1024) __nv_bfloat16 q[kTile * D];
-  alignas(1024) __nv_bfloat16 k[kMainStages][kTile * D];
-  CandSmemT<(D == 64 ? 32 : kCand)> cand;  // d = 64 leaves room for twice the candidates
+  alignas(1024) __nv_bfloat16 k[kStages][kTile * D];
+  CandSmemT<tau_slots(D, BK)> cand;
   uint64_t q_full;
   uint64_t q_empty;
-  uint64_t k_full[kMainStages];
-  uint64_t k_empty[kMainStages];
+  uint64_t k_full[kStages];
+  uint64_t k_empty[kStages];
   uint64_t s_full[kMainSBufs];
   uint64_t s_empty[kMainSBufs];
   uint64_t drain;
@@ -335,8 +345,9 @@ template <int D, int BK>
 __global__ void __launch_bounds__(kTauThreads, 1)
     tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   Problem P) {
+  constexpr int kStages = TauSmem<D, BK>::kStages;
   extern __shared__ unsigned char smem_raw[];
-  TauSmem<D>& sm = *reinterpret_cast<TauSmem<D>*>(
+  TauSmem<D, BK>& sm = *reinterpret_cast<TauSmem<D, BK>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   auto& cs = sm.cand;
   const int tid = threadIdx.x;
@@ -349,7 +360,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    for (int s = 0; s < kMainStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
     }
@@ -391,9 +402,9 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         ++it;
         const int nkt = t.nkt, nsteps = nkt + warm_tiles(nkt);
         for (int i = 0; i < nsteps; ++i, ++gk) {
-          const int s = gk % kMainStages;
-          if (gk >= kMainStages &&
-              !mbar_wait(&sm.k_empty[s], ((gk / kMainStages) - 1) & 1, abort, P.status)) {
+          const int s = gk % kStages;
+          if (gk >= kStages &&
+              !mbar_wait(&sm.k_empty[s], ((gk / kStages) - 1) & 1, abort, P.status)) {
             ok = false;
             break;
           }
@@ -404,8 +415,8 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         }
       }
       // drain: every issued copy has landed before the CTA may exit
-      for (int g = (gk > kMainStages ? gk - kMainStages : 0); g < gk; ++g)
-        mbar_wait(&sm.k_full[g % kMainStages], (g / kMainStages) & 1, abort, P.status);
+      for (int g = (gk > kStages ? gk - kStages : 0); g < gk; ++g)
+        mbar_wait(&sm.k_full[g % kStages], (g / kStages) & 1, abort, P.status);
       if (it > 0) mbar_wait(&sm.q_full, (it - 1) & 1, abort, P.status);
     }
   } else if (warp == kTauMmaWarp) {
@@ -424,8 +435,8 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         ++it;
         const int nsteps = t.nkt + warm_tiles(t.nkt);
         for (int i = 0; i < nsteps; ++i, ++gk) {
-          const int s = gk % kMainStages, b = gk % kMainSBufs;
-          if (!mbar_wait(&sm.k_full[s], (gk / kMainStages) & 1, abort, P.status) ||
+          const int s = gk % kStages, b = gk % kMainSBufs;
+          if (!mbar_wait(&sm.k_full[s], (gk / kStages) & 1, abort, P.status) ||
               (gk >= kMainSBufs &&
                !mbar_wait(&sm.s_empty[b], ((gk / kMainSBufs) - 1) & 1, abort, P.status))) {
             ok = false;
@@ -1319,7 +1330,7 @@ cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
   cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
   if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(TauSmem<D>) + 1024;
+  const size_t smem = sizeof(TauSmem<D, BK>) + 1024;
   auto kern = tau_tc_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
