@@ -28,7 +28,10 @@ constexpr int kXchWarps = 16;  // warps feeding candidates per CTA (one exchange
 constexpr int kExchangeMax = 2;  // up to this many passing rows of a warp go through the exchange row
 constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
 
-enum BetaKind { kBetaOne = 0, kBetaTwo = 1, kBetaGeneral = 2 };
+// beta = 1 and 2 have exact closed forms; kBetaNear3 is beta within kNearIntFrac of 3 (alpha
+// near 4/3, e.g. the fp32 value of 1.333: beta = 3.003); the rest is general.
+enum BetaKind { kBetaOne = 0, kBetaTwo = 1, kBetaGeneral = 2, kBetaNear3 = 3 };
+constexpr float kNearIntFrac = 0.004f;
 
 // Everything a kernel needs; passed by value.
 struct Problem {
@@ -117,6 +120,16 @@ __device__ __forceinline__ void store_elem(__nv_bfloat16* p, int64_t i, float x)
   p[i] = __float2bfloat16_rn(x);
 }
 
+// For beta = 3 + f with |f| <= kNearIntFrac: x^f = exp(f ln x) by its second-order Taylor
+// polynomial in l = f ln x.  Every x the passes raise to beta lies in (0, 1] (tau >= m - 1), and
+// wherever x^beta >= 1e-16 (x >= 4e-6) |l| <= 0.05, so the relative error |l|^3 / 6 stays below
+// 2.2e-5; below that x^3 is itself under 1e-16 and the polynomial stays positive.  One
+// logarithm instead of the logarithm and exponential of exp2(beta log2 x).
+__device__ __forceinline__ float near_int_frac_pow(float x, float f) {
+  const float l = f * 0.69314718f * __log2f(x);
+  return fmaf(l, fmaf(0.5f, l, 1.f), 1.f);
+}
+
 // x^beta and the two lower powers needed by the Halley step, for x > 0.
 template <int BK>
 __device__ __forceinline__ void entmax_powers(float x, float beta, float& p0, float& p1,
@@ -125,6 +138,10 @@ __device__ __forceinline__ void entmax_powers(float x, float beta, float& p0, fl
     p0 = x; p1 = 1.f; p2 = 0.f;
   } else if (BK == kBetaTwo) {
     p0 = x * x; p1 = x; p2 = 1.f;
+  } else if (BK == kBetaNear3) {
+    p2 = x * near_int_frac_pow(x, beta - 3.f);
+    p1 = p2 * x;
+    p0 = p1 * x;
   } else {
     p0 = exp2f(beta * __log2f(x));
     const float inv = __frcp_rn(x);
@@ -139,7 +156,19 @@ __device__ __forceinline__ float entmax_p(float x, float beta) {
   if (!(x > 0.f)) return 0.f;
   if (BK == kBetaOne) return x;
   if (BK == kBetaTwo) return x * x;
+  if (BK == kBetaNear3) return (x * x) * (x * near_int_frac_pow(x, beta - 3.f));
   return exp2f(beta * __log2f(x));
+}
+
+// [x]_+^beta without a branch on the sign of x: the same values as entmax_p (x <= 0 gives 0:
+// max(x, 0) is 0, and log2(0) = -inf sends exp2 to 0).
+template <int BK>
+__device__ __forceinline__ float entmax_p_clamped(float x, float beta) {
+  const float y = fmaxf(x, 0.f);
+  if (BK == kBetaOne) return y;
+  if (BK == kBetaTwo) return y * y;
+  if (BK == kBetaNear3) return (y * y) * (y * near_int_frac_pow(fmaxf(y, 1e-30f), beta - 3.f));
+  return exp2f(beta * __log2f(y));
 }
 
 // State of the bracketed Halley + bisection search for one row: the iterate, the bracket, and

@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <cmath>
+
 #include "common.cuh"
 
 namespace ea {
@@ -25,7 +27,10 @@ cudaError_t launch_entmax_rows(const void* x, int64_t ldx, void* p, int64_t ldp,
                                cudaStream_t s);
 
 inline int beta_kind(float beta) {
-  return beta == 1.f ? kBetaOne : (beta == 2.f ? kBetaTwo : kBetaGeneral);
+  if (beta == 1.f) return kBetaOne;
+  if (beta == 2.f) return kBetaTwo;
+  if (fabsf(beta - 3.f) <= kNearIntFrac) return kBetaNear3;
+  return kBetaGeneral;
 }
 
 }  // namespace ea

@@ -79,6 +79,10 @@ cudaError_t launch_rows_t(const void* x, int64_t ldx, void* p, int64_t ldp, floa
       entmax_rows_kernel<T, kBetaTwo><<<grid, block, 0, s>>>(xp, ldx, pp, ldp, tau, rows, n,
                                                              alpha, beta, n_iter);
       break;
+    case kBetaNear3:
+      entmax_rows_kernel<T, kBetaNear3><<<grid, block, 0, s>>>(xp, ldx, pp, ldp, tau, rows,
+                                                                 n, alpha, beta, n_iter);
+      break;
     default:
       entmax_rows_kernel<T, kBetaGeneral><<<grid, block, 0, s>>>(xp, ldx, pp, ldp, tau, rows,
                                                                  n, alpha, beta, n_iter);

@@ -228,6 +228,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// p of 32 consecutive keys j0 .. j0 + 31 of a row from their raw scores (TMEM words u), packed
+// as bf16 pairs; keys at or past jmax (the row's causal / sequence end) give 0.  Rows whose 32
+// keys are all valid -- every tile but the diagonal one -- skip the per-key range test.
+template <int BK>
+__device__ __forceinline__ void p_row32(const uint32_t (&u)[32], float c, float tau, float beta,
+                                        int j0, int jmax, uint32_t (&pk)[16]) {
+  if (j0 + 32 <= jmax) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float p0 = entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e]) - tau, beta);
+      const float p1 = entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e + 1]) - tau, beta);
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float p0 = (j0 + 2 * e < jmax)
+                           ? entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e]) - tau, beta)
+                           : 0.f;
+      const float p1 = (j0 + 2 * e + 1 < jmax)
+                           ? entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e + 1]) - tau, beta)
+                           : 0.f;
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+  }
+}
+
 // Descriptor of a K-major 128B-swizzled operand tile of R rows whose d columns sit in 64-column
 // halves of R x 128 bytes; k16 selects the 16-column (32-byte) slice of the K dimension.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int rows, int k16) {
@@ -285,10 +312,10 @@ __device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&w
 // keeps hundreds of keys within 1 of a row's max, so its rows take 28 slots at the price of one
 // key stage; alpha 1.5 and 2 keep 16 slots and four stages.
 __host__ __device__ constexpr int tau_slots(int d, int bk) {
-  return d == 64 ? 32 : (bk == kBetaGeneral ? 28 : kCand);
+  return d == 64 ? 32 : (bk >= kBetaGeneral ? 28 : kCand);
 }
 __host__ __device__ constexpr int tau_stages(int d, int bk) {
-  return (d == 128 && bk == kBetaGeneral) ? 3 : 4;
+  return (d == 128 && bk >= kBetaGeneral) ? 3 : 4;
 }
 constexpr int kMainSBufs = 4;   // TMEM score buffers
 
@@ -935,14 +962,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + kColS + b * 128 + c0, u);
         uint32_t pk[16];
-        const int j0 = kt * kTile + c0;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float s0 = __uint_as_float(u[2 * e]), s1 = __uint_as_float(u[2 * e + 1]);
-          const float p0 = (j0 + 2 * e < jmax) ? entmax_p<BK>(P.c * s0 - tau, P.beta) : 0.f;
-          const float p1 = (j0 + 2 * e + 1 < jmax) ? entmax_p<BK>(P.c * s1 - tau, P.beta) : 0.f;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
+        p_row32<BK>(u, P.c, tau, P.beta, kt * kTile + c0, jmax, pk);
         tmem_st16(tmem + lane_off + kColP + b * 64 + c0 / 2, pk);
       }
       tmem_wait_st();
@@ -1229,14 +1249,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         uint32_t u[32];
         tmem_ld32(sx + static_cast<uint32_t>(c0), u);
         uint32_t pk[16];
-        const int j0 = kt * kTile + c0;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float s0 = __uint_as_float(u[2 * e]), s1 = __uint_as_float(u[2 * e + 1]);
-          const float p0 = (j0 + 2 * e < jmax) ? entmax_p<BK>(P.c * s0 - tau, P.beta) : 0.f;
-          const float p1 = (j0 + 2 * e + 1 < jmax) ? entmax_p<BK>(P.c * s1 - tau, P.beta) : 0.f;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
+        p_row32<BK>(u, P.c, tau, P.beta, kt * kTile + c0, jmax, pk);
         // keys c0 .. c0 + 31 as 16 packed columns over S columns this warp has already read
         tmem_st16(sx + static_cast<uint32_t>(half * 64 + q2 * 16), pk);
       }
@@ -1391,10 +1404,12 @@ cudaError_t launch_out_pair_t(const Problem& P, cudaStream_t s) {
     if (P.d == 64) {                                                \
       if (bk == kBetaOne) return FN<64, kBetaOne>(P, s);            \
       if (bk == kBetaTwo) return FN<64, kBetaTwo>(P, s);            \
+      if (bk == kBetaNear3) return FN<64, kBetaNear3>(P, s);    \
       return FN<64, kBetaGeneral>(P, s);                            \
     }                                                               \
     if (bk == kBetaOne) return FN<128, kBetaOne>(P, s);             \
     if (bk == kBetaTwo) return FN<128, kBetaTwo>(P, s);             \
+    if (bk == kBetaNear3) return FN<128, kBetaNear3>(P, s);     \
     return FN<128, kBetaGeneral>(P, s);                             \
   } while (0)
 
@@ -1407,10 +1422,12 @@ cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t 
   if (P.d == 64) {
     if (bk == kBetaOne) return launch_sweep_t<64, kBetaOne>(P, num_ctas, s);
     if (bk == kBetaTwo) return launch_sweep_t<64, kBetaTwo>(P, num_ctas, s);
+    if (bk == kBetaNear3) return launch_sweep_t<64, kBetaNear3>(P, num_ctas, s);
     return launch_sweep_t<64, kBetaGeneral>(P, num_ctas, s);
   }
   if (bk == kBetaOne) return launch_sweep_t<128, kBetaOne>(P, num_ctas, s);
   if (bk == kBetaTwo) return launch_sweep_t<128, kBetaTwo>(P, num_ctas, s);
+  if (bk == kBetaNear3) return launch_sweep_t<128, kBetaNear3>(P, num_ctas, s);
   return launch_sweep_t<128, kBetaGeneral>(P, num_ctas, s);
 }
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) {
