@@ -32,6 +32,7 @@ SIGNATURES = {
     "entmax_attn_mask_layout": (_c_int, [_c_int, _c_int, _c_int, _c_int,
                                          ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "entmax_attn_workspace_bytes": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
+    "entmax_attn_workspace_min_bytes": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "entmax_attn_tau_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),

@@ -83,6 +83,11 @@ def workspace_bytes(B, Hq, T, packed: bool) -> int:
     return int(N.lib().entmax_attn_workspace_bytes(B, Hq, T, int(packed)))
 
 
+def workspace_min_bytes(B, Hq, T, packed: bool) -> int:
+    """The smallest workspace the passes accept (the tau pass then runs without warm-up keys)."""
+    return int(N.lib().entmax_attn_workspace_min_bytes(B, Hq, T, int(packed)))
+
+
 def alloc_outputs(q, k, cu_seqlens):
     B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
     packed = cu_seqlens is not None

@@ -33,6 +33,9 @@ struct Layout {
   int W;          // mask words per query tile
   int nkt_max;    // longest compact list
   int64_t tiles;  // query tiles over all (batch, head)
+  int warm_levels;       // warm-up key levels per key group
+  int64_t norm_rows;     // key rows with a norm slot (Hq bounds Hkv)
+  int64_t warm_bytes;    // warm-up tiles of every key group at d = 128
 };
 
 bool make_layout(int B, int Hq, int T, int has_cu, Layout* L) {
@@ -44,16 +47,22 @@ bool make_layout(int B, int Hq, int T, int has_cu, Layout* L) {
   L->W = static_cast<int>((nt + 31) / 32);
   L->nkt_max = static_cast<int>(nt);
   L->tiles = (has_cu ? 1 : static_cast<int64_t>(B)) * Hq * slots;
+  L->warm_levels = ea::warm_levels_for(T);
+  L->norm_rows = (has_cu ? 1 : static_cast<int64_t>(B)) * Hq * T;
+  L->warm_bytes = static_cast<int64_t>(B) * Hq * L->warm_levels * ea::kTile * 128 * 2;
   return L->tiles < (int64_t(1) << 31);
 }
 
-// Workspace: [queue_count | count[tiles] | queue[tiles] | list[tiles][nkt_max]], each section
-// 256-byte aligned.
+// Workspace: [queue_count | count[tiles] | queue[tiles] | list[tiles][nkt_max] | key norms |
+// warm-up tiles], each section 256-byte aligned.
 struct WsView {
   int* queue_count;
   int* count;
   int* queue;
   int* list;
+  float* norms;
+  void* warm;
+  size_t min_bytes;  // without the warm-up sections
   size_t bytes;
 };
 
@@ -69,6 +78,11 @@ WsView ws_view(void* base, const Layout& L) {
   off += align256(sizeof(int) * L.tiles);
   v.list = reinterpret_cast<int*>(p + off);
   off += align256(sizeof(int) * static_cast<size_t>(L.tiles) * L.nkt_max);
+  v.min_bytes = off;  // everything past here is the tau pass's warm-up keys
+  v.norms = reinterpret_cast<float*>(p + off);
+  off += align256(sizeof(float) * static_cast<size_t>(L.norm_rows));
+  v.warm = p + off;
+  off += align256(static_cast<size_t>(L.warm_bytes));
   v.bytes = off;
   return v;
 }
@@ -154,6 +168,8 @@ void attach_workspace(ea::Problem* P, const WsView& v) {
   P->count = v.count;
   P->queue = v.queue;
   P->queue_count = v.queue_count;
+  P->norms = v.norms;
+  P->warm = v.warm;
 }
 
 bool use_tensor_cores(int dtype, unsigned flags) {
@@ -191,6 +207,12 @@ size_t entmax_attn_workspace_bytes(int B, int Hq, int T, int has_cu_seqlens) {
   return ws_view(nullptr, L).bytes;
 }
 
+size_t entmax_attn_workspace_min_bytes(int B, int Hq, int T, int has_cu_seqlens) {
+  Layout L;
+  if (!make_layout(B, Hq, T, has_cu_seqlens != 0, &L)) return 0;
+  return ws_view(nullptr, L).min_bytes;
+}
+
 int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
                          void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
                          int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
@@ -206,7 +228,7 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return ENTMAX_ATTN_EALIGN;
   const WsView v = ws_view(workspace, L);
-  if (workspace_bytes < v.bytes) return ENTMAX_ATTN_ENOMEM;
+  if (workspace_bytes < v.min_bytes) return ENTMAX_ATTN_ENOMEM;
   int err = ENTMAX_ATTN_OK;
   P.status = status_ptr(&err);
   if (!P.status) return err;
@@ -219,6 +241,11 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
 
   cudaError_t e = cudaMemsetAsync(v.queue_count, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (use_tensor_cores(dtype, flags) && workspace_bytes >= v.bytes) {
+    P.warm_levels = L.warm_levels;
+    e = ea::launch_warm(P, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   e = use_tensor_cores(dtype, flags) ? ea::launch_tau_tc(P, stream)
                                      : ea::launch_tau_simt(P, dtype, stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -248,7 +275,7 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return ENTMAX_ATTN_EALIGN;
   const WsView wv = ws_view(const_cast<void*>(workspace), L);
-  if (workspace_bytes < wv.bytes) return ENTMAX_ATTN_ENOMEM;
+  if (workspace_bytes < wv.min_bytes) return ENTMAX_ATTN_ENOMEM;
   int err = ENTMAX_ATTN_OK;
   P.status = status_ptr(&err);
   if (!P.status) return err;

@@ -61,6 +61,11 @@ struct Problem {
   int test_stall;      // test hook: the tensor-core tau kernel never requests its query tile
   int no_mask;         // no block mask: the tau pass writes neither mask nor lists, and the
                        // output pass visits every causally valid key tile
+  // warm-up keys of the tensor-core tau pass (workspace; see warm_level)
+  float* norms;        // [kv rows] squared key norms
+  void* warm;          // [groups][warm_levels][128][d] bf16: per (batch or sequence, kv head)
+                       // and level, the 128 keys of largest norm of the level's key range
+  int warm_levels;     // levels per group; 0 = no warm-up keys
 };
 
 struct TileInfo {
@@ -75,6 +80,7 @@ struct TileInfo {
   int64_t qhead;    // row offset of this (batch, q head) in q / out / tau
   int64_t khead;    // row offset of this (batch, kv head) in k / v
   int64_t tile_id;  // (batch * Hq + h) * slots + slot
+  int grp;          // (batch or sequence) * Hkv + kv head: the key group of the tile
 };
 
 // Maps a (slot, head, batch) grid coordinate to its query tile.  For a packed batch, sequence s
@@ -89,6 +95,7 @@ __device__ __forceinline__ TileInfo map_tile(const Problem& P, int slot, int h, 
     t.qt = slot;
     t.qhead = ((int64_t)b * P.Hq + h) * P.T;
     t.khead = ((int64_t)b * P.Hkv + h / P.G) * P.T;
+    t.grp = b * P.Hkv + h / P.G;
   } else {
     int lo = 0, hi = P.B - 1;
     while (lo < hi) {
@@ -101,6 +108,7 @@ __device__ __forceinline__ TileInfo map_tile(const Problem& P, int slot, int h, 
     t.qt = slot - (P.cu[lo] / kTile + lo);
     t.qhead = (int64_t)h * P.T;
     t.khead = (int64_t)(h / P.G) * P.T;
+    t.grp = lo * P.Hkv + h / P.G;
   }
   const int nqt = (t.seq_len + kTile - 1) / kTile;
   t.valid = (t.qt >= 0 && t.qt < nqt);
@@ -109,6 +117,25 @@ __device__ __forceinline__ TileInfo map_tile(const Problem& P, int slot, int h, 
   t.nkt = P.causal ? t.qt + 1 : nqt;
   t.tile_id = ((int64_t)b * P.Hq + h) * P.slots + slot;
   return t;
+}
+
+// Warm-up keys.  A row's candidate threshold is (running max) - 1/c, and it is loose until the
+// running max has met the row's largest scores; keys of large norm are the likeliest to give
+// them.  So for every key group and level j the library keeps the 128 keys of largest norm among
+// the group's first 1024 * 2^j keys, and the tau pass starts each query tile with one product
+// against the widest level inside the keys that every row of the tile may attend to (all keys
+// before the tile's first row when causal, the whole sequence otherwise).  Their scores are real
+// scores of the row, so their max is a lower bound of the row max and the threshold stays exact.
+constexpr int kWarmBase = 1024;  // keys in the range of level 0
+__host__ __device__ inline int warm_levels_for(int64_t n) {
+  int j = 0;
+  while ((static_cast<int64_t>(kWarmBase) << j) <= n) ++j;
+  return j;
+}
+// Level of a query tile's warm-up product, -1 for none.
+__device__ __forceinline__ int warm_level(const Problem& P, const TileInfo& t) {
+  const int prefix = P.causal ? t.row0 : t.seq_len;
+  return min(warm_levels_for(prefix), P.warm_levels) - 1;
 }
 
 __device__ __forceinline__ float load_elem(const float* p, int64_t i) { return p[i]; }
@@ -458,22 +485,23 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
   }
 }
 
-// Takes 32 raw scores of a key tile into the row's running max without inserting candidates
-// (the keys are fed again later): raises the segment max, the row max shared with the other
-// segments and the threshold.
+// Takes 32 scores of the warm-up keys (-inf for an unused row) into the row's threshold: the
+// chunk max, lowered by 1e-5 relative (and 1e-6 absolute) so that it stays below the same scores as the key tiles
+// give them whatever the rounding, raises the row max shared with the other segments and the
+// threshold.  The segment max (rc.m) is left to the key tiles themselves.
 template <int N, class CS>
-__device__ __forceinline__ void observe_max(RowCand& rc, CS& cs, int row,
-                                            const float (&x)[N]) {
+__device__ __forceinline__ void observe_bound(RowCand& rc, CS& cs, int row,
+                                              const float (&x)[N]) {
   static_assert(N == 32, "32-key chunks");
-  const float cmax = fmaxf(max16(x, 0), max16(x, 16));
-  rc.m = fmaxf(rc.m, cmax);
+  float b = fmaxf(max16(x, 0), max16(x, 16));
+  b = b - fabsf(b) * 1e-5f - 1e-6f;
   const float shared_max = *reinterpret_cast<volatile float*>(&cs.rowmax[row]);
-  const float mx = fmaxf(shared_max, cmax);
+  const float mx = fmaxf(shared_max, b);
   if (mx > rc.mx) {
     rc.mx = mx;
     rc.thr = fmaxf(rc.mx - rc.inv_c, rc.floor_);
   }
-  if (cmax > shared_max) cs.rowmax[row] = cmax;
+  if (b > shared_max) cs.rowmax[row] = b;
 }
 
 // Solves tau for every row of the tile from the published candidate buffers of both segments,

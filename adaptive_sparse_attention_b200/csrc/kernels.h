@@ -19,6 +19,8 @@ cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s);
 // Multi-sweep tau search on the tensor cores for the overflow queue (one CTA per SM at most).
 cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t s);
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s);
+// Warm-up keys of the tensor-core tau pass (P.norms, P.warm); nothing when P.warm_levels == 0.
+cudaError_t launch_warm(const Problem& P, cudaStream_t s);
 
 // Row-wise alpha-entmax of a [rows, n] matrix x (row stride ldx elements) into p (row stride
 // ldp); dtype 0 = fp32, 1 = bf16 for both x and p; tau may be null.

@@ -38,7 +38,7 @@ extern "C" int entmax_attn_fwd_noalloc(const void* q, const void* k, const void*
                                        int T, int d, float alpha, int n_iter, int causal,
                                        const int32_t* cu_seqlens, int dtype,
                                        cudaStream_t stream) {
-  const size_t need = entmax_attn_workspace_bytes(B, Hq, T, cu_seqlens != nullptr);
+  const size_t need = entmax_attn_workspace_min_bytes(B, Hq, T, cu_seqlens != nullptr);
   if (need == 0) return ENTMAX_ATTN_EINVAL;
   if (need > ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES) return ENTMAX_ATTN_ENOMEM;  // too large for it
 

@@ -319,13 +319,12 @@ __host__ __device__ constexpr int tau_stages(int d, int bk) {
 }
 constexpr int kMainSBufs = 4;   // TMEM score buffers
 
-// Key-tile order of the tau pass.  Until a row's running max has seen a few hundred keys, its
-// threshold is low and most scores are inserted as candidates, only to be dropped again later.
-// So the first w key tiles are first swept for the row max alone and fed as candidates once more
-// after the last tile; step i of the sweep handles key tile i (i < nkt) or i - nkt.  Costs w
-// extra Q K^T tiles; used when a row spans enough tiles for them to pay off.
-__device__ __forceinline__ int warm_tiles(int nkt) { return nkt >= 32 ? 8 : (nkt >= 16 ? 4 : 0); }
-__device__ __forceinline__ int step_tile(int i, int nkt) { return i < nkt ? i : i - nkt; }
+// Steps of a query tile in the tau pass: with a warm-up level (warm_level), step 0 is the
+// product with the level's 128 warm-up keys, which only raises the rows' thresholds; the key
+// tiles 0 .. nkt - 1 follow in order.
+__device__ __forceinline__ int warm_steps(const Problem& P, const TileInfo& t) {
+  return warm_level(P, t) >= 0 ? 1 : 0;
+}
 
 template <int D, int BK>
 struct TauSmem {
@@ -371,7 +370,7 @@ __device__ __forceinline__ TileInfo tau_tile(const Problem& P, int L, int per_sl
 template <int D, int BK>
 __global__ void __launch_bounds__(kTauThreads, 1)
     tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  Problem P) {
+                  const __grid_constant__ CUtensorMap tmw, Problem P) {
   constexpr int kStages = TauSmem<D, BK>::kStages;
   extern __shared__ unsigned char smem_raw[];
   TauSmem<D, BK>& sm = *reinterpret_cast<TauSmem<D, BK>*>(
@@ -427,7 +426,8 @@ __global__ void __launch_bounds__(kTauThreads, 1)
             tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
         }
         ++it;
-        const int nkt = t.nkt, nsteps = nkt + warm_tiles(nkt);
+        const int lvl = warm_level(P, t), ws = lvl >= 0 ? 1 : 0, nsteps = t.nkt + ws;
+        const int wrow = (t.grp * P.warm_levels + lvl) * kTile;
         for (int i = 0; i < nsteps; ++i, ++gk) {
           const int s = gk % kStages;
           if (gk >= kStages &&
@@ -436,9 +436,14 @@ __global__ void __launch_bounds__(kTauThreads, 1)
             break;
           }
           mbar_expect_tx(&sm.k_full[s], kTileBytes);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
-                        krow0 + step_tile(i, nkt) * kTile);
+          if (i < ws) {
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_2d(sm.k[s] + h * kTile * 64, &tmw, &sm.k_full[s], h * 64, wrow);
+          } else {
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
+                          krow0 + (i - ws) * kTile);
+          }
         }
       }
       // drain: every issued copy has landed before the CTA may exit
@@ -460,7 +465,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         if (!t.valid) continue;
         if (!mbar_wait(&sm.q_full, it & 1, abort, P.status)) break;
         ++it;
-        const int nsteps = t.nkt + warm_tiles(t.nkt);
+        const int nsteps = t.nkt + warm_steps(P, t);
         for (int i = 0; i < nsteps; ++i, ++gk) {
           const int s = gk % kStages, b = gk % kMainSBufs;
           if (!mbar_wait(&sm.k_full[s], (gk / kStages) & 1, abort, P.status) ||
@@ -506,13 +511,13 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       score_warps_sync();
       if (tid < kMaxWords) cs.words[tid] = 0u;
       if (tid == 0) cs.fallback = P.force_fallback;
-      const int nkt = t.nkt, warm = warm_tiles(nkt), nsteps = nkt + warm;
+      const int ws = warm_steps(P, t), nsteps = t.nkt + ws;
       const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
       RowCand rc;
       rc.init(1.f / P.c);
       for (int i = 0; i < nsteps; ++i, ++gs) {
         const int b = gs % kMainSBufs;
-        const int kt = step_tile(i, nkt);
+        const int kt = i - ws;  // -1: the warm-up keys
         // the warp leaves together: feed_warp needs all 32 lanes
         if (!__all_sync(0xffffffffu,
                         mbar_wait(&sm.s_full[b], (gs / kMainSBufs) & 1, abort, P.status)))
@@ -521,12 +526,15 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(b * 128 + seg * 32);
         float x[32];
-        tmem_row32(ta, kt * kTile + seg * 32, jmax, x);
+        if (kt < 0)  // every warm-up key is visible to every row of the tile
+          tmem_row32(ta, 0, r < t.nrows ? kTile : 0, x);
+        else
+          tmem_row32(ta, kt * kTile + seg * 32, jmax, x);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_empty[b]);  // scores are in registers: release S[b]
-        if (i < warm)
-          observe_max(rc, cs, r, x);
+        if (kt < 0)
+          observe_bound(rc, cs, r, x);
         else
           feed_warp<32>(rc, cs, cs.xrow[warp], col, r, lane, x, kt);
       }
@@ -1326,6 +1334,9 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int64_t rows, int d) {
 
 int64_t q_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) * P.Hq * P.T; }
 int64_t kv_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) * P.Hkv * P.T; }
+int64_t warm_rows(const Problem& P) {
+  return static_cast<int64_t>(P.B) * P.Hkv * P.warm_levels * kTile;
+}
 
 dim3 tile_grid(const Problem& P) { return dim3(P.slots, P.Hq, P.cu ? 1 : P.B); }
 
@@ -1339,9 +1350,13 @@ cudaError_t device_sms(int* sms) {
 
 template <int D, int BK>
 cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
-  CUtensorMap mq, mk;
+  CUtensorMap mq, mk, mw;
   cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
   if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
+  // warm-up tiles: [groups * levels * 128, d]; without them the map is never read
+  if (e == cudaSuccess)
+    e = P.warm_levels > 0 ? make_map(&mw, P.warm, warm_rows(P), D)
+                          : make_map(&mw, P.k, kv_rows(P), D);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(TauSmem<D, BK>) + 1024;
   auto kern = tau_tc_kernel<D, BK>;
@@ -1351,7 +1366,8 @@ cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
   e = device_sms(&sms);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = static_cast<int64_t>(P.slots) * P.Hq * (P.cu ? 1 : P.B);
-  kern<<<static_cast<unsigned>(std::min<int64_t>(ntiles, sms)), kTauThreads, smem, s>>>(mq, mk, P);
+  kern<<<static_cast<unsigned>(std::min<int64_t>(ntiles, sms)), kTauThreads, smem, s>>>(mq, mk, mw,
+                                                                                        P);
   return cudaGetLastError();
 }
 

@@ -117,11 +117,19 @@ int entmax_attn_fwd_no_block_mask(const void* q, const void* k, const void* v, v
 /* Two-pass form, for callers that own the scratch memory or time the passes apart.
  * workspace: device memory of at least entmax_attn_workspace_bytes(...) bytes, 256-byte
  * aligned, owned by the caller; the tau pass fills it and the output pass reads it, so both
- * must see the same workspace, sizes and cu_seqlens, in stream order. */
+ * must see the same workspace, sizes and cu_seqlens, in stream order.  Returns 0 on bad sizes. */
 size_t entmax_attn_workspace_bytes(int B, int Hq, int T, int has_cu_seqlens);
 
+/* The smallest workspace the passes accept: the lists, counts and overflow queue without the
+ * tau pass's warm-up keys (the squared key norms and, per key group, the 128 keys of largest
+ * norm of a few prefix ranges, whose scores start every query tile's candidate threshold).  A
+ * workspace between this size and entmax_attn_workspace_bytes() gives the same results, with
+ * the bf16 tau pass running without warm-up keys.  Returns 0 on bad sizes. */
+size_t entmax_attn_workspace_min_bytes(int B, int Hq, int T, int has_cu_seqlens);
+
 /* Tau pass: writes tau, every word of block_mask, and the compact list of active key tiles of
- * every query tile into the workspace. */
+ * every query tile into the workspace.  ENTMAX_ATTN_ENOMEM if workspace_bytes is below
+ * entmax_attn_workspace_min_bytes(). */
 int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
                          void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
                          int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
@@ -165,8 +173,9 @@ void entmax_attn_release_workspaces(void);
  * Same arguments, outputs and semantics as entmax_attn_fwd, but the scratch memory lives in a
  * file-scope device array of ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES that every GPU loading the
  * library holds until the process exits; the call allocates and frees nothing.
- *   - Problems whose scratch (entmax_attn_workspace_bytes) exceeds that size are rejected with
- *     ENTMAX_ATTN_ENOMEM before anything is launched.
+ *   - Problems whose smallest scratch (entmax_attn_workspace_min_bytes) exceeds that size are
+ *     rejected with ENTMAX_ATTN_ENOMEM before anything is launched; those whose full scratch
+ *     (entmax_attn_workspace_bytes) exceeds it run without the tau pass's warm-up keys.
  *   - The first call on a device, with that device current, looks up the array's device
  *     address (cudaGetSymbolAddress) and caches it; make that first call before any stream
  *     capture.

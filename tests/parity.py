@@ -2,7 +2,9 @@
 seeded inputs.
 
 Tolerances (the acceptance bar of the forward pass):
-  out   max-abs error <= 1e-4 for fp32 inputs, <= 2e-2 for bf16 inputs (fp32 accumulate)
+  out   max-abs error <= 1e-4 for fp32 inputs, <= 2e-2 for bf16 inputs (fp32 accumulate); a bf16
+        output is stored in bf16, which adds up to half a unit in its last place, 2^-9 |o|, to
+        the error of the accumulated value: its bar is 2e-2 + 2^-9 |o_ref| per element
   tau   |tau_gpu - tau_ref| <= 1e-4 * max(1, |tau_ref|)
   mask  bit-exact per (query tile, key tile), except tiles whose largest p is below 1e-6 both at
         the exact tau and at the GPU's tau (p evaluated in fp64 on the host by the oracle).
@@ -34,6 +36,15 @@ def out_tolerance(w: Workload) -> float:
     if w.dtype == "fp32" and beta < 1.0:
         tol += 2.0 ** (-20.0 * beta)
     return tol
+def out_bar(w: Workload, ref_out: np.ndarray) -> np.ndarray:
+    """Per-element bar on |o_gpu - o_ref|: out_tolerance, plus for bf16 the rounding of the
+    stored output (round to nearest with 8 significant bits: at most 2^-9 |o|)."""
+    bar = np.full(ref_out.shape, out_tolerance(w))
+    if w.dtype == "bf16":
+        bar += 2.0 ** -9 * np.abs(ref_out)
+    return bar
+
+
 TAU_RTOL = 1e-4
 MASK_EXEMPT_P = 1e-6
 
@@ -117,14 +128,17 @@ def compare(w: Workload, inputs, g: GpuResult, whole_tiles, loose_rows=None, lab
     rows = np.concatenate(groups + ([np.asarray(loose_rows, dtype=np.int64)]
                                     if loose_rows is not None and len(loose_rows) else []))
     ref = oracle.attention_rows(q, k, v, alpha, w.causal, cu, rows)
-    tol = out_tolerance(w)
     err_out = np.abs(g.out[rows] - ref["out"])
+    bar = out_bar(w, ref["out"])
     max_out = float(err_out.max()) if err_out.size else 0.0
+    over = float((err_out / bar).max()) if err_out.size else 0.0
     tau_g = g.tau[rows].astype(np.float64)
     err_tau = np.abs(tau_g - ref["tau"]) / np.maximum(1.0, np.abs(ref["tau"]))
     max_tau = float(err_tau.max()) if err_tau.size else 0.0
-    worst = int(np.argmax(err_out.max(axis=1))) if err_out.size else 0
-    assert max_out <= tol, (f"{label}: out max-abs {max_out:.3e} > {tol} at row {rows[worst]}")
+    worst = int(np.argmax((err_out / bar).max(axis=1))) if err_out.size else 0
+    assert over <= 1.0, (f"{label}: out error {err_out[worst].max():.3e} above its bar "
+                         f"{bar[worst][np.argmax(err_out[worst] / bar[worst])]:.3e} at row "
+                         f"{rows[worst]}")
     assert max_tau <= TAU_RTOL, (f"{label}: tau rel err {max_tau:.3e} at row "
                                  f"{rows[int(np.argmax(err_tau))]}")
 

@@ -200,11 +200,34 @@ def test_misaligned_pointers_are_rejected(native):
 
 def test_small_workspace_is_rejected(native):
     lib = native.lib()
-    need = lib.entmax_attn_workspace_bytes(1, 2, 256, 0)
-    rc = lib.entmax_attn_tau_pass(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000),
-                                  _fake(0x10000), need - 1, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
-                                  0, None)
+    need = lib.entmax_attn_workspace_min_bytes(1, 2, 256, 0)
+    for fn in ("entmax_attn_tau_pass",):
+        rc = getattr(lib, fn)(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000),
+                              _fake(0x10000), need - 1, 1, 2, 2, 256, 64, 1.5, 10, 1, None, 1,
+                              0, None)
+        assert rc == native.ENOMEM
+    rc = lib.entmax_attn_out_pass(_fake(0x1000), _fake(0x2000), _fake(0x3000), _fake(0x4000),
+                                  _fake(0x10000), need - 1, _fake(0x5000), 1, 2, 2, 256, 64, 1.5,
+                                  1, None, 1, 0, None)
     assert rc == native.ENOMEM
+
+
+@pytest.mark.parametrize("B,Hq,T,packed", [(1, 2, 256, 0), (2, 32, 16384, 0), (4, 32, 32192, 1),
+                                           (1, 32, 131072, 0), (1, 8, 1023, 0)])
+def test_workspace_sizes_nest(native, B, Hq, T, packed):
+    """The full workspace adds the warm-up sections after the smallest one: squared norms of
+    (B or 1) * Hq * T key rows and B * Hq * levels warm-up tiles of 128 x 128 bf16, levels being
+    the ranges 1024 * 2^j that fit in T keys."""
+    from adaptive_sparse_attention_b200 import api
+    lo, hi = api.workspace_min_bytes(B, Hq, T, bool(packed)), api.workspace_bytes(B, Hq, T, bool(packed))
+    levels = 0
+    while (1024 << levels) <= T:
+        levels += 1
+    rows = (1 if packed else B) * Hq * T
+    def up(x):
+        return (x + 255) // 256 * 256
+    assert 0 < lo <= hi
+    assert hi - lo == up(4 * rows) + up(B * Hq * levels * 128 * 128 * 2)
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

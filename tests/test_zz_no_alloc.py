@@ -53,7 +53,7 @@ def test_noalloc_matches_fwd_on_two_calls_in_a_row():
     w2 = WORKLOADS["t4k_bf16_d64_a1.5"]
     in2 = make_inputs(w2)
     for w, inputs in ((w1, in1), (w2, in2)):
-        need = ea.workspace_bytes(w.B, w.Hq, w.T, w.varlen)
+        need = ea.workspace_min_bytes(w.B, w.Hq, w.T, w.varlen)
         assert need <= _native.NOALLOC_SCRATCH_BYTES
         ref, got = _run_both(w, inputs)
         _check(w, ref, got)
@@ -64,7 +64,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
         pytest.fail("a CUDA device is required for -m gpu tests")
     lib = _native.lib()
     w = WORKLOADS["t128k_gqa4_bf16_d128_a1.5"]
-    assert ea.workspace_bytes(w.B, w.Hq, w.T, False) > _native.NOALLOC_SCRATCH_BYTES
+    assert ea.workspace_min_bytes(w.B, w.Hq, w.T, False) > _native.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
     rc = lib.entmax_attn_fwd_noalloc(fake, fake, fake, fake, fake, fake, w.B, w.Hq, w.Hkv, w.T,
                                      w.d, 1.5, 10, 1, None, _native.BF16, None)
