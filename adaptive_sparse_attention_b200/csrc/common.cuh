@@ -402,12 +402,14 @@ __device__ __forceinline__ void coop_insert(CS& cs, RowCand& rc, int src, int co
 
 // Feeds 32 raw scores of key tile kt (keys outside the row's range already -inf) for the 32
 // (row, segment) columns of a warp; every lane of the warp must call it together.  The hot path
-// is the max of each 16-key block.  A row whose chunk max passes its threshold is, when few rows
-// of the warp pass, handled by the whole warp: its lane writes the chunk to the warp's exchange
-// row xrow (32 floats, 16-byte aligned, private to the warp), every lane compares one value, and
-// a ballot gives each passing value its slot -- one compare per lane instead of 32 per passing
-// row.  When many rows pass (more than kExchangeMax), each lane stores its own values and only
-// rows without room take the exchange path.  The threshold uses the largest max any segment of
+// is the max of each 16-key block.  A row whose chunk max passes its threshold counts its values
+// above it; when that is one (the common case once the row max has settled) the value is the
+// chunk max and the row's lane stores it, in parallel with every other such lane.  Rows with
+// several values are, when few rows of the warp have them, handled by the whole warp: its lane
+// writes the chunk to the warp's exchange row xrow (32 floats, 16-byte aligned, private to the
+// warp), every lane compares one value, and a ballot gives each passing value its slot.  When
+// many do (more than kExchangeMax), each lane stores its own values and only rows without room
+// take the exchange path.  The threshold uses the largest max any segment of
 // the row has published in cs.rowmax[row]: a lower bound of the row's max, so every key with
 // z > (row max) - 1 is still kept, while records of one segment's max no longer trigger
 // insertions in the others.  A stale or overwritten rowmax value only loosens the threshold.
@@ -433,14 +435,28 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
       cs.rowmax[row] = cmax;  // publish to the row's other segments
     }
   }
-  unsigned serial = passing;
-  if (__popc(passing) > kExchangeMax) {
-    // Many rows pass (the first key tiles of a row, before its max settles): each lane counts
-    // and stores its own passing values, all lanes at once; rows without room go on below.
-    int incoming = 0;
+  // Most passing chunks hold a single value above the threshold, which is then the chunk max:
+  // each such lane stores it itself, all at once.  The others go on below.
+  bool single = false;
+  int incoming = 0;  // this lane's values above its threshold
+  if (pass) {
 #pragma unroll
-    for (int i = 0; i < N; ++i) incoming += (x[i] > rc.thr) ? 1 : 0;  // branch-free count
-    const bool fits = pass && rc.cnt + incoming <= CS::kSlots;
+    for (int i = 0; i < N; ++i) incoming += (x[i] > rc.thr) ? 1 : 0;  // >= 1: cmax > rc.thr
+    if (incoming == 1 && rc.cnt < CS::kSlots) {
+      cs.s[rc.cnt * kCols + col] = cmax;
+      cs.kt[rc.cnt * kCols + col] = static_cast<uint16_t>(kt);
+      ++rc.cnt;
+      single = true;
+    }
+  }
+  unsigned serial = __ballot_sync(full, pass && !single);
+  if (!serial) return;
+  __syncwarp();  // the single-value stores are visible to the warp's lanes
+  if (__popc(serial) > kExchangeMax) {
+    // Many rows with several values pass (the first key tiles of a row, before its max
+    // settles): each lane stores its own passing values, all lanes at once; rows without room
+    // go on below.
+    const bool fits = pass && !single && rc.cnt + incoming <= CS::kSlots;
     if (fits) {
       int c = rc.cnt;
       const uint16_t kt16 = static_cast<uint16_t>(kt);
@@ -453,7 +469,7 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
       }
       rc.cnt = c;
     }
-    serial = __ballot_sync(full, pass && !fits);
+    serial = __ballot_sync(full, pass && !single && !fits);
     __syncwarp();  // these stores are visible to the lanes that read the buffers below
   }
   const unsigned below = (1u << lane) - 1u;
