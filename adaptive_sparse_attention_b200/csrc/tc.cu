@@ -228,28 +228,45 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// p = [x]_+^beta for the output pass, where p is rounded to bf16 before the P V product.  For
+// beta = 3 + f near 3, x^beta = x^3 e^(f ln x) with the exponential cut after its linear term:
+// relative error <= (f ln x)^2 / 2 <= 4e-4 for x >= 1e-4 (|f| <= 0.004), a fifth of the bf16
+// rounding of p, while smaller x give p < 1e-12.  x is clamped to 1e-30 instead of 0 there,
+// which keeps the logarithm finite and still gives p = 0 (x^3 underflows).  kf = f ln 2.
+template <int BK>
+__device__ __forceinline__ float entmax_p_out(float x, float beta, float kf) {
+  if (BK == kBetaNear3) {
+    const float y = fmaxf(x, 1e-30f);
+    const float y3 = y * y * y;
+    return fmaf(y3, kf * __log2f(y), y3);
+  }
+  return entmax_p_clamped<BK>(x, beta);
+}
+
 // p of 32 consecutive keys j0 .. j0 + 31 of a row from their raw scores (TMEM words u), packed
 // as bf16 pairs; keys at or past jmax (the row's causal / sequence end) give 0.  Rows whose 32
 // keys are all valid -- every tile but the diagonal one -- skip the per-key range test.
 template <int BK>
 __device__ __forceinline__ void p_row32(const uint32_t (&u)[32], float c, float tau, float beta,
                                         int j0, int jmax, uint32_t (&pk)[16]) {
+  const float kf = (beta - 3.f) * 0.69314718f;
   if (j0 + 32 <= jmax) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float p0 = entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e]) - tau, beta);
-      const float p1 = entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e + 1]) - tau, beta);
+      const float p0 = entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, kf);
+      const float p1 = entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, kf);
       pk[e] = pack_bf16x2(p0, p1);
     }
   } else {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const float p0 = (j0 + 2 * e < jmax)
-                           ? entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e]) - tau, beta)
+                           ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, kf)
                            : 0.f;
-      const float p1 = (j0 + 2 * e + 1 < jmax)
-                           ? entmax_p_clamped<BK>(c * __uint_as_float(u[2 * e + 1]) - tau, beta)
-                           : 0.f;
+      const float p1 =
+          (j0 + 2 * e + 1 < jmax)
+              ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, kf)
+              : 0.f;
       pk[e] = pack_bf16x2(p0, p1);
     }
   }
