@@ -229,16 +229,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // p = [x]_+^beta for the output pass, where p is rounded to bf16 before the P V product.  For
-// beta = 3 + f near 3, x^beta = x^3 e^(f ln x) with the exponential cut after its linear term:
-// relative error <= (f ln x)^2 / 2 <= 4e-4 for x >= 1e-4 (|f| <= 0.004), a fifth of the bf16
-// rounding of p, while smaller x give p < 1e-12.  x is clamped to 1e-30 instead of 0 there,
-// which keeps the logarithm finite and still gives p = 0 (x^3 underflows).  kf = f ln 2.
+// beta = 3 + f near 3, x^beta = x^3 e^(f ln x) with the exponential cut after its linear term,
+// and log2 x taken from the bits of x by Mitchell's approximation (x = 2^e (1 + m) read as
+// e + m, within 0.09 of log2 x; J. N. Mitchell, "Computer multiplication and division using
+// binary logarithms", 1962), so that no special-function unit is needed.  Relative error of p:
+// (f ln x)^2 / 2 + |f| ln2 * 0.09 <= 5.5e-4 for x >= 1e-4 and |f| <= 0.004, below the bf16
+// rounding of p (2^-9), while smaller x give p < 1e-12.  x is clamped to 1e-30 instead of 0,
+// which keeps the logarithm finite and still gives p = 0 (x^3 underflows).
+// With y = bits(x) >> 9 placed in the mantissa of 2^23, e + m = y 2^-14 - 639, so
+// f ln x ~= y * ka + kb with ka = f ln2 2^-14 and kb = -639 f ln2.
 template <int BK>
-__device__ __forceinline__ float entmax_p_out(float x, float beta, float kf) {
+__device__ __forceinline__ float entmax_p_out(float x, float beta, float ka, float kb) {
   if (BK == kBetaNear3) {
     const float y = fmaxf(x, 1e-30f);
     const float y3 = y * y * y;
-    return fmaf(y3, kf * __log2f(y), y3);
+    const float e = __int_as_float((__float_as_int(y) >> 9) | 0x4B000000);
+    return fmaf(y3, fmaf(e, ka, kb), y3);
   }
   return entmax_p_clamped<BK>(x, beta);
 }
@@ -250,22 +256,23 @@ template <int BK>
 __device__ __forceinline__ void p_row32(const uint32_t (&u)[32], float c, float tau, float beta,
                                         int j0, int jmax, uint32_t (&pk)[16]) {
   const float kf = (beta - 3.f) * 0.69314718f;
+  const float ka = kf * (1.f / 16384.f), kb = -639.f * kf;
   if (j0 + 32 <= jmax) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float p0 = entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, kf);
-      const float p1 = entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, kf);
+      const float p0 = entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, ka, kb);
+      const float p1 = entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, ka, kb);
       pk[e] = pack_bf16x2(p0, p1);
     }
   } else {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const float p0 = (j0 + 2 * e < jmax)
-                           ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, kf)
+                           ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, ka, kb)
                            : 0.f;
       const float p1 =
           (j0 + 2 * e + 1 < jmax)
-              ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, kf)
+              ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, ka, kb)
               : 0.f;
       pk[e] = pack_bf16x2(p0, p1);
     }
