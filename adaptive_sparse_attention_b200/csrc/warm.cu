@@ -10,7 +10,8 @@ namespace ea {
 namespace {
 
 constexpr int kNormThreads = 256;
-constexpr int kSelectThreads = 256;
+constexpr int kSelectThreads = 1024;
+static_assert(kWarmBase % kSelectThreads == 0, "every level's range is a whole number of CTA rows");
 
 // ||k_r||^2 in fp32 for every key row r: D / 8 lanes per row, 16 bytes each.
 template <int D>
@@ -37,10 +38,19 @@ __global__ void __launch_bounds__(kNormThreads) key_norms_kernel(const __nv_bflo
   if (row < rows && lane % kLanes == 0) norms[row] = s;
 }
 
+// Adds 1 to hist[bin] for every lane with bin < 256, one shared-memory atomic per distinct bin
+// of the warp: the norms of a key range share their leading bits, so most lanes of a warp hit
+// the same bin in the first digits.  Call with the whole warp.
+__device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t bin, int lane) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+}
+
 // One CTA per (level, group): radix select (four 8-bit digits of the nonnegative fp32 norm) of
 // the 128th largest norm in the level's range, then the 128 rows -- every key above it and as
 // many keys equal to it as needed -- copied to the level's warm tile.  Levels whose range is
-// wider than any query tile of the group may use are skipped.
+// wider than any query tile of the group may use are skipped.  The range holds 1024 * 2^level
+// keys, a multiple of the CTA size, so every warp runs the same number of loop trips.
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) warm_select_kernel(Problem P) {
   const int level = blockIdx.x, grp = blockIdx.y;
@@ -63,30 +73,51 @@ __global__ void __launch_bounds__(kSelectThreads) warm_select_kernel(Problem P) 
   __shared__ uint32_t s_prefix;
   __shared__ int s_need, s_gt, s_eq;
   __shared__ int idx[kTile];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   uint32_t prefix = 0, mask = 0;
   int need = kTile;  // keys still to take at or below the current prefix
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    hist[tid] = 0u;
+    if (tid < 256) hist[tid] = 0u;
     __syncthreads();
-    for (int i = tid; i < n; i += kSelectThreads) {
-      const uint32_t u = bits[i];
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    for (int i = tid; i < n; i += 4 * kSelectThreads) {  // four loads in flight per thread
+      uint32_t u[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        u[e] = i + e * kSelectThreads < n ? bits[i + e * kSelectThreads] : 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i + e * kSelectThreads < n)  // the same for the whole warp
+          warp_hist_add(hist, (u[e] & mask) == prefix ? (u[e] >> shift) & 255u : 256u, lane);
     }
     __syncthreads();
-    if (tid == 0) {
-      int acc = 0, dsel = 0;
-      for (int b = 255; b >= 0; --b) {
-        const int h = static_cast<int>(hist[b]);
-        if (acc + h >= need) {
-          dsel = b;
-          break;
-        }
-        acc += h;
+    if (tid < 32) {  // the digit that holds the need-th largest key, by warp 0
+      // lane l owns bins 8 l .. 8 l + 7; above = keys in the bins of lanes above l
+      int h[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        h[j] = static_cast<int>(hist[8 * lane + j]);
+        sum += h[j];
       }
-      s_prefix = prefix | (static_cast<uint32_t>(dsel) << shift);
-      s_need = need - acc;
+      int incl = sum;  // keys in bins >= 8 l
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += t;
+      }
+      int acc = incl - sum;
+      if (acc < need && incl >= need) {  // exactly one lane
+        int dsel = 8 * lane;
+        for (int j = 7; j >= 0; --j) {
+          if (acc + h[j] >= need) {
+            dsel = 8 * lane + j;
+            break;
+          }
+          acc += h[j];
+        }
+        s_prefix = prefix | (static_cast<uint32_t>(dsel) << shift);
+        s_need = need - acc;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -104,8 +135,8 @@ __global__ void __launch_bounds__(kSelectThreads) warm_select_kernel(Problem P) 
     if (u > prefix) {
       idx[atomicAdd(&s_gt, 1)] = i;
     } else if (u == prefix) {
-      const int e = atomicAdd(&s_eq, 1);
-      if (e < need) idx[kTile - need + e] = i;
+      const int k = atomicAdd(&s_eq, 1);
+      if (k < need) idx[kTile - need + k] = i;
     }
   }
   __syncthreads();
