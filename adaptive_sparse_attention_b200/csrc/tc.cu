@@ -21,7 +21,8 @@
 //               from TMEM as the A operand and V (MN-major in shared memory) as B.
 //   warps 4..11 p warps, two per TMEM lane quarter, each owning 64 keys of every tile: load S,
 //               p = [c s - tau]_+^beta (0 off the causal / sequence range), store p as packed
-//               bf16 into TMEM; at the end each reads half of O's columns from TMEM and stores them.
+//               bf16 into TMEM; at the end each reads half of O's columns from TMEM and stores
+//               them.
 // tau is known before this pass, so p needs neither a running max nor a final normalisation.
 //
 // Every mbarrier wait is bounded (about 2 s of %globaltimer): on expiry the waiting thread
@@ -125,6 +126,20 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// TMA store of one 128-row x 64-column box from shared memory (128-byte swizzle, as the map
+// describes) to global coordinates (x, y); the calling thread then waits until the copy has read
+// shared memory, so the buffer may be reused or the CTA may exit.
+__device__ __forceinline__ void tma_store_2d_and_wait(const CUtensorMap* map, const void* src,
+                                                      int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(smem_u32(src))
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* holder, uint32_t ncols) {
@@ -267,9 +282,10 @@ __device__ __forceinline__ void p_row32(const uint32_t (&u)[32], float c, float 
   } else {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float p0 = (j0 + 2 * e < jmax)
-                           ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, ka, kb)
-                           : 0.f;
+      const float p0 =
+          (j0 + 2 * e < jmax)
+              ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e]), -tau), beta, ka, kb)
+              : 0.f;
       const float p1 =
           (j0 + 2 * e + 1 < jmax)
               ? entmax_p_out<BK>(fmaf(c, __uint_as_float(u[2 * e + 1]), -tau), beta, ka, kb)
@@ -1097,8 +1113,10 @@ struct UnionWalk {
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kPairThreads, 1)
-    out_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                    const __grid_constant__ CUtensorMap tmv, Problem P) {
+    out_pair_kernel(const __grid_constant__ CUtensorMap tmq,
+                    const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv,
+                    const __grid_constant__ CUtensorMap tmo, Problem P) {
   extern __shared__ unsigned char smem_raw[];
   PairSmem<D>& sm = *reinterpret_cast<PairSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1187,7 +1205,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
       for (int x = 0; x < 2; ++x)
 #pragma unroll
-        for (int k16 = 0; k16 < D / 16; ++k16) qdesc[x][k16] = kmajor_desc(smem_u32(sm.q[x]), kTile, k16);
+        for (int k16 = 0; k16 < D / 16; ++k16)
+          qdesc[x][k16] = kmajor_desc(smem_u32(sm.q[x]), kTile, k16);
       const uint64_t kdesc0 = kmajor_desc(smem_u32(sm.k[0]), kTile, 0);
       const uint64_t vdesc0 = value_desc(smem_u32(sm.v[0]), 0);
       auto issue_s = [&](int x, int ks) {  // S_X = Q_X K^T from key stage ks
@@ -1296,7 +1315,44 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     constexpr int kHalfD = D / 2;
     __nv_bfloat16* op =
         static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D + half * kHalfD;
-    if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (only after a failed tau pass)
+    // Full tiles at d = 128: the four warps of a (head, half) stage their 32 rows x 64 columns
+    // in the key ring (idle once o_full has arrived: every key tile loaded has been used) as one
+    // 128-row box in the 128-byte swizzled layout, and one TMA store writes it.  box_tile is the
+    // same for the four warps (it depends on the head only), so all four reach the barrier; the
+    // store is issued only if every one of them staged its rows (no timeout, no abort).
+    const bool box_tile = D == 128 && cnt > 0 && t.nrows == kTile;
+    if (box_tile) {
+      const bool staged = o_ok && !*abort;
+      const int box = (warp - kScoreWarp0) >> 2;  // (head, half) = (box >> 1, box & 1)
+      unsigned char* stage = reinterpret_cast<unsigned char*>(sm.k[0]) + box * (kTile * 128);
+#pragma unroll
+      for (int c0 = 0; c0 < (staged ? kHalfD : 0); c0 += 32) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + kPairColO + static_cast<uint32_t>(x * 128 + half * kHalfD + c0),
+                  u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // 16-byte chunk (c0 / 8 + e) of row r, swizzled
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(u[8 * e + 0]), __uint_as_float(u[8 * e + 1]));
+          w.y = pack_bf16x2(__uint_as_float(u[8 * e + 2]), __uint_as_float(u[8 * e + 3]));
+          w.z = pack_bf16x2(__uint_as_float(u[8 * e + 4]), __uint_as_float(u[8 * e + 5]));
+          w.w = pack_bf16x2(__uint_as_float(u[8 * e + 6]), __uint_as_float(u[8 * e + 7]));
+          const int chunk = (c0 / 8 + e) ^ (r & 7);
+          *reinterpret_cast<uint4*>(stage + r * 128 + chunk * 16) = w;
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      uint32_t all_staged;
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.b32 p, %1, 0;\n"
+          " barrier.red.and.pred q, %2, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+          : "=r"(all_staged)
+          : "r"(static_cast<int>(staged)), "r"(1 + box)
+          : "memory");
+      if (all_staged && quarter == 0 && lane == 0)
+        tma_store_2d_and_wait(&tmo, stage, half * kHalfD,
+                              static_cast<int>(t.qhead + t.seq_start + t.row0));
+    } else if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (failed tau pass only)
       uint4* dst = reinterpret_cast<uint4*>(op);
       for (int e = 0; e < kHalfD / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
     } else if (o_ok && !*abort) {
@@ -1425,16 +1481,17 @@ cudaError_t launch_out_t(const Problem& P, cudaStream_t s) {
 
 template <int D, int BK>
 cudaError_t launch_out_pair_t(const Problem& P, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
   if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
   if (e == cudaSuccess) e = make_map(&mv, P.v, kv_rows(P), D);
+  if (e == cudaSuccess) e = make_map(&mo, P.out, q_rows(P), D);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(PairSmem<D>) + 1024;
   auto kern = out_pair_kernel<D, BK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(P.slots, P.Hq / 2, P.cu ? 1 : P.B), kPairThreads, smem, s>>>(mq, mk, mv, P);
+  kern<<<dim3(P.slots, P.Hq / 2, P.cu ? 1 : P.B), kPairThreads, smem, s>>>(mq, mk, mv, mo, P);
   return cudaGetLastError();
 }
 
