@@ -25,7 +25,7 @@ constexpr int kCand = 16;       // candidate slots per (row, segment) held in sh
                                 // default; kernels with shared memory to spare take more
 constexpr int kCols = kSeg * kTile;  // (row, segment) columns of the candidate buffers
 constexpr int kXchWarps = 16;  // warps feeding candidates per CTA (one exchange row each)
-constexpr int kExchangeMax = 2;  // up to this many passing rows of a warp go through the exchange row
+constexpr int kExchangeMax = 2;  // up to this many rows of a warp take the exchange row
 constexpr int kMaxWords = 64;   // mask words per query tile the kernels support (T <= 262144)
 
 // beta = 1 and 2 have exact closed forms; kBetaNear3 is beta within kNearIntFrac of 3 (alpha
@@ -478,7 +478,8 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
     if (lane == src) {
       float4* d = reinterpret_cast<float4*>(xrow);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) d[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+      for (int i = 0; i < 8; ++i)
+        d[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
     }
     __syncwarp();
     const float v = xrow[lane];
@@ -502,9 +503,9 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
 }
 
 // Takes 32 scores of the warm-up keys (-inf for an unused row) into the row's threshold: the
-// chunk max, lowered by 1e-5 relative (and 1e-6 absolute) so that it stays below the same scores as the key tiles
-// give them whatever the rounding, raises the row max shared with the other segments and the
-// threshold.  The segment max (rc.m) is left to the key tiles themselves.
+// chunk max, lowered by 1e-5 relative (and 1e-6 absolute) so that it stays below the same
+// scores as the key tiles give them whatever the rounding, raises the row max shared with the
+// other segments and the threshold.  The segment max (rc.m) is left to the key tiles themselves.
 template <int N, class CS>
 __device__ __forceinline__ void observe_bound(RowCand& rc, CS& cs, int row,
                                               const float (&x)[N]) {

@@ -140,10 +140,18 @@ __global__ void __launch_bounds__(kThreads) tau_simt_kernel(Problem P) {
 #pragma unroll
     for (int jj = 0; jj < kChunk; ++jj) x[jj] = sm.xs[jj * kTile + tid];
     switch (chunk++ & 3) {  // uniform across the block
-      case 0: feed_warp<kChunk>(rc0, cs, cs.xrow[tid >> 5], tid, tid, tid & 31, x, kt); break;
-      case 1: feed_warp<kChunk>(rc1, cs, cs.xrow[tid >> 5], kTile + tid, tid, tid & 31, x, kt); break;
-      case 2: feed_warp<kChunk>(rc2, cs, cs.xrow[tid >> 5], 2 * kTile + tid, tid, tid & 31, x, kt); break;
-      default: feed_warp<kChunk>(rc3, cs, cs.xrow[tid >> 5], 3 * kTile + tid, tid, tid & 31, x, kt); break;
+      case 0:
+        feed_warp<kChunk>(rc0, cs, cs.xrow[tid >> 5], tid, tid, tid & 31, x, kt);
+        break;
+      case 1:
+        feed_warp<kChunk>(rc1, cs, cs.xrow[tid >> 5], kTile + tid, tid, tid & 31, x, kt);
+        break;
+      case 2:
+        feed_warp<kChunk>(rc2, cs, cs.xrow[tid >> 5], 2 * kTile + tid, tid, tid & 31, x, kt);
+        break;
+      default:
+        feed_warp<kChunk>(rc3, cs, cs.xrow[tid >> 5], 3 * kTile + tid, tid, tid & 31, x, kt);
+        break;
     }
   });
   rc0.publish(cs, tid);
