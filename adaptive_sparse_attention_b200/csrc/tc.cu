@@ -119,6 +119,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Asks for a box of the map to be brought into L2 ahead of its load.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {
   asm volatile(
@@ -464,6 +472,14 @@ __global__ void __launch_bounds__(kTauThreads, 1)
           mbar_expect_tx(&sm.q_full, kTileBytes);
           for (int h = 0; h < D / 64; ++h)
             tma_load_2d(sm.q + h * kTile * 64, &tmq, &sm.q_full, h * 64, qrow);
+        }
+        // the query tile this CTA takes next comes from HBM: start it towards L2 now, so that its
+        // load, issued only once this tile's products are done, finds it there
+        if (L + static_cast<int>(gridDim.x) < ntiles) {
+          const TileInfo tn = tau_tile(P, L + gridDim.x, per_slot);
+          if (tn.valid)
+            for (int h = 0; h < D / 64; ++h)
+              tma_prefetch_2d(&tmq, h * 64, static_cast<int>(tn.qhead + tn.seq_start + tn.row0));
         }
         ++it;
         const int lvl = warm_level(P, t), ws = lvl >= 0 ? 1 : 0, nsteps = t.nkt + ws;
