@@ -66,6 +66,8 @@ struct Problem {
   void* warm;          // [groups][warm_levels][128][d] bf16: per (batch or sequence, kv head)
                        // and level, the 128 keys of largest norm of the level's key range
   int warm_levels;     // levels per group; 0 = no warm-up keys
+  int kv_major;        // tau pass tile order: 1 = all query tiles of one key group before the
+                       // next (keys larger than L2), 0 = slot-major (see tau_tile)
 };
 
 struct TileInfo {

@@ -407,9 +407,19 @@ __device__ __forceinline__ bool score_warps_any(bool flag) {
   return r != 0;
 }
 
-// Query tile L of the tau pass's tile order: the longest tiles (highest slot) of every head
-// first, so that the tiles a persistent CTA takes in turn shrink as the pass runs out.
+// Query tile L of the tau pass's tile order.  Slot-major: the longest tiles (highest slot) of
+// every head first, so that the tiles a persistent CTA takes in turn shrink as the pass runs
+// out.  Key-group-major (P.kv_major, when the keys do not fit in L2): all query tiles of one
+// (batch or sequence, kv head) -- its G heads, longest slot first -- before the next group, so
+// that the CTAs running at a time sweep the keys of one or two groups, which stay in L2, instead
+// of every group's; the load balance is a little worse (the tile lengths saw-tooth per group).
 __device__ __forceinline__ TileInfo tau_tile(const Problem& P, int L, int per_slot) {
+  if (P.kv_major) {
+    const int per_group = P.slots * P.G;
+    const int grp = L / per_group, r = L - grp * per_group;
+    const int hk = grp % P.Hkv;
+    return map_tile(P, P.slots - 1 - r / P.G, hk * P.G + r % P.G, grp / P.Hkv);
+  }
   const int slot = P.slots - 1 - L / per_slot;
   const int hb = L % per_slot;
   return map_tile(P, slot, hb % P.Hq, hb / P.Hq);
@@ -1444,8 +1454,13 @@ cudaError_t device_sms(int* sms) {
   return e;
 }
 
+// Keys above this many bytes do not stay in L2 (126 MB) next to the streaming queries.
+constexpr int64_t kKeysInL2Bytes = 96ll << 20;
+
 template <int D, int BK>
-cudaError_t launch_tau_t(const Problem& P, cudaStream_t s) {
+cudaError_t launch_tau_t(const Problem& P0, cudaStream_t s) {
+  Problem P = P0;
+  P.kv_major = kv_rows(P) * D * 2 > kKeysInL2Bytes ? 1 : 0;
   CUtensorMap mq, mk, mw;
   cudaError_t e = make_map(&mq, P.q, q_rows(P), D);
   if (e == cudaSuccess) e = make_map(&mk, P.k, kv_rows(P), D);
