@@ -39,6 +39,9 @@ SIGNATURES = {
     "entmax_attn_out_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _vp, _c_int, _c_int,
                                       _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),
+    "entmax_attn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_size_t, _vp, _vp, _vp, _vp,
+                                 _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp,
+                                 _c_int, _c_uint, _vp]),
     "entmax_attn_fallback_tiles": (_c_int, [_vp, _vp]),
     "entmax_attn_rows": (_c_int, [_vp, ctypes.c_longlong, _vp, ctypes.c_longlong, _vp, _c_int,
                                   _c_int, _c_float, _c_int, _c_int, _vp]),

@@ -197,6 +197,27 @@ def out_pass(q, k, v, tau, workspace, out, alpha=1.5, causal=True, cu_seqlens=No
     N.check(rc, "entmax_attn_out_pass")
 
 
+def entmax_attn_bwd(q, k, v, dout, tau, workspace, alpha=1.5, causal=True, cu_seqlens=None,
+                    flags=0, stream=None):
+    """Backward pass (gradients of sum(dout * out)) for the forward whose tau and workspace are
+    given.  Returns fp32 (dq, dk, dv, delta), dq / dk / dv in the layouts of q / k / v."""
+    _check_inputs(q, k, v, cu_seqlens)
+    if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_contiguous():
+        raise ValueError("dout must be a contiguous tensor with q's shape and dtype")
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    delta = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    rc = N.lib().entmax_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(tau),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _ptr(delta), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, T, d,
+                                 float(alpha), int(bool(causal)), _ptr(cu_seqlens), _DT[q.dtype],
+                                 int(flags), _stream(stream))
+    N.check(rc, "entmax_attn_bwd")
+    return dq, dk, dv, delta
+
+
 def alloc_workspace(q, k, cu_seqlens):
     B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
     n = workspace_bytes(B, Hq, T, cu_seqlens is not None)

@@ -290,6 +290,38 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
   return ENTMAX_ATTN_OK;
 }
 
+int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                    const float* tau, const void* workspace, size_t workspace_bytes,
+                    float* delta, float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int T,
+                    int d, float alpha, int causal, const int32_t* cu_seqlens, int dtype,
+                    unsigned flags, cudaStream_t stream) {
+  Layout L;
+  ea::Problem P;
+  int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, 1, causal, cu_seqlens, dtype, &L,
+                              &P);
+  if (rc != ENTMAX_ATTN_OK) return rc;
+  if (!v || !dout || !tau || !workspace || !delta || !dq || !dk || !dv) return ENTMAX_ATTN_EINVAL;
+  if (!aligned16(v) || !aligned16(dout) || !aligned16(tau) || !aligned16(delta) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ENTMAX_ATTN_EALIGN;
+  const WsView wv = ws_view(const_cast<void*>(workspace), L);
+  if (workspace_bytes < wv.min_bytes) return ENTMAX_ATTN_ENOMEM;
+  int err = ENTMAX_ATTN_OK;
+  P.status = status_ptr(&err);
+  if (!P.status) return err;
+  P.v = v;
+  P.tau = const_cast<float*>(tau);
+  attach_workspace(&P, wv);
+  P.no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) ? 1 : 0;
+  const size_t kv_bytes = sizeof(float) * static_cast<size_t>(cu_seqlens ? 1 : B) * Hkv * T * d;
+  cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, stream);
+  if (e == cudaSuccess) e = ea::launch_bwd(P, dtype, dout, delta, dq, dk, dv, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ENTMAX_ATTN_OK;
+}
+
 namespace {
 
 // Both passes on the library's cached workspace of (device, stream); flags as the two-pass form.

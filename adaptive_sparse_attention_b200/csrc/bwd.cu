@@ -1,0 +1,254 @@
+// bwd.cu -- backward pass of causal alpha-entmax attention on the CUDA cores (fp32 arithmetic).
+//
+// Gradients of L = sum(dout * out), from the alpha-entmax Jacobian
+//   dp/ds = diag(w) - w w^T / sum(w),   w_j = p_j^(2 - alpha) = [z_j - tau]_+^(beta - 1)
+// (Peters, Niculae & Martins 2019, "Sparse Sequence-to-Sequence Models", Proposition 2; the
+// AdaSplash page says the forward pass's block mask serves the backward pass too, without a
+// formula).  Per query row i, with g_i = dout_i and u_ij = g_i . v_j:
+//   delta_i = sum_j w_ij u_ij / sum_j w_ij,   ds_ij = w_ij (u_ij - delta_i)
+//   dq_i = sum_j ds_ij k_j / sqrt(d),   dk_j += ds_ij q_i / sqrt(d),   dv_j += p_ij g_i
+// p and w come from the forward pass's tau, over the key tiles of the compact lists the tau pass
+// wrote (every key with p > 0 lies in a listed tile).
+//
+//   bwd_delta_kernel  one CTA of 128 threads per query tile, thread r owning row r: sweeps the
+//                     listed key tiles in chunks of 32 keys and sums w u and w -> delta.
+//   bwd_grad_kernel   the same sweep again: ds and p of each chunk go to shared memory; thread r
+//                     accumulates dq_r in registers; then every thread takes one key of the
+//                     chunk and a quarter of the columns and adds that key's dk and dv, summed
+//                     over the tile's rows, into fp32 global memory with atomics (several query
+//                     tiles and the query heads of a group meet on each key).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ea {
+namespace {
+
+constexpr int kBT = 128;     // threads per CTA: one per query row
+constexpr int kBChunk = 32;  // keys per chunk
+constexpr int kXS = kTile + 1;  // padded row of the [key][query row] chunk arrays
+
+template <int D>
+struct BwdSmem {
+  static constexpr int QS = D + 4;  // padded row of the query and upstream-gradient tiles
+  float qs[kTile * QS];
+  float gs[kTile * QS];
+  float ks[kBChunk * D];
+  float vs[kBChunk * D];
+  float xs[kBChunk * kXS];  // scores, then ds
+  float us[kBChunk * kXS];  // g . v, then p
+};
+
+template <typename T, int D>
+__device__ __forceinline__ void load_rows(const T* base, int64_t row0, int nrows, float* dst,
+                                          int stride, int nrow_tile, int tid) {
+  for (int i = tid; i < nrow_tile * D; i += kBT) {
+    const int r = i / D, c = i % D;
+    dst[r * stride + c] = (r < nrows) ? load_elem(base, (row0 + r) * D + c) : 0.f;
+  }
+}
+
+// Dot products of row tid of rows[128][QS] with the 32 rows of chunk[32][D] -> out[jj][tid];
+// keys at or past jmax give -inf when masked, else their dot product.
+template <int D>
+__device__ __forceinline__ void rows_dot_chunk(const float* rows, const float* chunk, float* out,
+                                               int tid, int j0, int jmax, bool masked) {
+  const float4* r4 = reinterpret_cast<const float4*>(rows + tid * BwdSmem<D>::QS);
+  const float4* c4 = reinterpret_cast<const float4*>(chunk);
+  for (int jj = 0; jj < kBChunk; ++jj) {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < D / 4; e += 2) {
+      const float4 x = r4[e], y = r4[e + 1];
+      const float4 u = c4[jj * (D / 4) + e], w = c4[jj * (D / 4) + e + 1];
+      a0 = fmaf(x.x, u.x, fmaf(x.y, u.y, fmaf(x.z, u.z, fmaf(x.w, u.w, a0))));
+      a1 = fmaf(y.x, w.x, fmaf(y.y, w.y, fmaf(y.z, w.z, fmaf(y.w, w.w, a1))));
+    }
+    out[jj * kXS + tid] = (masked && j0 + jj >= jmax) ? -INFINITY : a0 + a1;
+  }
+}
+
+// The listed key tiles of query tile t in chunks of 32 keys: fn(j0) runs after the chunk's keys
+// (rows j0 .. j0 + 31 of the sequence, zero past its end) are in ks and its values in vs.
+template <typename T, int D, typename Fn>
+__device__ __forceinline__ void sweep_listed(const Problem& P, const TileInfo& t,
+                                             BwdSmem<D>& sm, int tid, Fn&& fn) {
+  const T* kp = static_cast<const T*>(P.k);
+  const T* vp = static_cast<const T*>(P.v);
+  const int* list = P.list + t.tile_id * P.nkt_max;
+  const int cnt = list_count(P, t);
+  for (int i = 0; i < cnt; ++i) {
+    const int kt = list_tile(P, list, i, t.nkt);
+    for (int ch = 0; ch < kTile / kBChunk; ++ch) {
+      const int j0 = kt * kTile + ch * kBChunk;
+      if (j0 >= t.seq_len) break;
+      const int n = min(kBChunk, t.seq_len - j0);
+      __syncthreads();  // the previous chunk is no longer read
+      load_rows<T, D>(kp, t.khead + t.seq_start + j0, n, sm.ks, D, kBChunk, tid);
+      load_rows<T, D>(vp, t.khead + t.seq_start + j0, n, sm.vs, D, kBChunk, tid);
+      __syncthreads();
+      fn(j0);
+    }
+  }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void load_tiles(const Problem& P, const TileInfo& t, const T* g,
+                                           BwdSmem<D>& sm, int tid) {
+  const int64_t row0 = t.qhead + t.seq_start + t.row0;
+  load_rows<T, D>(static_cast<const T*>(P.q), row0, t.nrows, sm.qs, BwdSmem<D>::QS, kTile, tid);
+  load_rows<T, D>(g, row0, t.nrows, sm.gs, BwdSmem<D>::QS, kTile, tid);
+}
+
+template <typename T, int D, int BK>
+__global__ void __launch_bounds__(kBT) bwd_delta_kernel(Problem P, const T* g, float* delta) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem);
+  const int tid = threadIdx.x;
+  const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
+  if (!t.valid) return;
+  load_tiles<T, D>(P, t, g, sm, tid);
+  const bool row_ok = tid < t.nrows;
+  const int jmax = row_ok ? (P.causal ? t.row0 + tid + 1 : t.seq_len) : 0;
+  const int64_t row = t.qhead + t.seq_start + t.row0 + tid;
+  const float tau = row_ok ? P.tau[row] : INFINITY;
+  float a = 0.f, b = 0.f;
+  sweep_listed<T, D>(P, t, sm, tid, [&](int j0) {
+    rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, tid, j0, jmax, true);
+    rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, tid, j0, jmax, false);
+    for (int jj = 0; jj < kBChunk; ++jj) {
+      const float x = P.c * sm.xs[jj * kXS + tid] - tau;
+      if (x > 0.f) {
+        float p0, p1, p2;
+        entmax_powers<BK>(x, P.beta, p0, p1, p2);
+        a = fmaf(p1, sm.us[jj * kXS + tid], a);
+        b += p1;
+      }
+    }
+  });
+  if (row_ok) delta[row] = b > 0.f ? a / b : 0.f;
+}
+
+template <typename T, int D, int BK>
+__global__ void __launch_bounds__(kBT) bwd_grad_kernel(Problem P, const T* g, const float* delta,
+                                                       float* dq, float* dk, float* dv) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem);
+  constexpr int QS = BwdSmem<D>::QS;
+  const int tid = threadIdx.x;
+  const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
+  if (!t.valid) return;
+  load_tiles<T, D>(P, t, g, sm, tid);
+  const bool row_ok = tid < t.nrows;
+  const int jmax = row_ok ? (P.causal ? t.row0 + tid + 1 : t.seq_len) : 0;
+  const int64_t row = t.qhead + t.seq_start + t.row0 + tid;
+  const float tau = row_ok ? P.tau[row] : INFINITY;
+  const float dl = row_ok ? delta[row] : 0.f;
+  const float scale = rsqrtf(static_cast<float>(D));
+  float acc_q[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) acc_q[c] = 0.f;
+  // dk / dv role: key jj_k of the chunk, columns g4 + 4 m (interleaved: the four column groups
+  // of a key read four consecutive words of a query row)
+  const int jj_k = tid >> 2, g4 = tid & 3;
+  sweep_listed<T, D>(P, t, sm, tid, [&](int j0) {
+    rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, tid, j0, jmax, true);
+    rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, tid, j0, jmax, false);
+    for (int jj = 0; jj < kBChunk; ++jj) {
+      const float x = P.c * sm.xs[jj * kXS + tid] - tau;
+      float ds = 0.f, p = 0.f;
+      if (x > 0.f) {
+        float p0, p1, p2;
+        entmax_powers<BK>(x, P.beta, p0, p1, p2);
+        ds = p1 * (sm.us[jj * kXS + tid] - dl);
+        p = p0;
+      }
+      sm.xs[jj * kXS + tid] = ds;  // this thread's own column: no other thread reads it yet
+      sm.us[jj * kXS + tid] = p;
+#pragma unroll
+      for (int c = 0; c < D; ++c) acc_q[c] = fmaf(ds, sm.ks[jj * D + c], acc_q[c]);
+    }
+    __syncthreads();  // every row's ds and p of the chunk are in shared memory
+    const int j = j0 + jj_k;
+    const bool key_ok = j < t.seq_len;
+    const int64_t krow = t.khead + t.seq_start + j;
+    constexpr int kCols = D / 4;  // columns per thread
+    constexpr int kBlk = 16;
+#pragma unroll
+    for (int m0 = 0; m0 < kCols; m0 += kBlk) {
+      float ak[kBlk], av[kBlk];
+#pragma unroll
+      for (int m = 0; m < kBlk; ++m) {
+        ak[m] = 0.f;
+        av[m] = 0.f;
+      }
+      for (int r = 0; r < kTile; ++r) {
+        const float dsr = sm.xs[jj_k * kXS + r], pr = sm.us[jj_k * kXS + r];
+#pragma unroll
+        for (int m = 0; m < kBlk; ++m) {
+          const int c = g4 + 4 * (m0 + m);
+          ak[m] = fmaf(dsr, sm.qs[r * QS + c], ak[m]);
+          av[m] = fmaf(pr, sm.gs[r * QS + c], av[m]);
+        }
+      }
+      if (key_ok) {
+#pragma unroll
+        for (int m = 0; m < kBlk; ++m) {
+          const int c = g4 + 4 * (m0 + m);
+          if (ak[m] != 0.f) atomicAdd(dk + krow * D + c, ak[m] * scale);
+          if (av[m] != 0.f) atomicAdd(dv + krow * D + c, av[m]);
+        }
+      }
+    }
+  });
+  if (row_ok) {
+    float* o = dq + row * D;
+#pragma unroll
+    for (int c = 0; c < D; c += 4)
+      *reinterpret_cast<float4*>(o + c) =
+          make_float4(acc_q[c] * scale, acc_q[c + 1] * scale, acc_q[c + 2] * scale,
+                      acc_q[c + 3] * scale);
+  }
+}
+
+template <typename T, int D, int BK>
+cudaError_t launch_bwd_t(const Problem& P, const void* g, float* delta, float* dq, float* dk,
+                         float* dv, cudaStream_t s) {
+  const size_t smem = sizeof(BwdSmem<D>);
+  auto k1 = bwd_delta_kernel<T, D, BK>;
+  auto k2 = bwd_grad_kernel<T, D, BK>;
+  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(P.slots, P.Hq, P.cu ? 1 : P.B);
+  k1<<<grid, kBT, smem, s>>>(P, static_cast<const T*>(g), delta);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k2<<<grid, kBT, smem, s>>>(P, static_cast<const T*>(g), delta, dq, dk, dv);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_bwd_d(const Problem& P, const void* g, float* delta, float* dq, float* dk,
+                         float* dv, cudaStream_t s) {
+  switch (beta_kind(P.beta)) {
+    case kBetaOne: return launch_bwd_t<T, D, kBetaOne>(P, g, delta, dq, dk, dv, s);
+    case kBetaTwo: return launch_bwd_t<T, D, kBetaTwo>(P, g, delta, dq, dk, dv, s);
+    default: return launch_bwd_t<T, D, kBetaGeneral>(P, g, delta, dq, dk, dv, s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const Problem& P, int dtype, const void* g, float* delta, float* dq,
+                       float* dk, float* dv, cudaStream_t s) {
+  if (dtype == 0)
+    return P.d == 64 ? launch_bwd_d<float, 64>(P, g, delta, dq, dk, dv, s)
+                     : launch_bwd_d<float, 128>(P, g, delta, dq, dk, dv, s);
+  return P.d == 64 ? launch_bwd_d<__nv_bfloat16, 64>(P, g, delta, dq, dk, dv, s)
+                   : launch_bwd_d<__nv_bfloat16, 128>(P, g, delta, dq, dk, dv, s);
+}
+
+}  // namespace ea

@@ -22,6 +22,11 @@ cudaError_t launch_out_tc(const Problem& P, cudaStream_t s);
 // Warm-up keys of the tensor-core tau pass (P.norms, P.warm); nothing when P.warm_levels == 0.
 cudaError_t launch_warm(const Problem& P, cudaStream_t s);
 
+// Backward pass on the CUDA cores: delta (fp32 per query row), then dq (fp32, written) and dk,
+// dv (fp32, accumulated: zero them first).  g is the upstream gradient in the input dtype.
+cudaError_t launch_bwd(const Problem& P, int dtype, const void* g, float* delta, float* dq,
+                       float* dk, float* dv, cudaStream_t s);
+
 // Row-wise alpha-entmax of a [rows, n] matrix x (row stride ldx elements) into p (row stride
 // ldp); dtype 0 = fp32, 1 = bf16 for both x and p; tau may be null.
 cudaError_t launch_entmax_rows(const void* x, int64_t ldx, void* p, int64_t ldp, float* tau,

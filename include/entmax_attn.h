@@ -142,6 +142,31 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
                          const int32_t* cu_seqlens, int dtype, unsigned flags,
                          cudaStream_t stream);
 
+/* Backward pass: gradients of L = sum(dout * out) with respect to q, k and v, for the forward
+ * pass whose tau and workspace (compact lists of active key tiles) the caller passes: run the tau
+ * pass first (or entmax_attn_two_pass-style tau + output passes) on the same q, k, sizes and
+ * cu_seqlens.  The AdaSplash page ("AdaSplash with Block Masking") says the forward's block mask
+ * serves the backward pass too; only listed key tiles are visited.  The gradient follows the
+ * alpha-entmax Jacobian diag(w) - w w^T / sum(w), w = p^(2 - alpha) (Peters, Niculae & Martins
+ * 2019, Proposition 2): per query row, u_j = dout . v_j, delta = sum w u / sum w,
+ * ds_j = w_j (u_j - delta), dq = sum ds_j k_j / sqrt(d), dk_j += ds_j q / sqrt(d),
+ * dv_j += p_j dout.
+ *   dout:  the upstream gradient, the layout and dtype of q.
+ *   delta: fp32 [rows of q] written with the per-row delta (scratch the caller owns).
+ *   dq:    fp32, the layout of q, fully written.
+ *   dk, dv: fp32, the layout of k / v, fully written (zeroed, then accumulated over the query
+ *          heads of each group).
+ * Computed on the CUDA cores in fp32 from the stored inputs.  flags: ENTMAX_ATTN_FLAG_NO_BLOCK_MASK
+ * visits every causally valid key tile instead of the lists (for a tau pass run with that flag).
+ * Device pointers 16-byte aligned (workspace 256), asynchronous on `stream`.  Returns
+ * ENTMAX_ATTN_OK, ENTMAX_ATTN_EINVAL (as the forward, or a null pointer), ENTMAX_ATTN_EALIGN,
+ * ENTMAX_ATTN_ENOMEM (workspace below entmax_attn_workspace_min_bytes) or ENTMAX_ATTN_ECUDA. */
+int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                    const float* tau, const void* workspace, size_t workspace_bytes,
+                    float* delta, float* dq, float* dk, float* dv, int B, int Hq, int Hkv, int T,
+                    int d, float alpha, int causal, const int32_t* cu_seqlens, int dtype,
+                    unsigned flags, cudaStream_t stream);
+
 /* Number of query tiles that the last tau pass on this workspace sent through the multi-sweep
  * overflow path.  Synchronises `stream`.  Returns -1 on a CUDA error. */
 int entmax_attn_fallback_tiles(const void* workspace, cudaStream_t stream);

@@ -236,3 +236,22 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(_native.NativeLibraryError):
         _native.lib()
+
+
+def test_backward_argument_checks(native):
+    """entmax_attn_bwd returns its argument errors before any launch (fake pointers)."""
+    lib = native.lib()
+    p = _fake(0x10000)
+    rc = lib.entmax_attn_bwd(p, p, p, None, p, p, 1 << 30, p, p, p, p, 1, 2, 2, 256, 64, 1.5, 1,
+                             None, native.BF16, 0, None)
+    assert rc == native.EINVAL  # null dout
+    rc = lib.entmax_attn_bwd(p, p, p, p, p, p, 1 << 30, p, p, p, p, 1, 2, 2, 256, 48, 1.5, 1,
+                             None, native.BF16, 0, None)
+    assert rc == native.EINVAL  # d not in {64, 128}
+    rc = lib.entmax_attn_bwd(p, p, p, p, p, _fake(0x10010), 1 << 30, p, p, p, p, 1, 2, 2, 256, 64,
+                             1.5, 1, None, native.BF16, 0, None)
+    assert rc == native.EALIGN  # workspace not 256-byte aligned
+    need = lib.entmax_attn_workspace_min_bytes(1, 2, 256, 0)
+    rc = lib.entmax_attn_bwd(p, p, p, p, p, p, need - 1, p, p, p, p, 1, 2, 2, 256, 64, 1.5, 1,
+                             None, native.BF16, 0, None)
+    assert rc == native.ENOMEM
