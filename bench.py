@@ -478,6 +478,124 @@ def run_native(args, rank, world, local):
     return 0
 
 
+BWD_METRIC = "effective TFLOP/s of the entmax attention backward pass (dq, dk, dv)"
+
+
+def run_backward(args, rank, world, local):
+    """The backward pass (entmax_attn_bwd) of the workload, after one forward pass whose tau
+    and compact lists it reuses.  A step is one backward call over resident inputs and upstream
+    gradient.  Effective FLOPs: 10 d per valid pair inside active tiles (recomputed scores,
+    dout v^T, and the dq, dk, dv products); the kernels execute 14 d (scores and dout v^T are
+    formed in both of their sweeps), which the roofline line counts against the fp32 FMA peak of
+    the CUDA cores the pass runs on."""
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    q, k, v, cu = make_inputs(w, seed=rank)
+    gen = torch.Generator().manual_seed(1000 + rank)
+    g = torch.randn(q.shape, generator=gen).to(q.dtype)
+    qd, kd, vd, gd = q.to(dev), k.to(dev), v.to(dev), g.to(dev)
+    cud = cu.to(dev) if cu is not None else None
+    from oracle.oracle import alpha_as_float32  # the fp32 rounding of alpha, no oracle work
+    alpha = alpha_as_float32(w.alpha)
+    stream = torch.cuda.current_stream(dev)
+    out, tau, mask = ea.alloc_outputs(qd, kd, cud)
+    ws = ea.alloc_workspace(qd, kd, cud)
+    ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, stream=stream)
+    ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, stream=stream)
+    for _ in range(args.warmup):
+        grads = ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud, stream=stream)
+    torch.cuda.synchronize()
+    assert ea.status(stream) == 0
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            grads = ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud,
+                                       stream=stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(stop)
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+    assert ea.status(stream) == 0
+    bits = ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, cu)
+    act_pairs, _ = count_pairs(w, bits, cu)
+    eff_flops = 10 * w.d * act_pairs
+    value = job_rate(eff_flops, total_ms / args.steps, world) / 1e12
+    peaks, _ = load_peaks()
+    peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    achieved = 14 * w.d * act_pairs / (total_ms / args.steps * 1e-3) / 1e12
+    roofline = {"kernel": "bwd_grad_kernel + bwd_delta_kernel", "bound": "alu",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock",
+                "algorithmic": "14 d flops per valid pair inside active tiles (both sweeps)"}
+
+    # end to end: H2D of the upstream gradient from pinned memory, the backward call, D2H of
+    # dq, dk and dv, every step (forward state resident)
+    gh = g.pin_memory()
+    dq, dk, dv, _ = grads
+    hosts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    e2e_steps = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        gd.copy_(gh, non_blocking=True)
+        res = ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud, stream=stream)
+        for hst, dev_t in zip(hosts, res[:3]):
+            hst.copy_(dev_t, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import backward as obwd  # the timed CPU baseline only
+        import time
+        # a bounded sample: the oracle backward of the workload's first (batch, head) over a
+        # prefix of its rows, grown until it takes about the budget
+        nrow, spent, done_flops = 128, 0.0, 0
+        per_pair = 10 * w.d
+        while spent < args.cpu_budget / 3 and nrow <= w.T:
+            if cu is None:
+                qs, ks_, vs_, gs = (t[:1, :1, :nrow] for t in (q, k, v, g))
+            else:
+                qs, ks_, vs_, gs = (t[:1, :nrow] for t in (q, k, v, g))
+                qs, ks_, vs_, gs = qs[None], ks_[None], vs_[None], gs[None]
+            t0 = time.perf_counter()
+            obwd.attention_backward(qs, ks_, vs_, gs, alpha, w.causal, None)
+            spent = time.perf_counter() - t0
+            pairs = nrow * (nrow + 1) // 2 if w.causal else nrow * nrow
+            done_flops = per_pair * pairs
+            sample = f"oracle backward of one head over its first {nrow} rows"
+            nrow *= 2
+        cpu = {"value": done_flops / spent / 1e12, "unit": "TFLOP/s", "cores": 1,
+               "kind": "oracle", "sample": sample + f", {spent:.1f} s (numpy fp64, one thread; "
+               "all valid pairs counted)"}
+
+    line = {
+        "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(w, world), variant="backward",
+                       grads="fp32 dq, dk, dv"),
+        "active_tile_pair_fraction": None,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": job_rate(eff_flops, e2e_ms, world) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": g.numel() * g.element_size(),
+                "d2h_bytes_per_step": sum(t.numel() * 4 for t in (dq, dk, dv))},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -488,6 +606,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline figure")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (entmax_attn_bwd) instead of the forward pass")
     ap.add_argument("--no-block-mask", action="store_true",
                     help="time the variant without block mask (output pass over every causal "
                          "tile); the effective FLOPs keep counting active tiles only")
@@ -500,6 +620,8 @@ def main():
         return run_reference(args, rank, world)
     rank, world, local = dist_setup(args)
     try:
+        if args.backward:
+            return run_backward(args, rank, world, local)
         return run_native(args, rank, world, local)
     finally:
         if world > 1:
