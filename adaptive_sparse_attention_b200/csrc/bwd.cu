@@ -10,13 +10,16 @@
 // p and w come from the forward pass's tau, over the key tiles of the compact lists the tau pass
 // wrote (every key with p > 0 lies in a listed tile).
 //
-//   bwd_delta_kernel  one CTA of 128 threads per query tile, thread r owning row r: sweeps the
-//                     listed key tiles in chunks of 32 keys and sums w u and w -> delta.
-//   bwd_grad_kernel   the same sweep again: ds and p of each chunk go to shared memory; thread r
-//                     accumulates dq_r in registers; then every thread takes one key of the
-//                     chunk and a quarter of the columns and adds that key's dk and dv, summed
-//                     over the tile's rows, into fp32 global memory with atomics (several query
-//                     tiles and the query heads of a group meet on each key).
+//   bwd_delta_kernel  one CTA of 256 threads per query tile, two threads per row r, each owning
+//                     half of the head dimension (their partial dot products meet by a shuffle):
+//                     sweeps the listed key tiles in chunks of 32 keys and sums w u and w
+//                     -> delta.
+//   bwd_grad_kernel   the same sweep again: ds and p of each chunk go to shared memory; the two
+//                     threads of row r accumulate the two halves of dq_r in registers; then
+//                     eight threads take each key of the chunk, an eighth of the columns each,
+//                     and add that key's dk and dv, summed over the tile's rows, into fp32 global
+//                     memory with atomics (several query tiles and the query heads of a group
+//                     meet on each key).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -25,7 +28,7 @@
 namespace ea {
 namespace {
 
-constexpr int kBT = 128;     // threads per CTA: one per query row
+constexpr int kBT = 256;     // threads per CTA: two per query row
 constexpr int kBChunk = 32;  // keys per chunk
 constexpr int kXS = kTile + 1;  // padded row of the [key][query row] chunk arrays
 
@@ -49,23 +52,27 @@ __device__ __forceinline__ void load_rows(const T* base, int64_t row0, int nrows
   }
 }
 
-// Dot products of row tid of rows[128][QS] with the 32 rows of chunk[32][D] -> out[jj][tid];
-// keys at or past jmax give -inf when masked, else their dot product.
+// Dot products of row r of rows[128][QS] with the 32 rows of chunk[32][D] -> out[jj][r], by the
+// two threads of the row (hf = 0, 1: columns hf D/2 .. hf D/2 + D/2 - 1), whose partial sums
+// meet by a shuffle with the neighbouring lane; keys at or past jmax give -inf when masked.
 template <int D>
 __device__ __forceinline__ void rows_dot_chunk(const float* rows, const float* chunk, float* out,
-                                               int tid, int j0, int jmax, bool masked) {
-  const float4* r4 = reinterpret_cast<const float4*>(rows + tid * BwdSmem<D>::QS);
-  const float4* c4 = reinterpret_cast<const float4*>(chunk);
+                                               int r, int hf, int j0, int jmax, bool masked) {
+  constexpr int kH4 = D / 8;  // float4 per half row
+  const float4* r4 = reinterpret_cast<const float4*>(rows + r * BwdSmem<D>::QS) + hf * kH4;
+  const float4* c4 = reinterpret_cast<const float4*>(chunk) + hf * kH4;
   for (int jj = 0; jj < kBChunk; ++jj) {
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < D / 4; e += 2) {
+    for (int e = 0; e < kH4; e += 2) {
       const float4 x = r4[e], y = r4[e + 1];
       const float4 u = c4[jj * (D / 4) + e], w = c4[jj * (D / 4) + e + 1];
       a0 = fmaf(x.x, u.x, fmaf(x.y, u.y, fmaf(x.z, u.z, fmaf(x.w, u.w, a0))));
       a1 = fmaf(y.x, w.x, fmaf(y.y, w.y, fmaf(y.z, w.z, fmaf(y.w, w.w, a1))));
     }
-    out[jj * kXS + tid] = (masked && j0 + jj >= jmax) ? -INFINITY : a0 + a1;
+    float a = a0 + a1;
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    if (hf == 0) out[jj * kXS + r] = (masked && j0 + jj >= jmax) ? -INFINITY : a;
   }
 }
 
@@ -105,29 +112,32 @@ template <typename T, int D, int BK>
 __global__ void __launch_bounds__(kBT) bwd_delta_kernel(Problem P, const T* g, float* delta) {
   extern __shared__ __align__(16) unsigned char smem[];
   BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem);
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, r = tid >> 1, hf = tid & 1;
   const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
   load_tiles<T, D>(P, t, g, sm, tid);
-  const bool row_ok = tid < t.nrows;
-  const int jmax = row_ok ? (P.causal ? t.row0 + tid + 1 : t.seq_len) : 0;
-  const int64_t row = t.qhead + t.seq_start + t.row0 + tid;
+  const bool row_ok = r < t.nrows;
+  const int jmax = row_ok ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+  const int64_t row = t.qhead + t.seq_start + t.row0 + r;
   const float tau = row_ok ? P.tau[row] : INFINITY;
   float a = 0.f, b = 0.f;
   sweep_listed<T, D>(P, t, sm, tid, [&](int j0) {
-    rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, tid, j0, jmax, true);
-    rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, tid, j0, jmax, false);
-    for (int jj = 0; jj < kBChunk; ++jj) {
-      const float x = P.c * sm.xs[jj * kXS + tid] - tau;
+    rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, r, hf, j0, jmax, true);
+    rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, r, hf, j0, jmax, false);
+    __syncwarp();  // both threads of a row see the sums their lane pair wrote
+    for (int jj = hf; jj < kBChunk; jj += 2) {  // the two threads split the chunk's keys
+      const float x = P.c * sm.xs[jj * kXS + r] - tau;
       if (x > 0.f) {
         float p0, p1, p2;
         entmax_powers<BK>(x, P.beta, p0, p1, p2);
-        a = fmaf(p1, sm.us[jj * kXS + tid], a);
+        a = fmaf(p1, sm.us[jj * kXS + r], a);
         b += p1;
       }
     }
   });
-  if (row_ok) delta[row] = b > 0.f ? a / b : 0.f;
+  a += __shfl_xor_sync(0xffffffffu, a, 1);
+  b += __shfl_xor_sync(0xffffffffu, b, 1);
+  if (row_ok && hf == 0) delta[row] = b > 0.f ? a / b : 0.f;
 }
 
 template <typename T, int D, int BK>
@@ -136,76 +146,77 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(Problem P, const T* g, co
   extern __shared__ __align__(16) unsigned char smem[];
   BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem);
   constexpr int QS = BwdSmem<D>::QS;
-  const int tid = threadIdx.x;
+  constexpr int kHalf = D / 2;
+  const int tid = threadIdx.x, r = tid >> 1, hf = tid & 1;
   const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
   load_tiles<T, D>(P, t, g, sm, tid);
-  const bool row_ok = tid < t.nrows;
-  const int jmax = row_ok ? (P.causal ? t.row0 + tid + 1 : t.seq_len) : 0;
-  const int64_t row = t.qhead + t.seq_start + t.row0 + tid;
+  const bool row_ok = r < t.nrows;
+  const int jmax = row_ok ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
+  const int64_t row = t.qhead + t.seq_start + t.row0 + r;
   const float tau = row_ok ? P.tau[row] : INFINITY;
   const float dl = row_ok ? delta[row] : 0.f;
   const float scale = rsqrtf(static_cast<float>(D));
-  float acc_q[D];
+  float acc_q[kHalf];  // columns hf D/2 .. hf D/2 + D/2 - 1 of dq_r
 #pragma unroll
-  for (int c = 0; c < D; ++c) acc_q[c] = 0.f;
-  // dk / dv role: key jj_k of the chunk, columns g4 + 4 m (interleaved: the four column groups
-  // of a key read four consecutive words of a query row)
-  const int jj_k = tid >> 2, g4 = tid & 3;
+  for (int c = 0; c < kHalf; ++c) acc_q[c] = 0.f;
+  // dk / dv role: key jj_k of the chunk, columns g8 + 8 m (interleaved: the eight column groups
+  // of a key read eight consecutive words of a query row)
+  const int jj_k = tid >> 3, g8 = tid & 7;
   sweep_listed<T, D>(P, t, sm, tid, [&](int j0) {
-    rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, tid, j0, jmax, true);
-    rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, tid, j0, jmax, false);
+    rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, r, hf, j0, jmax, true);
+    rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, r, hf, j0, jmax, false);
+    __syncwarp();  // both threads of a row see the sums their lane pair wrote
     for (int jj = 0; jj < kBChunk; ++jj) {
-      const float x = P.c * sm.xs[jj * kXS + tid] - tau;
+      const float x = P.c * sm.xs[jj * kXS + r] - tau;
       float ds = 0.f, p = 0.f;
       if (x > 0.f) {
         float p0, p1, p2;
         entmax_powers<BK>(x, P.beta, p0, p1, p2);
-        ds = p1 * (sm.us[jj * kXS + tid] - dl);
+        ds = p1 * (sm.us[jj * kXS + r] - dl);
         p = p0;
       }
-      sm.xs[jj * kXS + tid] = ds;  // this thread's own column: no other thread reads it yet
-      sm.us[jj * kXS + tid] = p;
 #pragma unroll
-      for (int c = 0; c < D; ++c) acc_q[c] = fmaf(ds, sm.ks[jj * D + c], acc_q[c]);
+      for (int c = 0; c < kHalf; ++c) acc_q[c] = fmaf(ds, sm.ks[jj * D + hf * kHalf + c], acc_q[c]);
+      __syncwarp();  // both threads of the row have read the scores of key jj
+      if (hf == 0) {
+        sm.xs[jj * kXS + r] = ds;
+        sm.us[jj * kXS + r] = p;
+      }
     }
     __syncthreads();  // every row's ds and p of the chunk are in shared memory
     const int j = j0 + jj_k;
     const bool key_ok = j < t.seq_len;
     const int64_t krow = t.khead + t.seq_start + j;
-    constexpr int kCols = D / 4;  // columns per thread
-    constexpr int kBlk = 16;
+    constexpr int kCols = D / 8;  // columns per thread
+    float ak[kCols], av[kCols];
 #pragma unroll
-    for (int m0 = 0; m0 < kCols; m0 += kBlk) {
-      float ak[kBlk], av[kBlk];
+    for (int m = 0; m < kCols; ++m) {
+      ak[m] = 0.f;
+      av[m] = 0.f;
+    }
+    for (int rr = 0; rr < kTile; ++rr) {
+      const float dsr = sm.xs[jj_k * kXS + rr], pr = sm.us[jj_k * kXS + rr];
 #pragma unroll
-      for (int m = 0; m < kBlk; ++m) {
-        ak[m] = 0.f;
-        av[m] = 0.f;
+      for (int m = 0; m < kCols; ++m) {
+        const int c = g8 + 8 * m;
+        ak[m] = fmaf(dsr, sm.qs[rr * QS + c], ak[m]);
+        av[m] = fmaf(pr, sm.gs[rr * QS + c], av[m]);
       }
-      for (int r = 0; r < kTile; ++r) {
-        const float dsr = sm.xs[jj_k * kXS + r], pr = sm.us[jj_k * kXS + r];
+    }
+    if (key_ok) {
 #pragma unroll
-        for (int m = 0; m < kBlk; ++m) {
-          const int c = g4 + 4 * (m0 + m);
-          ak[m] = fmaf(dsr, sm.qs[r * QS + c], ak[m]);
-          av[m] = fmaf(pr, sm.gs[r * QS + c], av[m]);
-        }
-      }
-      if (key_ok) {
-#pragma unroll
-        for (int m = 0; m < kBlk; ++m) {
-          const int c = g4 + 4 * (m0 + m);
-          if (ak[m] != 0.f) atomicAdd(dk + krow * D + c, ak[m] * scale);
-          if (av[m] != 0.f) atomicAdd(dv + krow * D + c, av[m]);
-        }
+      for (int m = 0; m < kCols; ++m) {
+        const int c = g8 + 8 * m;
+        if (ak[m] != 0.f) atomicAdd(dk + krow * D + c, ak[m] * scale);
+        if (av[m] != 0.f) atomicAdd(dv + krow * D + c, av[m]);
       }
     }
   });
   if (row_ok) {
-    float* o = dq + row * D;
+    float* o = dq + row * D + hf * kHalf;
 #pragma unroll
-    for (int c = 0; c < D; c += 4)
+    for (int c = 0; c < kHalf; c += 4)
       *reinterpret_cast<float4*>(o + c) =
           make_float4(acc_q[c] * scale, acc_q[c + 1] * scale, acc_q[c + 2] * scale,
                       acc_q[c + 3] * scale);
