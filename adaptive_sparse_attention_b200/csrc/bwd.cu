@@ -16,10 +16,10 @@
 //                     -> delta.
 //   bwd_grad_kernel   the same sweep again: ds and p of each chunk go to shared memory; the two
 //                     threads of row r accumulate the two halves of dq_r in registers; then
-//                     eight threads take each key of the chunk, an eighth of the columns each,
-//                     and add that key's dk and dv, summed over the tile's rows, into fp32 global
-//                     memory with atomics (several query tiles and the query heads of a group
-//                     meet on each key).
+//                     each thread takes a few keys of the chunk and four of the columns and adds
+//                     their dk and dv, summed over the tile's rows, into fp32 global memory with
+//                     atomics (several query tiles and the query heads of a group meet on each
+//                     key).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -61,17 +61,21 @@ __device__ __forceinline__ void rows_dot_chunk(const float* rows, const float* c
   constexpr int kH4 = D / 8;  // float4 per half row
   const float4* r4 = reinterpret_cast<const float4*>(rows + r * BwdSmem<D>::QS) + hf * kH4;
   const float4* c4 = reinterpret_cast<const float4*>(chunk) + hf * kH4;
-  for (int jj = 0; jj < kBChunk; ++jj) {
-    float a0 = 0.f, a1 = 0.f;
+  float acc[kBChunk];  // one partial sum per key: each row float4 is loaded once
 #pragma unroll
-    for (int e = 0; e < kH4; e += 2) {
-      const float4 x = r4[e], y = r4[e + 1];
-      const float4 u = c4[jj * (D / 4) + e], w = c4[jj * (D / 4) + e + 1];
-      a0 = fmaf(x.x, u.x, fmaf(x.y, u.y, fmaf(x.z, u.z, fmaf(x.w, u.w, a0))));
-      a1 = fmaf(y.x, w.x, fmaf(y.y, w.y, fmaf(y.z, w.z, fmaf(y.w, w.w, a1))));
+  for (int jj = 0; jj < kBChunk; ++jj) acc[jj] = 0.f;
+#pragma unroll 2
+  for (int e = 0; e < kH4; ++e) {
+    const float4 x = r4[e];
+#pragma unroll
+    for (int jj = 0; jj < kBChunk; ++jj) {
+      const float4 u = c4[jj * (D / 4) + e];
+      acc[jj] = fmaf(x.x, u.x, fmaf(x.y, u.y, fmaf(x.z, u.z, fmaf(x.w, u.w, acc[jj]))));
     }
-    float a = a0 + a1;
-    a += __shfl_xor_sync(0xffffffffu, a, 1);
+  }
+#pragma unroll
+  for (int jj = 0; jj < kBChunk; ++jj) {
+    const float a = acc[jj] + __shfl_xor_sync(0xffffffffu, acc[jj], 1);
     if (hf == 0) out[jj * kXS + r] = (masked && j0 + jj >= jmax) ? -INFINITY : a;
   }
 }
@@ -160,9 +164,6 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(Problem P, const T* g, co
   float acc_q[kHalf];  // columns hf D/2 .. hf D/2 + D/2 - 1 of dq_r
 #pragma unroll
   for (int c = 0; c < kHalf; ++c) acc_q[c] = 0.f;
-  // dk / dv role: key jj_k of the chunk, columns g8 + 8 m (interleaved: the eight column groups
-  // of a key read eight consecutive words of a query row)
-  const int jj_k = tid >> 3, g8 = tid & 7;
   sweep_listed<T, D>(P, t, sm, tid, [&](int j0) {
     rows_dot_chunk<D>(sm.qs, sm.ks, sm.xs, r, hf, j0, jmax, true);
     rows_dot_chunk<D>(sm.gs, sm.vs, sm.us, r, hf, j0, jmax, false);
@@ -185,31 +186,48 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(Problem P, const T* g, co
       }
     }
     __syncthreads();  // every row's ds and p of the chunk are in shared memory
-    const int j = j0 + jj_k;
-    const bool key_ok = j < t.seq_len;
-    const int64_t krow = t.khead + t.seq_start + j;
-    constexpr int kCols = D / 8;  // columns per thread
-    float ak[kCols], av[kCols];
+    // dk / dv of the chunk's keys: thread (key group kg, column group cg) sums, over the tile's
+    // rows, kKeys keys x 4 columns (columns cg + kCg m, so that a warp's column groups read
+    // consecutive words of a query row): 2 kKeys + 8 shared loads per 8 kKeys FMAs
+    constexpr int kCg = D / 4;           // column groups
+    constexpr int kKeys = kBChunk * kCg / kBT;  // keys per thread
+    const int kg = tid / kCg, cg = tid % kCg;
+    float ak[kKeys][4], av[kKeys][4];
 #pragma unroll
-    for (int m = 0; m < kCols; ++m) {
-      ak[m] = 0.f;
-      av[m] = 0.f;
-    }
+    for (int i = 0; i < kKeys; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        ak[i][m] = 0.f;
+        av[i][m] = 0.f;
+      }
     for (int rr = 0; rr < kTile; ++rr) {
-      const float dsr = sm.xs[jj_k * kXS + rr], pr = sm.us[jj_k * kXS + rr];
+      float qv[4], gv[4];
 #pragma unroll
-      for (int m = 0; m < kCols; ++m) {
-        const int c = g8 + 8 * m;
-        ak[m] = fmaf(dsr, sm.qs[rr * QS + c], ak[m]);
-        av[m] = fmaf(pr, sm.gs[rr * QS + c], av[m]);
+      for (int m = 0; m < 4; ++m) {
+        qv[m] = sm.qs[rr * QS + cg + kCg * m];
+        gv[m] = sm.gs[rr * QS + cg + kCg * m];
+      }
+#pragma unroll
+      for (int i = 0; i < kKeys; ++i) {
+        const float dsr = sm.xs[(kg * kKeys + i) * kXS + rr];
+        const float pr = sm.us[(kg * kKeys + i) * kXS + rr];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          ak[i][m] = fmaf(dsr, qv[m], ak[i][m]);
+          av[i][m] = fmaf(pr, gv[m], av[i][m]);
+        }
       }
     }
-    if (key_ok) {
 #pragma unroll
-      for (int m = 0; m < kCols; ++m) {
-        const int c = g8 + 8 * m;
-        if (ak[m] != 0.f) atomicAdd(dk + krow * D + c, ak[m] * scale);
-        if (av[m] != 0.f) atomicAdd(dv + krow * D + c, av[m]);
+    for (int i = 0; i < kKeys; ++i) {
+      const int j = j0 + kg * kKeys + i;
+      if (j >= t.seq_len) continue;
+      const int64_t krow = t.khead + t.seq_start + j;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int c = cg + kCg * m;
+        if (ak[i][m] != 0.f) atomicAdd(dk + krow * D + c, ak[i][m] * scale);
+        if (av[i][m] != 0.f) atomicAdd(dv + krow * D + c, av[i][m]);
       }
     }
   });
