@@ -1,7 +1,7 @@
 """fp64 CPU oracle of the backward pass of causal alpha-entmax attention -- TEST INFRASTRUCTURE.
 
-Only ``tests/`` and ``bench.py``'s CPU-baseline leg use this module; the CUDA library never does,
-and this module imports nothing from it.
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg use this module;
+the CUDA library never does, and this module imports nothing from it.
 
 The pages say the block mask of the forward pass also serves the backward pass ("AdaSplash with
 Block Masking", AdaSplash: Adaptive Sparse Flash Attention) but print no gradient formula.  It is
