@@ -48,7 +48,8 @@ def _packed(name, seqlens, **kw):
     return Workload(name=name, B=len(seqlens), T=int(sum(seqlens)), seqlens=tuple(seqlens), **kw)
 
 
-# The five workloads the forward pass is judged on (sizes, dtypes, alpha and spike recipes).
+# The five workloads the forward pass is measured and checked on (sizes, dtypes, alpha and spike
+# recipes).
 WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     Workload("t256_fp32_d64_a1.5", B=1, Hq=2, Hkv=2, T=256, d=64, dtype="fp32", alpha=1.5,
              note="small fp32 case, no spikes"),

@@ -214,7 +214,7 @@ double oracle_tau_halley(const double* z, int n, double alpha, int n_iter) {
  *   maxp[i * maxp_stride + kt]  max of p_ij over the valid keys j of key tile kt, counted from
  *                               the start of the row's sequence; 0 where the row has no valid
  *                               key; when maxp != NULL.  maxp_stride >= number of key tiles.
- * With tau_given, p is evaluated at that tau instead of the exact one (used to judge mask
+ * With tau_given, p is evaluated at that tau instead of the exact one (used to decide mask
  * bits that sit within rounding of the threshold).
  * Returns 0, or 1 on a malformed argument.                                                    */
 int oracle_entmax_attn_rows(const float* q, const float* k, const float* v, int B, int Hq, int Hkv,
