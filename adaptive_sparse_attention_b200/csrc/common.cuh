@@ -205,11 +205,15 @@ __device__ __forceinline__ float entmax_p_clamped(float x, float beta) {
 struct Search {
   float tau, lo, hi, dx, dxold, m;
 
-  // p_max <= 1 gives tau >= m - 1; n keys all at most m give tau <= m - n^(1 - alpha).
+  // p_max <= 1 gives tau >= m - 1; n keys all at most m give tau <= m - n^(1 - alpha), with
+  // equality when all n tie at m.  The upper end is raised by a rounding margin: a step that
+  // lands on a root at that end (exactly so for alpha = 2, where f is linear in tau) carries the
+  // rounding of tau - f / f', a few ulps of |m| + 1, and without the margin it would fall just
+  // outside the bracket at every step and leave tau to bisection.
   __device__ __forceinline__ void init(float m_, int n, float alpha) {
     m = m_;
     lo = m - 1.f;
-    hi = m - exp2f((1.f - alpha) * __log2f((float)n));
+    hi = m - exp2f((1.f - alpha) * __log2f((float)n)) + 8.f * FLT_EPSILON * (fabsf(m) + 1.f);
     tau = lo;
     dx = dxold = hi - lo;
   }

@@ -258,6 +258,26 @@ def test_constant_values_give_constant_output_and_single_key_row(oracle):
     assert r["maxp"][0, 0] == 1.0
 
 
+@pytest.mark.parametrize("alpha", [1.333, 1.5, 2.0, 3.0])
+def test_equal_scores_give_uniform_rows_and_the_value_prefix_mean(oracle, alpha):
+    """q = 0: every score of a row is 0, so p is uniform over the row's n valid keys.  From
+    sum_j (-tau)^(1/(alpha-1)) = 1: tau = -n^(1-alpha), and o_i is the mean of the first n value
+    rows (causal) or of all of them (non-causal)."""
+    rng = np.random.default_rng(6)
+    T, d = 37, 8
+    q = np.zeros((1, 2, T, d), dtype=np.float32)
+    k = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    v = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    a = float(np.float32(alpha))
+    for causal in (True, False):
+        r = oracle.attention_rows(q, k, v, alpha=a, causal=causal)
+        n = np.arange(1, T + 1, dtype=np.float64) if causal else np.full(T, float(T))
+        vf = v[0, 0].astype(np.float64)
+        mean = np.cumsum(vf, axis=0) / n[:, None] if causal else np.tile(vf.mean(axis=0), (T, 1))
+        assert np.max(np.abs(r["out"] - np.concatenate([mean, mean]))) <= 1e-12
+        assert np.max(np.abs(r["tau"] - np.concatenate([-(n ** (1.0 - a))] * 2))) <= 1e-12
+
+
 def test_gqa_equals_repeated_kv_heads(oracle):
     """The kv head of q head h is floor(h / G): GQA equals MHA with each kv head repeated G
     times in a row."""

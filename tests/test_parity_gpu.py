@@ -6,7 +6,8 @@ tiles sampled two-sided plus loose rows one-sided, through the same entry points
 times), ragged and tiny sequence lengths, non-causal attention, GQA, packed batches with empty
 and one-token sequences, d = 64 and 128, alpha in {1.333, 1.5, 2, 3}, the CUDA-core path for
 bf16, the multi-sweep overflow path forced on every tile, and inputs that overflow the
-candidate buffers naturally.
+candidate buffers naturally, and the degenerate rows: all scores equal (uniform p, tau at the
+upper end of the search bracket) and scores far apart (one-hot p).
 """
 import numpy as np
 import pytest
@@ -153,3 +154,43 @@ def test_candidate_overflow_is_exact(oracle, alpha):
     g = parity.run_gpu(w, inputs)
     assert g.fallback_tiles > 0
     parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"overflow/{alpha}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_equal_scores_give_uniform_rows(oracle, alpha, dtype):
+    """q = 0 makes every score of a row equal, so p is uniform over the row's valid keys
+    (p_j = 1/n for all j, tau = -n^(1-alpha)) and o is the mean of the value prefix.  Every key
+    is then a candidate: rows longer than the buffers take the overflow path.  Checked against
+    the oracle and against that closed form."""
+    w, (q, k, v, cu) = random_case(B=1, Hq=4, Hkv=2, T=300, d=128, dtype=dtype, alpha=alpha,
+                                   name="equal_scores", seed=13)
+    q = torch.zeros_like(q)
+    inputs = (q, k, v, cu)
+    g = parity.run_gpu(w, inputs)
+    assert g.fallback_tiles > 0
+    parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"equal_scores/{dtype}/{alpha}")
+    vf = v.double().numpy()
+    n = np.arange(1, w.T + 1, dtype=np.float64)
+    G = w.Hq // w.Hkv
+    want = np.stack([np.cumsum(vf[0, h // G], axis=0) / n[:, None] for h in range(w.Hq)])
+    want = want.reshape(-1, w.d)
+    bar = parity.out_bar(w, want)
+    assert np.all(np.abs(g.out - want) <= bar), "output is not the mean of the value prefix"
+    want_tau = -(n ** (1.0 - float(np.float32(alpha))))
+    np.testing.assert_allclose(g.tau.reshape(w.Hq, w.T), np.broadcast_to(want_tau, (w.Hq, w.T)),
+                               rtol=parity.TAU_RTOL, atol=parity.TAU_RTOL)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_far_apart_scores_give_one_hot_rows(oracle, dtype):
+    """q scaled by 16 against spiked keys spreads the scores of a row over hundreds of units, so
+    most rows put all their mass on one key (p one-hot, o = that key's value row).  The mask then
+    holds few tiles per row; the result must match the oracle, including rows whose support
+    still has two or more keys."""
+    w, (q, k, v, cu) = random_case(B=2, Hq=4, Hkv=1, T=400, d=64, dtype=dtype, alpha=1.5,
+                                   spike_frac=0.02, spike_scale=4.0, name="one_hot", seed=17)
+    q = (q.float() * 16).to(q.dtype)
+    inputs = (q, k, v, cu)
+    g = parity.run_gpu(w, inputs)
+    parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"one_hot/{dtype}")
