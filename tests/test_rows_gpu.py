@@ -62,3 +62,21 @@ def test_rows_strided_and_batched(oracle):
     torch.cuda.synchronize()
     assert p3.shape == x3.shape and t3.shape == (2, 3)
     _check(x3.reshape(-1, 77), p3.reshape(-1, 77), t3.reshape(-1), 2.0, "bf16")
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+def test_tied_rows_every_length(oracle, alpha):
+    """Rows whose entries all tie have tau = m - n^(1 - alpha) exactly, the upper end of the
+    search bracket, and p = 1/n.  Whether an fp32 search step lands inside or just outside that
+    end depends on the rounding at each n, so every n from 2 to 1200 is checked against the
+    closed forms, at three offsets m."""
+    a32 = orc.alpha_as_float32(alpha)
+    for n in range(2, 1201):
+        x = torch.tensor([0.0, 3.25, -7.5], dtype=torch.float32)[:, None].repeat(1, n).cuda()
+        p, tau = ea.entmax_rows(x, a32, 10)
+        torch.cuda.synchronize()
+        z = (a32 - 1.0) * np.array([0.0, 3.25, -7.5])
+        want = z - float(n) ** (1.0 - a32)
+        got = tau.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - want) <= 1e-4 * np.maximum(1.0, np.abs(want))), (n, got, want)
+        assert float((p.cpu().double() - 1.0 / n).abs().max()) <= 1e-4, n
