@@ -15,8 +15,9 @@
  * sequence otherwise.  tau_i is found by n_iter steps of a bracketed Halley + bisection search
  * ("Triton Entmax (Optimized Entmax Activation)" section of the same page).  The block mask
  * holds one bit per (128-row query tile, 128-key key tile): set iff some valid pair of the tile
- * has p > 0 ("Requires O(Tr x Tc) bits ... binary mask per block").  The output pass visits
- * only the key tiles whose bit is set.
+ * has p > 0 (the per-block binary mask of the "AdaSplash with Block Masking" section, whose
+ * memory grows with the product of the query-tile and key-tile counts).  The output pass
+ * visits only the key tiles whose bit is set.
  *
  * Conventions for every entry point below:
  *   - Pointers named q, k, v, out, tau, block_mask, cu_seqlens, workspace are DEVICE pointers
