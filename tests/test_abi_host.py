@@ -255,3 +255,33 @@ def test_backward_argument_checks(native):
     rc = lib.entmax_attn_bwd(p, p, p, p, p, p, need - 1, p, p, p, p, 1, 2, 2, 256, 64, 1.5, 1,
                              None, native.BF16, 0, None)
     assert rc == native.ENOMEM
+
+
+def test_product_never_reaches_the_oracle():
+    """The package (Python binding and CUDA sources) imports, includes and loads nothing from
+    oracle/, and the oracle nothing from the package but the seeded input generators."""
+    import ast
+    import pathlib
+    root = pathlib.Path(__file__).resolve().parent.parent
+    pkg = root / "adaptive_sparse_attention_b200"
+    for f in pkg.rglob("*.py"):
+        for node in ast.walk(ast.parse(f.read_text())):
+            if isinstance(node, ast.Import):
+                names = [a.name for a in node.names]
+            elif isinstance(node, ast.ImportFrom):
+                names = [node.module or ""]
+            else:
+                continue
+            assert not any(n == "oracle" or n.startswith("oracle.") for n in names), f
+    for f in list(pkg.rglob("*.cu")) + list(pkg.rglob("*.cuh")) + list(pkg.rglob("*.h")):
+        text = f.read_text()
+        assert "oracle" not in text.lower(), f
+    for f in (root / "oracle").rglob("*.py"):
+        for node in ast.walk(ast.parse(f.read_text())):
+            if isinstance(node, ast.ImportFrom) and (node.module or "").startswith(
+                    "adaptive_sparse_attention_b200"):
+                assert node.module == "adaptive_sparse_attention_b200.workloads", f
+            if isinstance(node, ast.Import):
+                for a in node.names:
+                    assert not a.name.startswith("adaptive_sparse_attention_b200") or \
+                        a.name == "adaptive_sparse_attention_b200.workloads", f
