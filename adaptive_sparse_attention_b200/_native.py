@@ -45,6 +45,9 @@ SIGNATURES = {
     "entmax_attn_fallback_tiles": (_c_int, [_vp, _vp]),
     "entmax_attn_rows": (_c_int, [_vp, ctypes.c_longlong, _vp, ctypes.c_longlong, _vp, _c_int,
                                   _c_int, _c_float, _c_int, _c_int, _vp]),
+    "entmax_attn_route_chunks": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
+                                          _c_int, _c_int, _c_float, _c_int, _c_int, _c_int,
+                                          _c_float, _c_int, _vp]),
     "entmax_attn_status": (_c_int, [_vp]),
     "entmax_attn_release_workspaces": (None, []),
     "entmax_attn_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,

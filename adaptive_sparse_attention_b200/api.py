@@ -154,6 +154,31 @@ def entmax_rows(x, alpha: float = 1.5, n_iter: int = 10, out=None, tau=None, str
     return p.reshape(x.shape), t.reshape(x.shape[:-1])
 
 
+def route_chunks(q, summaries, alpha: float = 1.5, chunk_size: int = 64, n_iter: int = 10,
+                 causal: bool = True, estimate_diagonal: bool = True, scaling_factor: float = 1.0,
+                 stream=None):
+    """Entmax block routing of every query row over the chunk summaries it may see.
+    q [B, Hq, T, d] and summaries [B, Hkv, ceil(T / chunk_size), d], same dtype, contiguous.
+    Returns (pi fp32 [B, Hq, T, n_chunks], tau fp32 [B, Hq, T])."""
+    if q.dtype not in _DT or summaries.dtype != q.dtype:
+        raise TypeError("q and summaries must both be float32 or both bfloat16")
+    if q.dim() != 4 or summaries.dim() != 4 or not q.is_contiguous() or \
+            not summaries.is_contiguous():
+        raise ValueError("q [B, Hq, T, d] and summaries [B, Hkv, n_chunks, d], contiguous")
+    B, Hq, T, d = q.shape
+    Hkv, nc = summaries.shape[1], summaries.shape[2]
+    if summaries.shape[0] != B or summaries.shape[3] != d or nc != -(-T // chunk_size):
+        raise ValueError("summaries must be [B, Hkv, ceil(T / chunk_size), d]")
+    pi = torch.empty((B, Hq, T, nc), dtype=torch.float32, device=q.device)
+    tau = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    rc = N.lib().entmax_attn_route_chunks(_ptr(q), _ptr(summaries), _ptr(pi), _ptr(tau), B, Hq,
+                                          Hkv, T, d, int(chunk_size), float(alpha), int(n_iter),
+                                          int(bool(causal)), int(bool(estimate_diagonal)),
+                                          float(scaling_factor), _DT[q.dtype], _stream(stream))
+    N.check(rc, "entmax_attn_route_chunks")
+    return pi, tau
+
+
 def entmax_attn_fwd_noalloc(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool = True,
                             cu_seqlens=None, out=None, tau=None, block_mask=None, stream=None):
     """Forward pass through the allocation-free entry point: the library's scratch is a fixed

@@ -26,6 +26,14 @@ int cuda_fail(cudaError_t e) {
   return ENTMAX_ATTN_ECUDA;
 }
 
+}  // namespace
+
+namespace ea {
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace ea
+
+namespace {
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
@@ -180,6 +188,10 @@ struct CachedWs {
   void* ptr = nullptr;
   size_t bytes = 0;
 };
+// The cached workspaces, one per (device, stream), and the lock that guards them.  A call holds
+// it from the lookup until both passes are enqueued, so another host thread's call on the same
+// (device, stream) cannot free (and regrow) the buffer in between.
+std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, CachedWs> g_ws;
 
 }  // namespace
@@ -339,30 +351,27 @@ int fwd_cached(const void* q, const void* k, const void* v, void* out, float* ta
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  void* ws = nullptr;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    CachedWs& c = g_ws[{dev, stream}];
-    if (c.bytes < need) {
-      if (c.ptr) {
-        e = cudaFreeAsync(c.ptr, stream);
-        c.ptr = nullptr;
-        c.bytes = 0;
-        if (e != cudaSuccess) return cuda_fail(e);
-      }
-      e = cudaMallocAsync(&c.ptr, need, stream);
-      if (e != cudaSuccess) {
-        c.ptr = nullptr;
-        return ENTMAX_ATTN_ENOMEM;
-      }
-      c.bytes = need;
+  std::lock_guard<std::mutex> lk(g_ws_mu);  // held until both passes are enqueued
+  CachedWs& c = g_ws[{dev, stream}];
+  if (c.bytes < need) {
+    if (c.ptr) {
+      e = cudaFreeAsync(c.ptr, stream);
+      c.ptr = nullptr;
+      c.bytes = 0;
+      if (e != cudaSuccess) return cuda_fail(e);
     }
-    ws = c.ptr;
+    e = cudaMallocAsync(&c.ptr, need, stream);
+    if (e != cudaSuccess) {
+      c.ptr = nullptr;
+      cuda_fail(e);
+      return ENTMAX_ATTN_ENOMEM;
+    }
+    c.bytes = need;
   }
-  rc = entmax_attn_tau_pass(q, k, tau, block_mask, ws, need, B, Hq, Hkv, T, d, alpha, n_iter,
+  rc = entmax_attn_tau_pass(q, k, tau, block_mask, c.ptr, need, B, Hq, Hkv, T, d, alpha, n_iter,
                             causal, cu_seqlens, dtype, flags, stream);
   if (rc != ENTMAX_ATTN_OK) return rc;
-  return entmax_attn_out_pass(q, k, v, tau, ws, need, out, B, Hq, Hkv, T, d, alpha, causal,
+  return entmax_attn_out_pass(q, k, v, tau, c.ptr, need, out, B, Hq, Hkv, T, d, alpha, causal,
                               cu_seqlens, dtype, flags, stream);
 }
 
@@ -381,6 +390,28 @@ int entmax_attn_rows(const void* x, long long ldx, void* p, long long ldp, float
   cudaError_t e = ea::launch_entmax_rows(x, static_cast<int64_t>(ldx), p,
                                          static_cast<int64_t>(ldp), tau, rows, n, alpha, n_iter,
                                          dtype, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ENTMAX_ATTN_OK;
+}
+
+int entmax_attn_route_chunks(const void* q, const void* summaries, float* pi, float* tau, int B,
+                             int Hq, int Hkv, int T, int d, int chunk_size, float alpha,
+                             int n_iter, int causal, int estimate_diagonal, float scaling_factor,
+                             int dtype, cudaStream_t stream) {
+  if (!q || !summaries || !pi || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0 ||
+      d < 1 || d > 1024 || chunk_size < 1 || !std::isfinite(alpha) || !(alpha > 1.f) ||
+      n_iter < 1 || n_iter > 1000 || (causal != 0 && causal != 1) ||
+      (estimate_diagonal != 0 && estimate_diagonal != 1) || !std::isfinite(scaling_factor) ||
+      (dtype != ENTMAX_ATTN_FP32 && dtype != ENTMAX_ATTN_BF16))
+    return ENTMAX_ATTN_EINVAL;
+  const int nc = (T - 1) / chunk_size + 1;
+  const uintptr_t esz = dtype == ENTMAX_ATTN_FP32 ? 4u : 2u;
+  if ((reinterpret_cast<uintptr_t>(q) % esz) || (reinterpret_cast<uintptr_t>(summaries) % esz) ||
+      (reinterpret_cast<uintptr_t>(pi) & 3u) || (reinterpret_cast<uintptr_t>(tau) & 3u))
+    return ENTMAX_ATTN_EALIGN;
+  cudaError_t e = ea::launch_route_chunks(q, summaries, pi, tau, B, Hq, Hkv, T, d, nc, chunk_size,
+                                          alpha, n_iter, causal, estimate_diagonal,
+                                          scaling_factor, dtype, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return ENTMAX_ATTN_OK;
 }
@@ -427,7 +458,7 @@ int entmax_attn_status(cudaStream_t stream) {
 }
 
 void entmax_attn_release_workspaces(void) {
-  std::lock_guard<std::mutex> lk(g_mu);
+  std::lock_guard<std::mutex> lk(g_ws_mu);
   int cur = 0;
   cudaGetDevice(&cur);
   for (auto& kv : g_ws) {

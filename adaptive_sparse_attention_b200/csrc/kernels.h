@@ -27,11 +27,20 @@ cudaError_t launch_warm(const Problem& P, cudaStream_t s);
 cudaError_t launch_bwd(const Problem& P, int dtype, const void* g, float* delta, float* dq,
                        float* dk, float* dv, cudaStream_t s);
 
+// Entmax block routing over chunk summaries (pi fp32 [B, Hq, T, nc], tau fp32 [B, Hq, T]).
+cudaError_t launch_route_chunks(const void* q, const void* sig, float* pi, float* tau, int B,
+                                int Hq, int Hkv, int T, int d, int nc, int chunk, float alpha,
+                                int n_iter, int causal, int diag, float scaling, int dtype,
+                                cudaStream_t s);
+
 // Row-wise alpha-entmax of a [rows, n] matrix x (row stride ldx elements) into p (row stride
 // ldp); dtype 0 = fp32, 1 = bf16 for both x and p; tau may be null.
 cudaError_t launch_entmax_rows(const void* x, int64_t ldx, void* p, int64_t ldp, float* tau,
                                int rows, int n, float alpha, int n_iter, int dtype,
                                cudaStream_t s);
+
+// Records e as the string entmax_attn_last_cuda_error reports and returns ENTMAX_ATTN_ECUDA.
+int record_cuda_error(cudaError_t e);
 
 inline int beta_kind(float beta) {
   if (beta == 1.f) return kBetaOne;

@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "entmax_attn.h"
+#include "kernels.h"
 
 namespace {
 
@@ -43,15 +44,17 @@ extern "C" int entmax_attn_fwd_noalloc(const void* q, const void* k, const void*
   if (need > ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES) return ENTMAX_ATTN_ENOMEM;  // too large for it
 
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return ENTMAX_ATTN_ECUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return ea::record_cuda_error(e);
+  if (dev < 0 || dev >= kMaxDevices) return ea::record_cuda_error(cudaErrorInvalidDevice);
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_scratch_ptr[dev]) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-        return ENTMAX_ATTN_ECUDA;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return ea::record_cuda_error(e);
+      if (p == nullptr) return ea::record_cuda_error(cudaErrorInvalidSymbol);
       g_scratch_ptr[dev] = p;
     }
     scratch = g_scratch_ptr[dev];

@@ -184,6 +184,28 @@ int entmax_attn_fallback_tiles(const void* workspace, cudaStream_t stream);
 int entmax_attn_rows(const void* x, long long ldx, void* p, long long ldp, float* tau, int rows,
                      int n, float alpha, int n_iter, int dtype, cudaStream_t stream);
 
+/* Entmax block routing over chunk summaries (MiniCPM-4-8B-NSA page, DashAttention, "How it
+ * works", stage 2).  Keys are cut into chunks of chunk_size tokens, nc = ceil(T / chunk_size);
+ * `summaries` holds one vector per (batch, kv head, chunk), [B, Hkv, nc, d], built by the caller.
+ * Every query row i of q [B, Hq, T, d] scores the chunks it may see,
+ *   s_c = scaling_factor * q_i . summaries[b, kv(h), c] / sqrt(d),   kv(h) = floor(h / (Hq / Hkv)),
+ * and routes by alpha-entmax over them: pi_c = [(alpha - 1) s_c - tau_i]_+^(1/(alpha - 1)) with
+ * sum_c pi_c = 1, tau_i by n_iter steps (fewer once settled) of the search of the attention passes.
+ * Visible chunks: causal -- those before the row's own chunk floor(i / chunk_size), and the own
+ * chunk too when estimate_diagonal is 1; not causal -- all.  Output: pi fp32 [B, Hq, T, nc], zero
+ * outside the visible chunks (the routing priors; their nonzeros are the sparse chunk support);
+ * tau fp32 [B, Hq, T] (may be NULL), +inf for a row that sees no chunk (its pi is all zero).
+ * q and summaries share the dtype (ENTMAX_ATTN_FP32 or ENTMAX_ATTN_BF16), d <= 1024.  Device
+ * pointers, aligned to their element size (pi, tau to 4 bytes); asynchronous on `stream`.
+ * Returns ENTMAX_ATTN_OK, ENTMAX_ATTN_EINVAL (a size < 1, Hq not a multiple of Hkv, d > 1024,
+ * alpha <= 1 or not finite, n_iter outside [1, 1000], causal or estimate_diagonal not 0/1,
+ * scaling_factor not finite, bad dtype, null q, summaries or pi), ENTMAX_ATTN_EALIGN or
+ * ENTMAX_ATTN_ECUDA. */
+int entmax_attn_route_chunks(const void* q, const void* summaries, float* pi, float* tau, int B,
+                             int Hq, int Hkv, int T, int d, int chunk_size, float alpha,
+                             int n_iter, int causal, int estimate_diagonal, float scaling_factor,
+                             int dtype, cudaStream_t stream);
+
 /* Synchronises `stream`, returns the device status word of the current device
  * (ENTMAX_ATTN_OK or ENTMAX_ATTN_ETIMEOUT) and clears it. */
 int entmax_attn_status(cudaStream_t stream);

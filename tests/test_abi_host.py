@@ -285,3 +285,29 @@ def test_product_never_reaches_the_oracle():
                 for a in node.names:
                     assert not a.name.startswith("adaptive_sparse_attention_b200") or \
                         a.name == "adaptive_sparse_attention_b200.workloads", f
+
+
+def test_route_chunks_argument_checks(native):
+    """entmax_attn_route_chunks returns its argument errors before any launch (fake pointers)."""
+    lib = native.lib()
+    p = _fake(0x10000)
+    good = [p, p, p, p, 1, 4, 2, 300, 64, 16, 1.5, 10, 1, 1, 1.0, native.BF16, None]
+
+    def call(**kw):
+        a = list(good)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.entmax_attn_route_chunks(*a)
+
+    assert call(a1=None) == native.EINVAL       # null summaries
+    assert call(a2=None) == native.EINVAL       # null pi
+    assert call(a5=3) == native.EINVAL          # Hq not a multiple of Hkv
+    assert call(a8=2000) == native.EINVAL       # d > 1024
+    assert call(a9=0) == native.EINVAL          # chunk_size < 1
+    assert call(a10=1.0) == native.EINVAL       # alpha <= 1
+    assert call(a11=0) == native.EINVAL         # n_iter < 1
+    assert call(a13=2) == native.EINVAL         # estimate_diagonal not 0/1
+    assert call(a14=float("inf")) == native.EINVAL  # scaling_factor not finite
+    assert call(a15=7) == native.EINVAL         # dtype
+    assert call(a1=_fake(0x10001)) == native.EALIGN  # bf16 summaries on an odd address
+    assert call(a2=_fake(0x10002)) == native.EALIGN  # pi not 4-byte aligned
