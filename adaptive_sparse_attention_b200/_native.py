@@ -16,6 +16,8 @@ FLAG_CUDA_CORES = 1
 FLAG_ALL_FALLBACK = 2
 FLAG_NO_BLOCK_MASK = 8  # ENTMAX_ATTN_FLAG_NO_BLOCK_MASK
 FLAG_TEST_STALL = 4  # test hook of the bounded device waits (ENTMAX_ATTN_FLAG_TEST_STALL)
+FLAG_PENDING_ONLY = 16  # output pass over the tiles the fused tau pass left (PENDING_ONLY)
+FLAG_OUT_FP32 = 32  # fp32 out for bf16 inputs (ENTMAX_ATTN_FLAG_OUT_FP32)
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES
 
 _c_int, _c_float, _c_size_t, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
@@ -36,6 +38,9 @@ SIGNATURES = {
     "entmax_attn_tau_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),
+    "entmax_attn_tau_out_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_size_t, _c_int,
+                                          _c_int, _c_int, _c_int, _c_int, _c_float, _c_int,
+                                          _c_int, _vp, _c_int, _c_uint, _vp]),
     "entmax_attn_out_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _vp, _c_int, _c_int,
                                       _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),
@@ -53,6 +58,9 @@ SIGNATURES = {
     "entmax_attn_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                          _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
                                          _vp]),
+    "entmax_attn_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                      _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
+                                      _vp]),
     "entmax_attn_strerror": (ctypes.c_char_p, [_c_int]),
     "entmax_attn_last_cuda_error": (ctypes.c_char_p, []),
 }

@@ -198,6 +198,41 @@ def entmax_attn_fwd_noalloc(q, k, v, alpha: float = 1.5, n_iter: int = 10, causa
     return out, tau, block_mask
 
 
+def entmax_attn_fwd_host(q, k, v, alpha: float = 1.5, n_iter: int = 10, causal: bool = True,
+                         cu_seqlens=None, out=None, tau=None, block_mask=None, stream=None,
+                         synchronize: bool = True):
+    """Forward pass on CPU tensors (pin them for asynchronous, full-speed copies): the library
+    streams the problem through the GPU in chunks, the copies in and out overlapping the
+    computation.  cu_seqlens is an int32 CPU tensor.  Outputs are CPU tensors (allocated
+    pinned here unless passed in); with synchronize=False they are complete only once `stream`
+    has finished.  Returns (out, tau, block_mask)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or not t.is_contiguous() or t.dtype not in _DT:
+            raise ValueError(f"{name} must be a contiguous float32 or bfloat16 CPU tensor")
+    if k.dtype != q.dtype or v.dtype != q.dtype or v.shape != k.shape:
+        raise ValueError("q, k, v must share one dtype; v must have the shape of k")
+    if cu_seqlens is not None and (cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32 or
+                                   not cu_seqlens.is_contiguous()):
+        raise ValueError("cu_seqlens must be a contiguous int32 CPU tensor")
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    pin = torch.cuda.is_available()
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=pin)
+    if tau is None:
+        tau = torch.empty(q.shape[:-1], dtype=torch.float32, pin_memory=pin)
+    if block_mask is None:
+        block_mask = torch.empty(mask_words(B, Hq, T, cu_seqlens is not None), dtype=torch.int32,
+                                 pin_memory=pin)
+    rc = N.lib().entmax_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(tau),
+                                      _ptr(block_mask), B, Hq, Hkv, T, d, float(alpha),
+                                      int(n_iter), int(bool(causal)), _ptr(cu_seqlens),
+                                      _DT[q.dtype], _stream(stream))
+    N.check(rc, "entmax_attn_fwd_host")
+    if synchronize:
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+    return out, tau, block_mask
+
+
 def tau_pass(q, k, tau, block_mask, workspace, alpha=1.5, n_iter=10, causal=True,
              cu_seqlens=None, flags=0, stream=None):
     _check_inputs(q, k, None, cu_seqlens)
@@ -208,6 +243,21 @@ def tau_pass(q, k, tau, block_mask, workspace, alpha=1.5, n_iter=10, causal=True
                                       int(bool(causal)), _ptr(cu_seqlens), _DT[q.dtype],
                                       int(flags), _stream(stream))
     N.check(rc, "entmax_attn_tau_pass")
+
+
+def tau_out_pass(q, k, v, tau, block_mask, workspace, out, alpha=1.5, n_iter=10, causal=True,
+                 cu_seqlens=None, flags=0, stream=None):
+    """The tau pass that also writes out for every query tile whose rows' supports it held;
+    finish with out_pass(..., flags=FLAG_PENDING_ONLY) on the same workspace."""
+    _check_inputs(q, k, v, cu_seqlens)
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    rc = N.lib().entmax_attn_tau_out_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(tau),
+                                          _ptr(block_mask), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), B, Hq,
+                                          Hkv, T, d, float(alpha), int(n_iter),
+                                          int(bool(causal)), _ptr(cu_seqlens), _DT[q.dtype],
+                                          int(flags), _stream(stream))
+    N.check(rc, "entmax_attn_tau_out_pass")
 
 
 def out_pass(q, k, v, tau, workspace, out, alpha=1.5, causal=True, cu_seqlens=None, flags=0,
@@ -254,9 +304,26 @@ def entmax_attn_two_pass(q, k, v, alpha=1.5, n_iter=10, causal=True, cu_seqlens=
     """Both passes through the two-pass entry points with a torch-allocated workspace.
     Returns (out, tau, block_mask, workspace)."""
     out, tau, mask = alloc_outputs(q, k, cu_seqlens)
+    if flags & N.FLAG_OUT_FP32:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     ws = alloc_workspace(q, k, cu_seqlens) if workspace is None else workspace
     tau_pass(q, k, tau, mask, ws, alpha, n_iter, causal, cu_seqlens, flags, stream)
     out_pass(q, k, v, tau, ws, out, alpha, causal, cu_seqlens, flags, stream)
+    return out, tau, mask, ws
+
+
+def entmax_attn_fused(q, k, v, alpha=1.5, n_iter=10, causal=True, cu_seqlens=None, flags=0,
+                      workspace=None, stream=None):
+    """The forward pass of entmax_attn_fwd through the two-pass entry points with a
+    torch-allocated workspace: tau_out_pass, then out_pass over the pending query tiles.
+    Returns (out, tau, block_mask, workspace)."""
+    out, tau, mask = alloc_outputs(q, k, cu_seqlens)
+    if flags & N.FLAG_OUT_FP32:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    ws = alloc_workspace(q, k, cu_seqlens) if workspace is None else workspace
+    tau_out_pass(q, k, v, tau, mask, ws, out, alpha, n_iter, causal, cu_seqlens, flags, stream)
+    out_pass(q, k, v, tau, ws, out, alpha, causal, cu_seqlens, flags | N.FLAG_PENDING_ONLY,
+             stream)
     return out, tau, mask, ws
 
 

@@ -61,12 +61,13 @@ bool make_layout(int B, int Hq, int T, int has_cu, Layout* L) {
   return L->tiles < (int64_t(1) << 31);
 }
 
-// Workspace: [queue_count | count[tiles] | queue[tiles] | list[tiles][nkt_max] | key norms |
-// warm-up tiles], each section 256-byte aligned.
+// Workspace: [queue_count | count[tiles] | queue[tiles] | pending[tiles] | list[tiles][nkt_max] |
+// key norms | warm-up tiles], each section 256-byte aligned.
 struct WsView {
   int* queue_count;
   int* count;
   int* queue;
+  int* pending;
   int* list;
   float* norms;
   void* warm;
@@ -83,6 +84,8 @@ WsView ws_view(void* base, const Layout& L) {
   v.count = reinterpret_cast<int*>(p + off);
   off += align256(sizeof(int) * L.tiles);
   v.queue = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * L.tiles);
+  v.pending = reinterpret_cast<int*>(p + off);
   off += align256(sizeof(int) * L.tiles);
   v.list = reinterpret_cast<int*>(p + off);
   off += align256(sizeof(int) * static_cast<size_t>(L.tiles) * L.nkt_max);
@@ -176,6 +179,7 @@ void attach_workspace(ea::Problem* P, const WsView& v) {
   P->count = v.count;
   P->queue = v.queue;
   P->queue_count = v.queue_count;
+  P->pending = v.pending;
   P->norms = v.norms;
   P->warm = v.warm;
 }
@@ -225,10 +229,16 @@ size_t entmax_attn_workspace_min_bytes(int B, int Hq, int T, int has_cu_seqlens)
   return ws_view(nullptr, L).min_bytes;
 }
 
-int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
-                         void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
-                         int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
-                         int dtype, unsigned flags, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The tau pass; with v and out (not null) it also writes o for every query tile whose rows'
+// supports its candidate buffers hold and marks the other tiles pending for the output pass.
+int tau_pass_impl(const void* q, const void* k, const void* v, void* out, float* tau,
+                  uint32_t* block_mask, void* workspace, size_t workspace_bytes, int B, int Hq,
+                  int Hkv, int T, int d, float alpha, int n_iter, int causal,
+                  const int32_t* cu_seqlens, int dtype, unsigned flags, cudaStream_t stream) {
   Layout L;
   ea::Problem P;
   int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
@@ -239,21 +249,38 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
   if (!aligned16(tau) || (block_mask && !aligned16(block_mask)) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return ENTMAX_ATTN_EALIGN;
-  const WsView v = ws_view(workspace, L);
-  if (workspace_bytes < v.min_bytes) return ENTMAX_ATTN_ENOMEM;
+  const WsView wv = ws_view(workspace, L);
+  if (workspace_bytes < wv.min_bytes) return ENTMAX_ATTN_ENOMEM;
   int err = ENTMAX_ATTN_OK;
   P.status = status_ptr(&err);
   if (!P.status) return err;
   P.tau = tau;
   P.mask = block_mask;
-  attach_workspace(&P, v);
+  attach_workspace(&P, wv);
   P.force_fallback = (flags & ENTMAX_ATTN_FLAG_ALL_FALLBACK) ? 1 : 0;
   P.test_stall = (flags & ENTMAX_ATTN_FLAG_TEST_STALL) ? 1 : 0;
   P.no_mask = no_mask ? 1 : 0;
+  const bool fused = out != nullptr;
 
-  cudaError_t e = cudaMemsetAsync(v.queue_count, 0, sizeof(int), stream);
+  cudaError_t e = cudaMemsetAsync(wv.queue_count, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (use_tensor_cores(dtype, flags) && workspace_bytes >= v.bytes) {
+  if ((flags & ENTMAX_ATTN_FLAG_OUT_FP32) && !use_tensor_cores(dtype, flags))
+    return ENTMAX_ATTN_EINVAL;  // fp32 outputs of bf16 inputs: the tensor-core path only
+  P.out_f32 = (flags & ENTMAX_ATTN_FLAG_OUT_FP32) ? 1 : 0;
+  if (fused) {
+    if (use_tensor_cores(dtype, flags)) {
+      // the tensor-core tau kernel writes o and the pending flag of every query tile it solves
+      P.fused_out = 1;
+      P.v = v;
+      P.out = out;
+    } else {
+      // the CUDA-core tau kernel keeps no key ids: every query tile is left to the output pass
+      // (a nonzero flag; unused slots of a packed batch are skipped by the output pass anyway)
+      e = cudaMemsetAsync(wv.pending, 0xff, sizeof(int) * static_cast<size_t>(L.tiles), stream);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+  }
+  if (use_tensor_cores(dtype, flags) && workspace_bytes >= wv.bytes) {
     P.warm_levels = L.warm_levels;
     e = ea::launch_warm(P, stream);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -270,6 +297,29 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
   }
   if (e != cudaSuccess) return cuda_fail(e);
   return ENTMAX_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
+                         void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
+                         int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
+                         int dtype, unsigned flags, cudaStream_t stream) {
+  return tau_pass_impl(q, k, nullptr, nullptr, tau, block_mask, workspace, workspace_bytes, B,
+                       Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype, flags, stream);
+}
+
+int entmax_attn_tau_out_pass(const void* q, const void* k, const void* v, void* out, float* tau,
+                             uint32_t* block_mask, void* workspace, size_t workspace_bytes, int B,
+                             int Hq, int Hkv, int T, int d, float alpha, int n_iter, int causal,
+                             const int32_t* cu_seqlens, int dtype, unsigned flags,
+                             cudaStream_t stream) {
+  if (!v || !out) return ENTMAX_ATTN_EINVAL;
+  if (!aligned16(v) || !aligned16(out)) return ENTMAX_ATTN_EALIGN;
+  return tau_pass_impl(q, k, v, out, tau, block_mask, workspace, workspace_bytes, B, Hq, Hkv, T,
+                       d, alpha, n_iter, causal, cu_seqlens, dtype, flags, stream);
 }
 
 int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,
@@ -296,6 +346,10 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
   P.tau = const_cast<float*>(tau);
   attach_workspace(&P, wv);
   P.no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) ? 1 : 0;
+  P.pending_only = (flags & ENTMAX_ATTN_FLAG_PENDING_ONLY) ? 1 : 0;
+  if ((flags & ENTMAX_ATTN_FLAG_OUT_FP32) && !use_tensor_cores(dtype, flags))
+    return ENTMAX_ATTN_EINVAL;  // fp32 outputs of bf16 inputs: the tensor-core path only
+  P.out_f32 = (flags & ENTMAX_ATTN_FLAG_OUT_FP32) ? 1 : 0;
   cudaError_t e = use_tensor_cores(dtype, flags) ? ea::launch_out_tc(P, stream)
                                                  : ea::launch_out_simt(P, dtype, stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -368,11 +422,18 @@ int fwd_cached(const void* q, const void* k, const void* v, void* out, float* ta
     }
     c.bytes = need;
   }
-  rc = entmax_attn_tau_pass(q, k, tau, block_mask, c.ptr, need, B, Hq, Hkv, T, d, alpha, n_iter,
-                            causal, cu_seqlens, dtype, flags, stream);
+  if (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) {  // the pages' variant: the full output pass
+    rc = entmax_attn_tau_pass(q, k, tau, block_mask, c.ptr, need, B, Hq, Hkv, T, d, alpha,
+                              n_iter, causal, cu_seqlens, dtype, flags, stream);
+    if (rc != ENTMAX_ATTN_OK) return rc;
+    return entmax_attn_out_pass(q, k, v, tau, c.ptr, need, out, B, Hq, Hkv, T, d, alpha, causal,
+                                cu_seqlens, dtype, flags, stream);
+  }
+  rc = entmax_attn_tau_out_pass(q, k, v, out, tau, block_mask, c.ptr, need, B, Hq, Hkv, T, d,
+                                alpha, n_iter, causal, cu_seqlens, dtype, flags, stream);
   if (rc != ENTMAX_ATTN_OK) return rc;
   return entmax_attn_out_pass(q, k, v, tau, c.ptr, need, out, B, Hq, Hkv, T, d, alpha, causal,
-                              cu_seqlens, dtype, flags, stream);
+                              cu_seqlens, dtype, flags | ENTMAX_ATTN_FLAG_PENDING_ONLY, stream);
 }
 
 }  // namespace

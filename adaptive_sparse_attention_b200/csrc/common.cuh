@@ -68,6 +68,14 @@ struct Problem {
   int warm_levels;     // levels per group; 0 = no warm-up keys
   int kv_major;        // tau pass tile order: 1 = all query tiles of one key group before the
                        // next (keys larger than L2), 0 = slot-major (see tau_tile)
+  // Output from the candidates (tensor-core tau pass): with fused_out the tau pass also writes
+  // o for every query tile whose rows' supports its candidate buffers hold (all but the
+  // overflowed tiles) and sets pending[tile] to 0 there, 1 where the tile output pass must
+  // compute o.  With pending_only the output pass skips the tiles whose pending flag is 0.
+  int* pending;        // [tiles] (workspace)
+  int fused_out;
+  int pending_only;
+  int out_f32;         // out is fp32 (bf16 inputs, tensor-core path): no rounding of o to bf16
 };
 
 struct TileInfo {
@@ -255,9 +263,11 @@ struct Search {
 
 // ---------------------------------------------------------------------------------------------
 // Candidate buffers: for every (row r, segment g) -- column c = g * 128 + r -- up to NC
-// (raw score, key tile) pairs in shared memory, entry e at [e * kCols + c], so that the 32 rows
+// (raw score, key id) pairs in shared memory, entry e at [e * kCols + c], so that the 32 rows
 // of a warp hit 32 distinct banks whatever their fill levels.  A segment owns the keys 32 g ..
-// 32 g + 31 of every key tile.
+// 32 g + 31 of every key tile; the key id of key 128 kt + 32 g + i is 32 kt + i (kt < 2048, so it
+// fits 16 bits), from which both the key tile (mask bits) and the key itself (the output gather)
+// are recovered.
 // ---------------------------------------------------------------------------------------------
 template <int NC>
 struct alignas(16) CandSmemT {
@@ -268,6 +278,7 @@ struct alignas(16) CandSmemT {
   float s[NC * kCols];
   uint16_t kt[NC * kCols];
   float rowmax[kTile];  // running max of the row over all segments (raw); see feed_warp
+  float tau_r[kTile];   // the row's tau once solved (read by the output gather)
   float m[kCols];       // segment max of raw scores
   float floor_[kCols];  // pruning floor (raw); -inf when the segment was never pruned
   int cnt[kCols];
@@ -344,7 +355,8 @@ struct RowCand {
 
 
 // Insertion of the passing values of one lane (src, buffer column col_src) when they do not fit
-// into its buffer.  Lane e < c0 holds old entry e, lane j holds value j of src's chunk (v).
+// into its buffer.  Lane e < c0 holds old entry e, lane j holds value j of src's chunk (v), whose
+// key id is kid0 + j.
 // Old entries and new values at or below the threshold th are dropped; if more than the buffer's
 // slots survive, the floor is raised by bisection to just above the (slots/2 + 1)-th largest
 // value, so that the slots/2 largest survive and the buffer has room again (entries below the floor
@@ -353,7 +365,7 @@ struct RowCand {
 // arguments; call with the whole warp converged.
 template <class CS>
 __device__ __forceinline__ void coop_insert(CS& cs, RowCand& rc, int src, int col_src,
-                                            float v, float th, int c0, int kt, int lane) {
+                                            float v, float th, int c0, int kid0, int lane) {
   const unsigned full = 0xffffffffu;
   float fl = __shfl_sync(full, rc.floor_, src);
   const float mm = __shfl_sync(full, rc.mx, src);
@@ -394,7 +406,7 @@ __device__ __forceinline__ void coop_insert(CS& cs, RowCand& rc, int src, int co
     const int at = no + __popc(bn & below);
     if (at < CS::kSlots) {
       cs.s[at * kCols + col_src] = v;
-      cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
+      cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kid0 + lane);
     }
   }
   if (lane == src) {
@@ -443,14 +455,20 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
   }
   // Most passing chunks hold a single value above the threshold, which is then the chunk max:
   // each such lane stores it itself, all at once.  The others go on below.
+  const int kid0 = kt * 32;  // key id of x[0] (see the candidate buffers)
   bool single = false;
   int incoming = 0;  // this lane's values above its threshold
   if (pass) {
+    int at1 = 0;     // position of the (last) value above it
 #pragma unroll
-    for (int i = 0; i < N; ++i) incoming += (x[i] > rc.thr) ? 1 : 0;  // >= 1: cmax > rc.thr
+    for (int i = 0; i < N; ++i) {  // >= 1: cmax > rc.thr
+      const bool up = x[i] > rc.thr;
+      incoming += up ? 1 : 0;
+      at1 = up ? i : at1;
+    }
     if (incoming == 1 && rc.cnt < CS::kSlots) {
       cs.s[rc.cnt * kCols + col] = cmax;
-      cs.kt[rc.cnt * kCols + col] = static_cast<uint16_t>(kt);
+      cs.kt[rc.cnt * kCols + col] = static_cast<uint16_t>(kid0 + at1);
       ++rc.cnt;
       single = true;
     }
@@ -465,12 +483,11 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
     const bool fits = pass && !single && rc.cnt + incoming <= CS::kSlots;
     if (fits) {
       int c = rc.cnt;
-      const uint16_t kt16 = static_cast<uint16_t>(kt);
 #pragma unroll
       for (int i = 0; i < N; ++i) {  // fixed trip count, predicated stores: no branches
         const bool take = x[i] > rc.thr;
         st_shared_if(take, &cs.s[c * kCols + col], x[i]);
-        st_shared_if(take, &cs.kt[c * kCols + col], kt16);
+        st_shared_if(take, &cs.kt[c * kCols + col], static_cast<uint16_t>(kid0 + i));
         c += take ? 1 : 0;
       }
       rc.cnt = c;
@@ -498,11 +515,11 @@ __device__ __forceinline__ void feed_warp(RowCand& rc, CS& cs, float* xrow, int 
       if ((take >> lane) & 1u) {
         const int at = c0 + __popc(take & below);
         cs.s[at * kCols + col_src] = v;
-        cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kt);
+        cs.kt[at * kCols + col_src] = static_cast<uint16_t>(kid0 + lane);
       }
       if (lane == src) rc.cnt = c0 + n;
     } else {
-      coop_insert(cs, rc, src, col_src, v, th, c0, kt, lane);
+      coop_insert(cs, rc, src, col_src, v, th, c0, kid0, lane);
     }
     __syncwarp();  // the exchange row is read by every lane before the next row overwrites it
   }
@@ -592,7 +609,10 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CS& cs, int tid,
     }
     const float tau = sr.tau;
     if (!valid) continue;
-    if (lane4 == 0) P.tau[t.qhead + t.seq_start + pos] = tau;
+    if (lane4 == 0) {
+      P.tau[t.qhead + t.seq_start + pos] = tau;
+      cs.tau_r[r] = tau;
+    }
     bool bad = false;
 #pragma unroll
     for (int g = 0; g < kSeg; ++g) {
@@ -605,7 +625,7 @@ __device__ void solve_rows(const Problem& P, const TileInfo& t, CS& cs, int tid,
 #pragma unroll
       for (int i = 0; i < CS::kSlots / 4; ++i) {
         if (P.c * raw[g][i] > tau) {
-          const int kt = cs.kt[(lane4 + 4 * i) * kCols + g * kTile + r];
+          const int kt = cs.kt[(lane4 + 4 * i) * kCols + g * kTile + r] >> 5;  // key id -> tile
           atomicOr(&cs.words[kt >> 5], 1u << (kt & 31));
         }
       }

@@ -251,6 +251,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// 32 consecutive output elements from fp32 words (TMEM), at element offset e of out: rounded to
+// bf16, or stored as fp32 when the caller asked for fp32 outputs (P.out_f32).  16-byte stores.
+__device__ __forceinline__ void store_out32(const Problem& P, int64_t e, const uint32_t (&u)[32]) {
+  if (P.out_f32) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(P.out) + e);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + e);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(u[8 * i + 0]), __uint_as_float(u[8 * i + 1]));
+      w.y = pack_bf16x2(__uint_as_float(u[8 * i + 2]), __uint_as_float(u[8 * i + 3]));
+      w.z = pack_bf16x2(__uint_as_float(u[8 * i + 4]), __uint_as_float(u[8 * i + 5]));
+      w.w = pack_bf16x2(__uint_as_float(u[8 * i + 6]), __uint_as_float(u[8 * i + 7]));
+      dst[i] = w;
+    }
+  }
+}
+
+// n zero output elements at element offset e (n a multiple of 8).
+__device__ __forceinline__ void zero_out(const Problem& P, int64_t e, int n) {
+  const int bytes = n * (P.out_f32 ? 4 : 2);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(P.out) + e * (P.out_f32 ? 4 : 2));
+  for (int i = 0; i < bytes / 16; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // p = [x]_+^beta for the output pass, where p is rounded to bf16 before the P V product.  For
 // beta = 3 + f near 3, x^beta = x^3 e^(f ln x) with the exponential cut after its linear term,
 // and log2 x taken from the bits of x by Mitchell's approximation (x = 2^e (1 + m) read as
@@ -382,6 +410,74 @@ __device__ __forceinline__ int warm_steps(const Problem& P, const TileInfo& t) {
   return warm_level(P, t) >= 0 ? 1 : 0;
 }
 
+// Output from the candidates.  Every key with p_ij > 0 has z_ij > tau_i >= m_i - 1, so once a
+// row's candidate buffers hold every key above their floor and tau lies above the floor (what
+// solve_rows checks; a tile that fails is queued for the overflow path), the row's support is
+// exactly its buffer entries with z > tau, and o_i = sum over them of p_ij v_j.  The support of a
+// row is a handful of keys where the tile output pass would multiply whole 128-key tiles of
+// mostly zero p; so the tau kernel computes o itself, right after the solve: p in fp32 from the
+// stored raw score (the value the output pass would recompute) and tau, v_j gathered from global
+// memory (L2), fp32 accumulation, one rounding to bf16 at the store.  The 4 lanes of a row
+// (consecutive threads) split the d columns, so a row's store is one contiguous d-element run.
+template <int D, int BK, class CS>
+__device__ __forceinline__ void gather_rows(const Problem& P, const TileInfo& t, const CS& cs,
+                                            int tid, int nthreads) {
+  constexpr int kDims = D / 4;     // columns per lane
+  constexpr int kVec = kDims / 8;  // 16-byte vectors (8 bf16) per lane
+  const int lane4 = tid & 3;
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(P.v) +
+                            (t.khead + t.seq_start) * D + lane4 * kDims;
+  const int64_t ob = (t.qhead + t.seq_start + t.row0) * D + lane4 * kDims;  // element offset
+  for (int r = tid >> 2; r < t.nrows; r += nthreads >> 2) {
+    const float tau = cs.tau_r[r];
+    float acc[kDims];
+#pragma unroll
+    for (int i = 0; i < kDims; ++i) acc[i] = 0.f;
+#pragma unroll 1
+    for (int g = 0; g < kSeg; ++g) {
+      const int col = g * kTile + r;
+      const int n = min(cs.cnt[col], CS::kSlots);
+#pragma unroll 1
+      for (int e = 0; e < n; ++e) {
+        const float x = P.c * cs.s[e * kCols + col] - tau;
+        if (!(x > 0.f)) continue;
+        const float p = entmax_p<BK>(x, P.beta);
+        const int id = cs.kt[e * kCols + col];
+        // key id -> key of the sequence; kept inside the sequence whatever the buffer holds
+        const int j = min((id >> 5) * kTile + g * 32 + (id & 31), t.seq_len - 1);
+        const uint4* src = reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(j) * D);
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+          const uint4 w = __ldg(src + u);
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[h]));
+            acc[8 * u + 2 * h] = fmaf(p, f.x, acc[8 * u + 2 * h]);
+            acc[8 * u + 2 * h + 1] = fmaf(p, f.y, acc[8 * u + 2 * h + 1]);
+          }
+        }
+      }
+    }
+    const int64_t oe = ob + static_cast<int64_t>(r) * D;
+    if (P.out_f32) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(P.out) + oe);
+#pragma unroll
+      for (int u = 0; u < 2 * kVec; ++u)
+        dst[u] = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
+                            __float_as_uint(acc[4 * u + 2]), __float_as_uint(acc[4 * u + 3]));
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + oe);
+#pragma unroll
+      for (int u = 0; u < kVec; ++u)
+        dst[u] = make_uint4(pack_bf16x2(acc[8 * u], acc[8 * u + 1]),
+                            pack_bf16x2(acc[8 * u + 2], acc[8 * u + 3]),
+                            pack_bf16x2(acc[8 * u + 4], acc[8 * u + 5]),
+                            pack_bf16x2(acc[8 * u + 6], acc[8 * u + 7]));
+    }
+  }
+}
+
 template <int D, int BK>
 struct TauSmem {
   static constexpr int kStages = tau_stages(D, BK);
@@ -398,6 +494,16 @@ struct TauSmem {
   uint32_t tmem_base;
   int abort;
 };
+
+// Every variant's shared memory (plus the 1024 bytes of alignment slack the launch adds) fits
+// the 227 KB a CTA may use.
+constexpr size_t kMaxSmemPerCta = 232448;
+static_assert(sizeof(TauSmem<128, kBetaOne>) + 1024 <= kMaxSmemPerCta, "tau smem, d = 128");
+static_assert(sizeof(TauSmem<128, kBetaTwo>) + 1024 <= kMaxSmemPerCta, "tau smem, d = 128");
+static_assert(sizeof(TauSmem<128, kBetaGeneral>) + 1024 <= kMaxSmemPerCta, "tau smem, d = 128");
+static_assert(sizeof(TauSmem<128, kBetaNear3>) + 1024 <= kMaxSmemPerCta, "tau smem, d = 128");
+static_assert(sizeof(TauSmem<64, kBetaGeneral>) + 1024 <= kMaxSmemPerCta, "tau smem, d = 64");
+static_assert(sizeof(TauSmem<64, kBetaNear3>) + 1024 <= kMaxSmemPerCta, "tau smem, d = 64");
 
 // Score warps only (named barrier 1): a barrier, and a barrier that also returns whether any
 // score thread passed a true flag (the same answer in every thread).
@@ -619,6 +725,10 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       if (score_warps_any(*abort != 0)) break;  // status already records the timeout
       solve_rows<BK>(P, t, cs, tid, kScoreThreads);
       score_warps_sync();
+      if (P.fused_out) {  // o from the candidates, unless the tile goes to the overflow path
+        if (!cs.fallback) gather_rows<D, BK>(P, t, cs, tid, kScoreThreads);
+        if (tid == 0) P.pending[t.tile_id] = cs.fallback ? 1 : 0;
+      }
       if (warp == 0) emit_tile_prefix(P, t, cs, lane);
       score_warps_sync();
       emit_tile_entries(P, t, cs, tid, kScoreThreads);
@@ -920,6 +1030,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   const int slot = gridDim.x - 1 - blockIdx.x;
   const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
+  if (P.pending_only && P.pending[t.tile_id] == 0) return;  // o already written by the tau pass
   // The list comes from the tau pass; clamping keeps every read inside this tile's list and key
   // range even if the workspace was never filled.
   const int cnt = list_count(P, t);
@@ -1059,28 +1170,15 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const bool o_ok = mbar_wait(&sm.o_full, 0, abort, P.status);
     tc_fence_after();
     constexpr int kHalfD = D / 2;
-    __nv_bfloat16* op =
-        static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D + half * kHalfD;
+    const int64_t oe = (t.qhead + t.seq_start + pos) * D + half * kHalfD;  // element offset
     if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (only after a failed tau pass)
-      uint4* dst = reinterpret_cast<uint4*>(op);
-      for (int e = 0; e < kHalfD / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      zero_out(P, oe, kHalfD);
     } else if (o_ok && !*abort) {
 #pragma unroll 1
       for (int c0 = 0; c0 < kHalfD; c0 += 32) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + kColO + half * kHalfD + c0, u);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(op + c0);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(u[8 * e + 0]), __uint_as_float(u[8 * e + 1]));
-            w.y = pack_bf16x2(__uint_as_float(u[8 * e + 2]), __uint_as_float(u[8 * e + 3]));
-            w.z = pack_bf16x2(__uint_as_float(u[8 * e + 4]), __uint_as_float(u[8 * e + 5]));
-            w.w = pack_bf16x2(__uint_as_float(u[8 * e + 6]), __uint_as_float(u[8 * e + 7]));
-            dst[e] = w;
-          }
-        }
+        if (row_ok) store_out32(P, oe + c0, u);
       }
     }
   }
@@ -1163,6 +1261,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const TileInfo ta = map_tile(P, slot, 2 * blockIdx.y, blockIdx.z);
   if (!ta.valid) return;
   const TileInfo tb = map_tile(P, slot, 2 * blockIdx.y + 1, blockIdx.z);
+  // o of both heads already written by the tau pass (one pending head recomputes both)
+  if (P.pending_only && P.pending[ta.tile_id] == 0 && P.pending[tb.tile_id] == 0) return;
   // Lists from the tau pass, clamped so that no workspace content sends a read outside them.
   const int cnt_a = list_count(P, ta);
   const int cnt_b = list_count(P, tb);
@@ -1350,14 +1450,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const bool o_ok = mbar_wait(&sm.o_full, 0, abort, P.status);
     tc_fence_after();
     constexpr int kHalfD = D / 2;
-    __nv_bfloat16* op =
-        static_cast<__nv_bfloat16*>(P.out) + (t.qhead + t.seq_start + pos) * D + half * kHalfD;
+    const int64_t oe = (t.qhead + t.seq_start + pos) * D + half * kHalfD;  // element offset
     // Full tiles at d = 128: the four warps of a (head, half) stage their 32 rows x 64 columns
     // in the key ring (idle once o_full has arrived: every key tile loaded has been used) as one
     // 128-row box in the 128-byte swizzled layout, and one TMA store writes it.  box_tile is the
     // same for the four warps (it depends on the head only), so all four reach the barrier; the
     // store is issued only if every one of them staged its rows (no timeout, no abort).
-    const bool box_tile = D == 128 && cnt > 0 && t.nrows == kTile;
+    const bool box_tile = D == 128 && cnt > 0 && t.nrows == kTile && !P.out_f32;
     if (box_tile) {
       const bool staged = o_ok && !*abort;
       const int box = (warp - kScoreWarp0) >> 2;  // (head, half) = (box >> 1, box & 1)
@@ -1390,26 +1489,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tma_store_2d_and_wait(&tmo, stage, half * kHalfD,
                               static_cast<int>(t.qhead + t.seq_start + t.row0));
     } else if (o_ok && !*abort && cnt == 0 && row_ok) {  // no listed tile (failed tau pass only)
-      uint4* dst = reinterpret_cast<uint4*>(op);
-      for (int e = 0; e < kHalfD / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      zero_out(P, oe, kHalfD);
     } else if (o_ok && !*abort) {
 #pragma unroll 1
       for (int c0 = 0; c0 < kHalfD; c0 += 32) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + kPairColO + static_cast<uint32_t>(x * 128 + half * kHalfD + c0),
                   u);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(op + c0);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(u[8 * e + 0]), __uint_as_float(u[8 * e + 1]));
-            w.y = pack_bf16x2(__uint_as_float(u[8 * e + 2]), __uint_as_float(u[8 * e + 3]));
-            w.z = pack_bf16x2(__uint_as_float(u[8 * e + 4]), __uint_as_float(u[8 * e + 5]));
-            w.w = pack_bf16x2(__uint_as_float(u[8 * e + 6]), __uint_as_float(u[8 * e + 7]));
-            dst[e] = w;
-          }
-        }
+        if (row_ok) store_out32(P, oe + c0, u);
       }
     }
   }

@@ -3,8 +3,11 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
 
-A step is one full forward pass (tau pass + output pass) over the workload's synthetic batch,
-with the inputs already resident in HBM.  The metric is effective TFLOP/s: 4 d FLOPs per
+A step is one full forward pass over the workload's synthetic batch, with the inputs already
+resident in HBM: the tau pass, which also writes the output of every query tile whose rows'
+supports its candidate buffers held, then the tile output pass over the query tiles left
+pending (those whose candidates overflowed).  The same step on the tile path (tau pass, then
+the output pass over every query tile's active key tiles) is timed beside it.  The metric is effective TFLOP/s: 4 d FLOPs per
 causally valid (query, key) pair inside the active 128 x 128 tiles (recomputed scores + p V),
 summed over heads and batch, divided by the step time; tokens/s and the fraction of the
 measured bf16 dense tensor-core peak ride along.  Rank 0 prints one JSON line.
@@ -33,7 +36,7 @@ sys.path.insert(0, ROOT)
 from adaptive_sparse_attention_b200 import api as ea  # noqa: E402
 from adaptive_sparse_attention_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
-DEFAULT_WORKLOAD = "b2_t16k_gqa4_bf16_d128_a2"
+DEFAULT_WORKLOAD = "t128k_gqa4_bf16_d128_a1.5"
 METRIC = "effective TFLOP/s and tokens/s of entmax attention fwd; % of bf16 TC peak"
 TILE = 128
 L2_BYTES = 126 * 2**20
@@ -312,110 +315,198 @@ def workload_config(w, world):
 
 
 def launches_per_step(w) -> int:
-    """Kernels of one step (tau pass + output pass) on the library's full workspace: the tau
-    kernel, the overflow kernel and the output kernel, plus for bf16 problems with at least 1024
-    keys the key-norm and warm-up selection kernels of the tau pass."""
+    """Kernels of one step on the library's full workspace: the tau kernel, the overflow kernel
+    and the output kernel, plus for bf16 problems with at least 1024 keys the key-norm and
+    warm-up selection kernels of the tau pass."""
     return 3 + (2 if w.dtype == "bf16" and w.T >= 1024 else 0)
+
+
+# The forward pass, three ways through the C ABI's two-pass entry points:
+#   fused    entmax_attn_tau_out_pass (tau, mask, lists, and o of every query tile whose rows'
+#            supports the tau pass held) + entmax_attn_out_pass over the pending tiles only:
+#            the path entmax_attn_fwd takes, and the step this benchmark times;
+#   tile     entmax_attn_tau_pass + entmax_attn_out_pass over every query tile's active key
+#            tiles (o recomputed tile by tile on the tensor cores), reported beside it;
+#   nomask   the variant without block mask (--no-block-mask).
+MODES = ("fused", "tile", "nomask")
+
+
+class Problem:
+    """Device copies of one workload's inputs, outputs and workspace."""
+
+    def __init__(self, w, rank, local):
+        self.w = w
+        self.dev = torch.device("cuda", local)
+        self.host = make_inputs(w, seed=rank)
+        q, k, v, cu = self.host
+        self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+        self.q, self.k, self.v = q.to(self.dev), k.to(self.dev), v.to(self.dev)
+        self.cu = cu.to(self.dev) if cu is not None else None
+        self.alpha = _alpha_f32(w.alpha)
+        self.stream = torch.cuda.current_stream(self.dev)
+        self.out, self.tau, self.mask = ea.alloc_outputs(self.q, self.k, self.cu)
+        self.ws = ea.alloc_workspace(self.q, self.k, self.cu)
+
+    def step(self, mode, ev=None):
+        from adaptive_sparse_attention_b200 import _native
+        w, s = self.w, self.stream
+        a = (self.q, self.k)
+        if ev:
+            ev[0].record(s)
+        if mode == "fused":
+            ea.tau_out_pass(*a, self.v, self.tau, self.mask, self.ws, self.out, self.alpha,
+                            w.n_iter, w.causal, self.cu, stream=s)
+            flags = _native.FLAG_PENDING_ONLY
+        else:
+            flags = _native.FLAG_NO_BLOCK_MASK if mode == "nomask" else 0
+            ea.tau_pass(*a, self.tau, self.mask, self.ws, self.alpha, w.n_iter, w.causal,
+                        self.cu, flags=flags, stream=s)
+        if ev:
+            ev[1].record(s)
+        ea.out_pass(*a, self.v, self.tau, self.ws, self.out, self.alpha, w.causal, self.cu,
+                    flags=flags, stream=s)
+        if ev:
+            ev[2].record(s)
+
+    def time(self, mode, steps, warmup, world, sampler=None):
+        """(ms per step of this rank, per-step tau-pass ms, per-step output-pass ms, overflow
+        tiles), CUDA events on the launching stream, barrier + synchronize on both sides."""
+        for _ in range(warmup):
+            self.step(mode)
+        torch.cuda.synchronize()
+        assert ea.status(self.stream) == 0
+        nfb = ea.fallback_tiles(self.ws, self.stream)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with (sampler if sampler is not None else _NullCtx()):
+            start.record(self.stream)
+            for i in range(steps):
+                self.step(mode, evs[i])
+            stop.record(self.stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        st = ea.status(self.stream)
+        assert st == 0, f"device status {st}"
+        return (start.elapsed_time(stop) / steps, [e[0].elapsed_time(e[1]) for e in evs],
+                [e[1].elapsed_time(e[2]) for e in evs], nfb)
+
+    def pair_counts(self):
+        """(pairs inside active tiles, all causally valid pairs) from the last masked tau pass."""
+        w = self.w
+        bits = ea.decode_block_mask(self.mask.cpu().numpy(), w.B, w.Hq, w.T, self.host[3])
+        return count_pairs(w, bits, self.host[3])
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def secondary(args):
+    """The other target workload measured in the same run (16K with 128K and back)."""
+    if args.also == "none":
+        return []
+    if args.also != "auto":
+        return [n for n in args.also.split(",") if n and n != args.workload]
+    pair = ("t128k_gqa4_bf16_d128_a1.5", "b2_t16k_gqa4_bf16_d128_a2")
+    if args.workload in pair and not args.no_block_mask:
+        return [pair[1] if args.workload == pair[0] else pair[0]]
+    return []
 
 
 def run_native(args, rank, world, local):
     w = WORKLOADS[args.workload]
-    dev = torch.device("cuda", local)
-    q, k, v, cu = make_inputs(w, seed=rank)
-    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    cud = cu.to(dev) if cu is not None else None
-    alpha = _alpha_f32(w.alpha)
-    stream = torch.cuda.current_stream(dev)
-    out, tau, mask = ea.alloc_outputs(qd, kd, cud)
-    ws = ea.alloc_workspace(qd, kd, cud)
-
-    from adaptive_sparse_attention_b200 import _native
+    pb = Problem(w, rank, local)
     nm = args.no_block_mask
-    flags = _native.FLAG_NO_BLOCK_MASK if nm else 0
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, flags=flags,
-                    stream=stream)
-        if ev:
-            ev[1].record(stream)
-        ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, flags=flags, stream=stream)
-        if ev:
-            ev[2].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert ea.status(stream) == 0
-    nfb = ea.fallback_tiles(ws, stream)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        stop.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    total_ms = start.elapsed_time(stop)
-    t_tau = [e[0].elapsed_time(e[1]) for e in evs]
-    t_out = [e[1].elapsed_time(e[2]) for e in evs]
-    ms_step = max_over_ranks(total_ms / args.steps, world)
-    st = ea.status(stream)
-    assert st == 0, f"device status {st}"
+    mode = "nomask" if nm else "fused"
+    clk = ClockSampler(local)  # samples the clocks during the timed region only
+    ms_one, t_tau, t_out, nfb = pb.time(mode, args.steps, args.warmup, world, sampler=clk)
+    ms_step = max_over_ranks(ms_one, world)
 
     if nm:  # the mask, for the effective FLOP count only: one masked tau pass, not timed
-        ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, stream=stream)
+        pb.step("tile")
         torch.cuda.synchronize()
-    bits = ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, cu)
-    act_pairs, dense_pairs = count_pairs(w, bits, cu)
+    act_pairs, dense_pairs = pb.pair_counts()
     eff_flops = 4 * w.d * act_pairs
     tau_flops = 2 * w.d * dense_pairs
-    out_flops = 4 * w.d * (dense_pairs if nm else act_pairs)  # the work the output pass does
+    q, k, v, cu = pb.host
     tokens = w.B * w.T * w.Hq if cu is None else w.T * w.Hq  # query rows (token x head)
     tokens_seq = w.B * w.T if cu is None else w.T
-    value = job_rate(eff_flops, total_ms / args.steps, world) / 1e12
+    value = job_rate(eff_flops, ms_one, world) / 1e12
+    dense_rate = job_rate(4 * w.d * dense_pairs, ms_one, world)
 
-    # end to end through the C ABI entry point: H2D of q, k, v from pinned host memory, the
-    # forward pass, D2H of out, every step
+    # the tile path (every query tile's output recomputed over its active key tiles on the
+    # tensor cores), on the same inputs, for comparison: same warm-up, same step count
+    tile = None
+    if not nm:
+        ms_t, tt_tau, tt_out, _ = pb.time("tile", args.steps, args.warmup, world)
+        ms_t = max_over_ranks(ms_t, world)
+        out_tile = float(np.mean(tt_out))
+        tile = {"ms_per_step": ms_t, "value": job_rate(eff_flops, ms_t, world) / 1e12,
+                "ms_tau_pass": float(np.mean(tt_tau)), "ms_out_pass": out_tile,
+                "out_pass_tflops": eff_flops / (out_tile * 1e-3) / 1e12}
+
+    # end to end through the C ABI: inputs and outputs in pinned host memory, every step.  The
+    # masked path goes through entmax_attn_fwd_host (the library streams (batch row, kv head)
+    # chunks: copies in and out overlap the computation); the variant without block mask
+    # copies with torch around entmax_attn_fwd_no_block_mask.
+    qd, kd, vd, cud, out, tau, mask, stream = (pb.q, pb.k, pb.v, pb.cu, pb.out, pb.tau, pb.mask,
+                                               pb.stream)
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
-
-    def fwd():
-        if nm:
-            ea.entmax_attn_fwd_no_block_mask(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau,
-                                             stream=stream)
-        else:
-            ea.entmax_attn_fwd(qd, kd, vd, alpha, w.n_iter, w.causal, cud, out, tau, mask,
-                               stream=stream)
-
     outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    tauh = torch.empty(tau.shape, dtype=tau.dtype).pin_memory()
+    maskh = torch.empty(mask.shape, dtype=mask.dtype).pin_memory()
+
+    def fwd_e2e():
+        if nm:
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            ea.entmax_attn_fwd_no_block_mask(qd, kd, vd, pb.alpha, w.n_iter, w.causal, cud, out,
+                                             tau, stream=stream)
+            outh.copy_(out, non_blocking=True)
+        else:
+            ea.entmax_attn_fwd_host(qh, kh, vh, pb.alpha, w.n_iter, w.causal, cu, out=outh,
+                                    tau=tauh, block_mask=maskh, stream=stream, synchronize=False)
+
     e2e_steps = max(2, min(args.steps, 5))
-    for _ in range(1):
-        qd.copy_(qh, non_blocking=True)
-        fwd()
-        outh.copy_(out, non_blocking=True)
+    for _ in range(2):
+        fwd_e2e()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        fwd()
-        outh.copy_(out, non_blocking=True)
+        fwd_e2e()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_one = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = max_over_ranks(e2e_one, world)
     e2e_rate = job_rate(eff_flops, e2e_one, world)
-    dense_rate = job_rate(4 * w.d * dense_pairs, total_ms / args.steps, world)
     assert ea.status(stream) == 0
+    d2h_bytes = out.numel() * out.element_size() + (0 if nm else tau.numel() * 4
+                                                    + mask.numel() * 4)
+
+    others = []
+    for name in secondary(args):
+        w2 = WORKLOADS[name]
+        p2 = Problem(w2, rank, local)
+        ms2, t2_tau, t2_out, nfb2 = p2.time("fused", args.steps, args.warmup, world)
+        a2, d2 = p2.pair_counts()
+        ms2_max = max_over_ranks(ms2, world)
+        v2 = job_rate(4 * w2.d * a2, ms2, world) / 1e12
+        others.append({"workload": name, "value": v2, "unit": "TFLOP/s", "ms_per_step": ms2_max,
+                       "frac_of_bf16_peak": None, "ms_tau_pass": float(np.mean(t2_tau)),
+                       "ms_out_pass": float(np.mean(t2_out)),
+                       "active_tile_pair_fraction": a2 / d2, "overflow_tiles": nfb2,
+                       "tau_pass_tflops": 2 * w2.d * d2 / (float(np.mean(t2_tau)) * 1e-3) / 1e12})
+        del p2
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return 0
@@ -424,7 +515,7 @@ def run_native(args, rank, world, local):
     mean_tau = float(np.mean(t_tau))
     mean_out = float(np.mean(t_out))
     dom_tau = mean_tau >= mean_out
-    timed_s = total_ms * 1e-3
+    timed_s = ms_one * args.steps * 1e-3
     sustained = timed_s > 1.0
     peak_key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
     if tc:
@@ -435,9 +526,11 @@ def run_native(args, rank, world, local):
         bound, unit = "alu", "TFLOP/s"
         peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
         peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock"
+    out_flops = 4 * w.d * (dense_pairs if nm else act_pairs)
     achieved = (tau_flops / (mean_tau * 1e-3) if dom_tau else out_flops / (mean_out * 1e-3)) / 1e12
-    traffic = ncu_traffic(w.name, "tau_pass" if dom_tau else "out_pass")
-    roofline = {"kernel": "tau_pass" if dom_tau else "out_pass", "bound": bound,
+    kname = ("tau_out_pass" if mode == "fused" else "tau_pass") if dom_tau else "out_pass"
+    traffic = ncu_traffic(w.name, kname)
+    roofline = {"kernel": kname, "bound": bound,
                 "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "peak_source": peak_note,
                 "algorithmic": ("2 d flops per causally valid pair (dense scores)" if dom_tau
@@ -446,12 +539,14 @@ def run_native(args, rank, world, local):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        fl, nr, dt, nt, thr = oracle_tile_sample(w, (q, k, v, cu), args.cpu_budget)
+        fl, nr, dt, nt, thr = oracle_tile_sample(w, pb.host, args.cpu_budget)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"{nt} whole 128-row query tiles ({nr} rows) drawn uniformly, "
                          f"{dt:.1f} s of fp64 oracle work"}
 
     bf16_peak = float(peaks["bf16_tflops"])
+    for o in others:
+        o["frac_of_bf16_peak"] = o["value"] / world / bf16_peak
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -459,8 +554,12 @@ def run_native(args, rank, world, local):
         "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": dict(workload_config(w, world),
                        variant="no_block_mask" if nm else "block_mask",
-                       l2=f"inputs {in_bytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB L2; "
-                          f"no flush" if in_bytes > L2_BYTES else "inputs fit in L2; no flush"),
+                       path=("tau pass + output pass over every causal tile" if nm else
+                             "tau pass with the output from its candidates + tile output pass "
+                             "over the overflowed query tiles"),
+                       l2=f"inputs {pb.in_bytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB "
+                          f"L2; no flush" if pb.in_bytes > L2_BYTES
+                       else "inputs fit in L2; no flush"),
         "tokens_per_s": world * tokens_seq / (ms_step * 1e-3),
         "query_rows_per_s": world * tokens / (ms_step * 1e-3),
         "frac_of_bf16_peak": value / world / bf16_peak,
@@ -470,13 +569,17 @@ def run_native(args, rank, world, local):
         "tau_pass_hbm_gbs": (q.numel() * q.element_size() + k.numel() * k.element_size()
                              + tau.numel() * 4 + mask.numel() * 4) / (mean_tau * 1e-3) / 1e9,
         "overflow_tiles": nfb,
+        "tile_path": tile,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_rate / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": out.numel() * out.element_size()},
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": pb.in_bytes,
+                "d2h_bytes_per_step": d2h_bytes,
+                "entry": ("entmax_attn_fwd_no_block_mask + torch copies" if nm
+                          else "entmax_attn_fwd_host (pinned host buffers)")},
         "gpu_launches": launches_per_step(w) * args.steps,
         "clocks": clk.summary(),
+        "other_workloads": others,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -611,6 +714,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (entmax_attn_bwd) instead of the forward pass")
+    ap.add_argument("--also", default="auto",
+                    help="other workloads timed in the same run (comma list, 'none'; 'auto': "
+                         "the 16K workload beside the 128K one and back)")
     ap.add_argument("--no-block-mask", action="store_true",
                     help="time the variant without block mask (output pass over every causal "
                          "tile); the effective FLOPs keep counting active tiles only")

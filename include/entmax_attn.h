@@ -81,6 +81,15 @@ extern "C" {
                                              mask and no tile lists (block_mask may be NULL), and
                                              the output pass visits every causally valid key tile.
                                              Give it to both passes. */
+#define ENTMAX_ATTN_FLAG_PENDING_ONLY 16u /* output pass only: visit only the query tiles that
+                                             the last entmax_attn_tau_out_pass on this
+                                             workspace left pending (its overflowed tiles) */
+#define ENTMAX_ATTN_FLAG_OUT_FP32 32u     /* bf16 inputs on the tensor-core path: out is float
+                                             (fp32 accumulations stored without rounding to
+                                             bf16), same layout.  Give it to every pass that
+                                             writes out (entmax_attn_tau_out_pass and
+                                             entmax_attn_out_pass); ENTMAX_ATTN_EINVAL with fp32
+                                             inputs or ENTMAX_ATTN_FLAG_CUDA_CORES. */
 #define ENTMAX_ATTN_FLAG_TEST_STALL 4u    /* test hook of the bounded waits: the tensor-core tau
                                              pass never requests its query tiles, so each of its
                                              CTAs gives up after one wait limit (about 2 s) and
@@ -88,10 +97,12 @@ extern "C" {
                                              status word; its outputs are void.  Use it on a
                                              problem of a few query tiles only. */
 
-/* Full forward pass: tau search + block mask, then the output pass over active tiles.
- * Writes out, tau and every word of block_mask.  Scratch memory (compact tile lists, overflow
- * queue) is allocated by the library on first use per (device, stream) with cudaMallocAsync on
- * `stream`, grown when a larger problem arrives, and kept until entmax_attn_release_workspaces().
+/* Full forward pass: entmax_attn_tau_out_pass (tau search, block mask, and the output of every
+ * query tile whose rows' supports the tau pass held), then entmax_attn_out_pass over the active
+ * tiles of the remaining (overflowed) query tiles.  Writes out, tau and every word of
+ * block_mask.  Scratch memory (compact tile lists, overflow queue, pending flags) is allocated
+ * by the library on first use per (device, stream) with cudaMallocAsync on `stream`, grown when a
+ * larger problem arrives, and kept until entmax_attn_release_workspaces().
  * Returns ENTMAX_ATTN_OK or an error code. */
 int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
                     uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
@@ -136,7 +147,25 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
                          int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
                          int dtype, unsigned flags, cudaStream_t stream);
 
-/* Output pass: o_i = sum over the listed key tiles of p_ij v_j, with p recomputed from tau. */
+/* Tau pass with the output: everything entmax_attn_tau_pass writes, and out for every query
+ * tile whose rows' supports the pass held in its candidate buffers (AdaSplash page, "AdaSplash
+ * with Block Masking": p_ij > 0 needs z_ij > tau_i >= max_j z_ij - 1, and these are the keys the
+ * pass keeps to find tau): o_i = sum_j p_ij v_j over those keys, p in fp32 from the pass's own
+ * scores and tau, fp32 accumulation, one rounding to the output dtype.  The other query tiles
+ * (those whose candidates overflowed into the multi-sweep search; every tile on the CUDA-core
+ * path) are marked pending in the workspace: complete out with entmax_attn_out_pass and
+ * ENTMAX_ATTN_FLAG_PENDING_ONLY on the same workspace, in stream order.  v and out as in
+ * entmax_attn_fwd (device, 16-byte aligned); the other arguments, flags and returns as
+ * entmax_attn_tau_pass (ENTMAX_ATTN_EINVAL for a null v or out). */
+int entmax_attn_tau_out_pass(const void* q, const void* k, const void* v, void* out, float* tau,
+                             uint32_t* block_mask, void* workspace, size_t workspace_bytes, int B,
+                             int Hq, int Hkv, int T, int d, float alpha, int n_iter, int causal,
+                             const int32_t* cu_seqlens, int dtype, unsigned flags,
+                             cudaStream_t stream);
+
+/* Output pass: o_i = sum over the listed key tiles of p_ij v_j, with p recomputed from tau
+ * (scores on the tensor cores, P rounded to bf16 for the P V product, fp32 accumulation).  With
+ * ENTMAX_ATTN_FLAG_PENDING_ONLY only the query tiles entmax_attn_tau_out_pass left pending. */
 int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,
                          const void* workspace, size_t workspace_bytes, void* out, int B, int Hq,
                          int Hkv, int T, int d, float alpha, int causal,
@@ -235,6 +264,29 @@ int entmax_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o
                             uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d,
                             float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
                             int dtype, cudaStream_t stream);
+
+/* The forward pass of entmax_attn_fwd on inputs and outputs in HOST memory.  q, k, v, out,
+ * tau, block_mask and cu_seqlens are host pointers with the layouts and sizes above (page-locked
+ * memory, e.g. from cudaHostAlloc, lets the copies run asynchronously and at full speed;
+ * pageable memory works but each copy then waits for the host).  Every (batch row, kv head)
+ * group -- packed batches: every kv head over all sequences -- is an independent problem and a
+ * contiguous run of every array, so the call cuts the problem into chunks of whole groups and
+ * streams them through a device staging buffer of two chunk slots: the copy in of chunk c + 1,
+ * the computation of chunk c (entmax_attn_fwd on `stream`) and the copy out of chunk c - 1
+ * overlap, with one cudaMemcpyAsync per contiguous run on two copy streams of the library.
+ * Asynchronous: the call returns once everything is enqueued, and every output is in host
+ * memory when `stream` has completed the work enqueued so far; keep the host buffers alive and
+ * unmodified until then.  The staging buffer, the device copy of cu_seqlens and the copy
+ * streams are allocated on first use per device and kept until the process exits; the
+ * forward's workspace is entmax_attn_fwd's.  Calls on one device share one pipeline and take
+ * turns (each call waits on the device for the previous one).  cu_seqlens (host) is checked on
+ * the host: cu_seqlens[0] == 0, nondecreasing, cu_seqlens[B] == T.  Returns ENTMAX_ATTN_OK,
+ * ENTMAX_ATTN_EINVAL (as entmax_attn_fwd, or a null pointer), ENTMAX_ATTN_ENOMEM (the staging
+ * buffer could not be allocated) or ENTMAX_ATTN_ECUDA. */
+int entmax_attn_fwd_host(const void* q, const void* k, const void* v, void* out, float* tau,
+                         uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
+                         int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                         cudaStream_t stream);
 
 /* Static text for a return code. */
 const char* entmax_attn_strerror(int code);

@@ -57,7 +57,16 @@ class GpuResult:
     fallback_tiles: int
 
 
-def run_gpu(w: Workload, inputs, flags: int = 0, use_fwd: bool = False) -> GpuResult:
+# The forward pass's paths through the C ABI:
+#   "fused": entmax_attn_tau_out_pass (o of every query tile whose rows' supports the tau pass
+#            held) + entmax_attn_out_pass over the pending tiles -- the path entmax_attn_fwd
+#            takes and bench.py times;
+#   "tile":  entmax_attn_tau_pass + entmax_attn_out_pass over every query tile's active tiles.
+PATHS = ("fused", "tile")
+
+
+def run_gpu(w: Workload, inputs, flags: int = 0, use_fwd: bool = False,
+            path: str = "fused") -> GpuResult:
     q, k, v, cu = inputs
     dev = torch.device("cuda:0")
     q, k, v = q.to(dev), k.to(dev), v.to(dev)
@@ -67,8 +76,8 @@ def run_gpu(w: Workload, inputs, flags: int = 0, use_fwd: bool = False) -> GpuRe
         out, tau, mask = ea.entmax_attn_fwd(q, k, v, alpha, w.n_iter, w.causal, cu_d)
         nfb = -1
     else:
-        out, tau, mask, ws = ea.entmax_attn_two_pass(q, k, v, alpha, w.n_iter, w.causal, cu_d,
-                                                     flags=flags)
+        run = ea.entmax_attn_fused if path == "fused" else ea.entmax_attn_two_pass
+        out, tau, mask, ws = run(q, k, v, alpha, w.n_iter, w.causal, cu_d, flags=flags)
         nfb = ea.fallback_tiles(ws)
     torch.cuda.synchronize()
     st = ea.status()
@@ -120,8 +129,11 @@ def all_tiles(w: Workload, cu):
     return tiles
 
 
-def compare(w: Workload, inputs, g: GpuResult, whole_tiles, loose_rows=None, label=""):
-    """Asserts parity on the given whole query tiles and loose rows.  Returns a summary dict."""
+def compare(w: Workload, inputs, g: GpuResult, whole_tiles, loose_rows=None, label="",
+            flat_bar: bool = False):
+    """Asserts parity on the given whole query tiles and loose rows.  Returns a summary dict.
+    flat_bar: o was stored in fp32 (ENTMAX_ATTN_FLAG_OUT_FP32), so its bar is the flat
+    out_tolerance, without the bf16 rounding of a stored bf16 output."""
     q, k, v, cu = inputs
     alpha = oracle.alpha_as_float32(w.alpha)
     groups = [tile_rows(w, cu, *t) for t in whole_tiles]
@@ -129,7 +141,7 @@ def compare(w: Workload, inputs, g: GpuResult, whole_tiles, loose_rows=None, lab
                                     if loose_rows is not None and len(loose_rows) else []))
     ref = oracle.attention_rows(q, k, v, alpha, w.causal, cu, rows)
     err_out = np.abs(g.out[rows] - ref["out"])
-    bar = out_bar(w, ref["out"])
+    bar = (np.full(ref["out"].shape, out_tolerance(w)) if flat_bar else out_bar(w, ref["out"]))
     max_out = float(err_out.max()) if err_out.size else 0.0
     over = float((err_out / bar).max()) if err_out.size else 0.0
     tau_g = g.tau[rows].astype(np.float64)

@@ -311,3 +311,32 @@ def test_route_chunks_argument_checks(native):
     assert call(a15=7) == native.EINVAL         # dtype
     assert call(a1=_fake(0x10001)) == native.EALIGN  # bf16 summaries on an odd address
     assert call(a2=_fake(0x10002)) == native.EALIGN  # pi not 4-byte aligned
+
+
+def test_host_entry_point_argument_checks(native):
+    """entmax_attn_fwd_host checks its arguments, host cu_seqlens included, before it touches
+    the GPU (fake pointers: never dereferenced on these paths)."""
+    import ctypes
+    lib = native.lib()
+    p = _fake(0x10000)
+
+    def call(B=2, Hq=4, Hkv=2, T=300, d=64, cu=None, dtype=native.BF16, null=None):
+        a = [p] * 6
+        if null is not None:
+            a[null] = None
+        return lib.entmax_attn_fwd_host(*a, B, Hq, Hkv, T, d, 1.5, 10, 1, cu, dtype, None)
+
+    for i in range(6):
+        assert call(null=i) == native.EINVAL  # a null host pointer
+    assert call(Hq=3) == native.EINVAL        # Hq not a multiple of Hkv
+    assert call(T=0) == native.EINVAL
+    assert call(dtype=9) == native.EINVAL
+
+    def cu(vals):
+        arr = (ctypes.c_int32 * len(vals))(*vals)
+        return ctypes.cast(arr, ctypes.c_void_p), arr
+
+    bad = [[1, 100, 300], [0, 200, 100, 300], [0, 100, 299]]  # start, order, end
+    for vals in bad:
+        ptr, keep = cu(vals)
+        assert call(B=len(vals) - 1, T=300, cu=ptr) == native.EINVAL, vals

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import adaptive_sparse_attention_b200 as ea
 from adaptive_sparse_attention_b200 import _native
 from adaptive_sparse_attention_b200.workloads import WORKLOADS, make_inputs, random_case
 import parity
@@ -45,11 +46,12 @@ def _sample_tiles(w, cu, per_head, rng, include_ends=True):
     return tiles
 
 
+@pytest.mark.parametrize("path", parity.PATHS)
 @pytest.mark.parametrize("name", ["t256_fp32_d64_a1.5", "t4k_bf16_d64_a1.5"])
-def test_small_workloads_every_row(oracle, name):
+def test_small_workloads_every_row(oracle, name, path):
     w = WORKLOADS[name]
     inputs = make_inputs(w)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     s = parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=name)
     print(name, s, "fallback tiles", g.fallback_tiles)
 
@@ -61,10 +63,11 @@ def test_small_workload_full_forward_entry_point(oracle):
     parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label="fwd")
 
 
-def test_16k_gqa_sparsemax_sampled(oracle):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_16k_gqa_sparsemax_sampled(oracle, path):
     w = WORKLOADS["b2_t16k_gqa4_bf16_d128_a2"]
     inputs = make_inputs(w)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     rng = np.random.default_rng(1000)
     tiles = _sample_tiles(w, None, 1, rng, include_ends=False)
     tiles += [(b, h, 0, 127) for b in range(2) for h in (0, 31)]  # longest rows
@@ -73,10 +76,11 @@ def test_16k_gqa_sparsemax_sampled(oracle):
     print(w.name, s, "fallback tiles", g.fallback_tiles)
 
 
-def test_varlen_gqa_alpha1333_sampled(oracle):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_varlen_gqa_alpha1333_sampled(oracle, path):
     w = WORKLOADS["varlen4_32k_gqa4_bf16_d128_a1.333"]
     inputs = make_inputs(w)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     rng = np.random.default_rng(1001)
     tiles = _sample_tiles(w, inputs[3], 1, rng, include_ends=True)
     loose = rng.choice(w.Hq * w.T, size=2048, replace=False)
@@ -84,12 +88,13 @@ def test_varlen_gqa_alpha1333_sampled(oracle):
     print(w.name, s, "fallback tiles", g.fallback_tiles)
 
 
-def test_128k_sampled_rows(oracle):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_128k_sampled_rows(oracle, path):
     """512 seeded rows per head (one-sided mask) plus 4 whole query tiles per head
     (two-sided)."""
     w = WORKLOADS["t128k_gqa4_bf16_d128_a1.5"]
     inputs = make_inputs(w)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     loose, tiles = [], []
     for h in range(w.Hq):
         rng = np.random.default_rng(1000 + h)
@@ -119,11 +124,12 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("path", parity.PATHS)
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 @pytest.mark.parametrize("name,kw", SMALL, ids=[s[0] for s in SMALL])
-def test_small_cases(oracle, name, kw, dtype):
+def test_small_cases(oracle, name, kw, dtype, path):
     w, inputs = random_case(dtype=dtype, name=name, seed=7, **kw)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"{name}/{dtype}")
 
 
@@ -132,16 +138,18 @@ def test_small_cases(oracle, name, kw, dtype):
                          ids=["cuda_cores", "all_fallback", "cuda_cores_all_fallback"])
 @pytest.mark.parametrize("name,kw", [SMALL[5], SMALL[7], SMALL[8]],
                          ids=[SMALL[5][0], SMALL[7][0], SMALL[8][0]])
-def test_alternate_paths(oracle, name, kw, flags):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_alternate_paths(oracle, name, kw, flags, path):
     w, inputs = random_case(dtype="bf16", name=name, seed=11, **kw)
-    g = parity.run_gpu(w, inputs, flags=flags)
+    g = parity.run_gpu(w, inputs, flags=flags, path=path)
     if flags & _native.FLAG_ALL_FALLBACK:
         assert g.fallback_tiles == sum(1 for _ in parity.all_tiles(w, inputs[3]))
     parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"{name}/{flags}")
 
 
 @pytest.mark.parametrize("alpha", [1.333, 1.5, 2.0])
-def test_candidate_overflow_is_exact(oracle, alpha):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_candidate_overflow_is_exact(oracle, alpha, path):
     """Tiny score spread (q, k scaled by 1/16) puts hundreds of keys within 1 of the row max, so
     rows overflow the 64-slot candidate buffers; tied keys (repeated rows of k) defeat the
     pruning too.  The result must stay exact."""
@@ -151,14 +159,15 @@ def test_candidate_overflow_is_exact(oracle, alpha):
     k = (k.float() / 16).to(torch.bfloat16)
     k[:, :, 200:400] = k[:, :, 200:201]  # 200 identical keys
     inputs = (q, k, v, cu)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     assert g.fallback_tiles > 0
     parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"overflow/{alpha}")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
-def test_equal_scores_give_uniform_rows(oracle, alpha, dtype):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_equal_scores_give_uniform_rows(oracle, alpha, dtype, path):
     """q = 0 makes every score of a row equal, so p is uniform over the row's valid keys
     (p_j = 1/n for all j, tau = -n^(1-alpha)) and o is the mean of the value prefix.  Every key
     is then a candidate: rows longer than the buffers take the overflow path.  Checked against
@@ -167,7 +176,7 @@ def test_equal_scores_give_uniform_rows(oracle, alpha, dtype):
                                    name="equal_scores", seed=13)
     q = torch.zeros_like(q)
     inputs = (q, k, v, cu)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     assert g.fallback_tiles > 0
     parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"equal_scores/{dtype}/{alpha}")
     vf = v.double().numpy()
@@ -183,7 +192,8 @@ def test_equal_scores_give_uniform_rows(oracle, alpha, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-def test_far_apart_scores_give_one_hot_rows(oracle, dtype):
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_far_apart_scores_give_one_hot_rows(oracle, dtype, path):
     """q scaled by 16 against spiked keys spreads the scores of a row over hundreds of units, so
     most rows put all their mass on one key (p one-hot, o = that key's value row).  The mask then
     holds few tiles per row; the result must match the oracle, including rows whose support
@@ -192,5 +202,37 @@ def test_far_apart_scores_give_one_hot_rows(oracle, dtype):
                                    spike_frac=0.02, spike_scale=4.0, name="one_hot", seed=17)
     q = (q.float() * 16).to(q.dtype)
     inputs = (q, k, v, cu)
-    g = parity.run_gpu(w, inputs)
+    g = parity.run_gpu(w, inputs, path=path)
     parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"one_hot/{dtype}")
+
+
+@pytest.mark.parametrize("name,kw", [SMALL[5], SMALL[8]], ids=[SMALL[5][0], SMALL[8][0]])
+def test_tau_out_pass_writes_exactly_the_settled_tiles(oracle, name, kw):
+    """entmax_attn_tau_out_pass alone (no output pass after it): every query tile it did not
+    leave pending holds its final output, and the tiles it left pending are untouched (the
+    output was NaN-filled before).  Forcing every tile through the overflow path must leave
+    every row untouched."""
+    w, inputs = random_case(dtype="bf16", name=name, seed=19, **kw)
+    q, k, v, cu = (t.cuda() if t is not None else None for t in inputs)
+    alpha = oracle.alpha_as_float32(w.alpha)
+    for flags, expect_all_pending in ((0, False), (_native.FLAG_ALL_FALLBACK, True)):
+        out, tau, mask = ea.alloc_outputs(q, k, cu)
+        out.fill_(float("nan"))
+        ws = ea.alloc_workspace(q, k, cu)
+        ea.tau_out_pass(q, k, v, tau, mask, ws, out, alpha, w.n_iter, w.causal, cu, flags=flags)
+        torch.cuda.synchronize()
+        assert ea.status() == 0
+        nan_rows = torch.isnan(out.float()).any(dim=-1).cpu().numpy().ravel()
+        valid_rows = np.concatenate([parity.tile_rows(w, inputs[3], *t)
+                                     for t in parity.all_tiles(w, inputs[3])])
+        if expect_all_pending:
+            assert nan_rows[valid_rows].all()
+            continue
+        ea.out_pass(q, k, v, tau, ws, out, alpha, w.causal, cu, flags=_native.FLAG_PENDING_ONLY)
+        torch.cuda.synchronize()
+        g = parity.GpuResult(out.float().cpu().numpy().reshape(-1, w.d), tau.cpu().numpy().ravel(),
+                             ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, inputs[3]),
+                             ea.fallback_tiles(ws))
+        parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"fused/{name}")
+        # the rows the tau pass wrote are the rows of the tiles it did not queue
+        assert nan_rows[valid_rows].sum() <= g.fallback_tiles * 128

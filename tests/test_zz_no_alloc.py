@@ -5,10 +5,10 @@ It exists for callers that cannot allocate device memory while they run (code in
 allocator or memory-pool callback, runtimes with a fixed post-start-up footprint, replayed
 launch sequences); its scratch is a fixed device array shared by all calls.  Two calls in a row
 on different problems check that what the first call leaves in the shared array does not leak
-into the second: each call's output is compared with entmax_attn_fwd's within the forward
-pass's parity bars, and with the fp64 oracle on every row (tau, output and the block mask under
-the exemption rule; tau may differ between runs by an ulp, so no bit-equality is asked of the
-masks of two runs).  A last test checks the property itself: after a first call, further calls
+into the second: each call's output is compared with the fp64 oracle on every row (tau, output
+and the block mask under the exemption rule; tau may differ between runs by an ulp, so no
+bit-equality is asked of the masks of two runs), and with entmax_attn_fwd's within twice the
+forward pass's parity bar.  A last test checks the property itself: after a first call, further calls
 leave the device's free memory unchanged.  This file sorts last so that a failure here, with -x,
 comes after every other test has run; it also passes on its own in a fresh process.
 """
@@ -63,12 +63,16 @@ def test_noalloc_matches_fwd_and_oracle_on_two_calls_in_a_row(oracle):
         assert ea.status() == 0
         r = _result(w, *ref, cu)
         g = _result(w, *got, cu)
-        # against the existing entry point, within the parity bars
-        ref_o = r.out.astype(np.float64)
-        assert np.all(np.abs(g.out - r.out) <= parity.out_bar(w, ref_o)), w.name
-        assert np.max(np.abs(g.tau - r.tau) / np.maximum(1.0, np.abs(r.tau))) <= parity.TAU_RTOL
         # against the oracle, every row
         parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"noalloc {w.name}")
+        # against the existing entry point: each lies within the parity bar of the exact value,
+        # so the two lie within twice the bar of each other.  (Without room for the warm-up keys
+        # the allocation-free call may send other query tiles through the overflow path, whose
+        # output comes from the tile pass with p rounded to bf16 rather than from the tau pass's
+        # fp32 gather, so the two need not round alike.)
+        ref_o = r.out.astype(np.float64)
+        assert np.all(np.abs(g.out - r.out) <= 2 * parity.out_bar(w, ref_o)), w.name
+        assert np.max(np.abs(g.tau - r.tau) / np.maximum(1.0, np.abs(r.tau))) <= parity.TAU_RTOL
 
 
 def test_noalloc_allocates_no_device_memory(oracle):
