@@ -1,17 +1,19 @@
 // tc.cu -- tensor-core (tcgen05) kernels of the entmax attention forward pass, bf16, sm_100a.
 //
-// tau_tc_kernel (one CTA of 576 threads per 128-row query tile):
+// tau_tc_kernel (persistent, one CTA of 608 threads per SM, one 128-row query tile at a time):
 //   warp 16     TMA producer: the query tile, then the tile's key tiles through a 4-stage
 //               shared-memory ring (128B-swizzled, K-major).
-//   warp 17     allocates tensor memory and issues the tcgen05.mma of S = Q K^T (M = N = 128,
-//               K = d, fp32 accumulators) into one of four TMEM score buffers, so that the score
-//               warps can fall up to three tiles behind during a burst of insertions.
+//   warps 17-18 issue the tcgen05.mma of S = Q K^T (M = N = 128, K = d, fp32 accumulators) into
+//               one of four TMEM score buffers, so that the score warps can fall up to three
+//               tiles behind during a burst of insertions; the two warps take alternate key
+//               tiles (warp 17 also allocates tensor memory).  A 3-stage ring (d = 128 with the
+//               larger candidate buffers) keeps one issuing warp.
 //   warps 0..15 score warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = query row),
 //               columns 32 g .. 32 g + 31 with g = w / 4, i.e. one 32-key segment of every key
 //               tile, into the segment's candidate buffer (common.cuh); the four segments of a
 //               row share its running max.
-//   then the score warps solve tau per row (4-lane groups) and warp 0 writes the block mask
-//   and the compact tile list.
+//   then the score warps solve tau per row (4-lane groups), compute the output of the rows
+//   from their candidates (gather_rows), and write the block mask and the compact tile list.
 //
 // out_tc_kernel (one CTA of 384 threads per query tile, over the listed key tiles only):
 //   warp 0      TMA producer of the query tile and the key tiles (3-stage ring; a key tile is
@@ -395,6 +397,21 @@ __host__ __device__ constexpr int tau_stages(int d, int bk) {
 }
 constexpr int kMainSBufs = 4;   // TMEM score buffers
 
+// MMA-issuing warps of the tau kernel.  A tcgen05.mma issue returns only once the tensor pipe
+// has room, a few instructions deep, so a single issuing thread cannot run ahead of the pipe:
+// every cycle it spends on its barrier waits and loop overhead between two groups of products
+// leaves the pipe idle (clock64 counters: ~500 of ~1200 cycles per key tile).  Two warps that
+// take alternate key tiles hide one's waits behind the other's issue.  Every key stage and every
+// score buffer must then belong to one warp (stage and buffer counts divisible by the warp
+// count), so that each warp waits on each barrier's phases in order: a warp that could wait on
+// a phase two ahead of a barrier would see its parity as completed.
+__host__ __device__ constexpr int tau_mma_warps(int d, int bk) {
+  return (tau_stages(d, bk) % 2 == 0 && kMainSBufs % 2 == 0) ? 2 : 1;
+}
+__host__ __device__ constexpr int tau_threads(int d, int bk) {
+  return 32 * (kTauScoreWarps + 1 + tau_mma_warps(d, bk));
+}
+
 // Query tile of a persistent CTA's round r: one tile per CTA and round, the CTAs taking them in
 // reverse order every other round ("snake"), so that with the longest tiles first every CTA's
 // total work comes out even (round-robin leaves the first CTAs ~3% more at 16K).
@@ -540,10 +557,14 @@ __device__ __forceinline__ TileInfo tau_tile(const Problem& P, int L, int per_sl
 }
 
 template <int D, int BK>
-__global__ void __launch_bounds__(kTauThreads, 1)
+__global__ void __launch_bounds__(tau_threads(D, BK), 1)
     tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmw, Problem P) {
   constexpr int kStages = TauSmem<D, BK>::kStages;
+  constexpr int kMmaWarps = tau_mma_warps(D, BK);
+  constexpr int kThreads = tau_threads(D, BK);
+  static_assert(kStages % kMmaWarps == 0 && kMainSBufs % kMmaWarps == 0,
+                "each key stage and score buffer belongs to one MMA warp");
   extern __shared__ unsigned char smem_raw[];
   TauSmem<D, BK>& sm = *reinterpret_cast<TauSmem<D, BK>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -557,7 +578,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
+    mbar_init(&sm.q_empty, kMmaWarps);  // one commit per MMA warp
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -566,12 +587,12 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.s_empty[b], kTauScoreWarps);  // one arrival per score warp
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain, kMmaWarps);
     sm.abort = 0;
     cs.fallback = P.force_fallback;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (int w = tid; w < kMaxWords; w += kTauThreads) cs.words[w] = 0u;
+  for (int w = tid; w < kMaxWords; w += kThreads) cs.words[w] = 0u;
   if (warp == kTauMmaWarp) tmem_alloc(&sm.tmem_base, kTauTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -632,8 +653,9 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         mbar_wait(&sm.k_full[g % kStages], (g / kStages) & 1, abort, P.status);
       if (it > 0) mbar_wait(&sm.q_full, (it - 1) & 1, abort, P.status);
     }
-  } else if (warp == kTauMmaWarp) {
+  } else if (warp >= kTauMmaWarp) {
     if (lane == 0) {
+      const int mine = warp - kTauMmaWarp;  // this warp issues the groups gk % kMmaWarps == mine
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
       uint64_t qdesc[D / 16];
 #pragma unroll
@@ -649,6 +671,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
         ++it;
         const int nsteps = t.nkt + warm_steps(P, t);
         for (int i = 0; i < nsteps; ++i, ++gk) {
+          if (gk % kMmaWarps != mine) continue;
           const int s = gk % kStages, b = gk % kMainSBufs;
           if (!mbar_wait(&sm.k_full[s], (gk / kStages) & 1, abort, P.status) ||
               (gk >= kMainSBufs &&
@@ -667,7 +690,7 @@ __global__ void __launch_bounds__(kTauThreads, 1)
           mma_commit(&sm.k_empty[s]);
           mma_commit(&sm.s_full[b]);
         }
-        if (ok) mma_commit(&sm.q_empty);  // the tile's S products have read Q
+        if (ok) mma_commit(&sm.q_empty);  // this warp's S products of the tile have read Q
       }
       if (gk > 0) {  // all issued MMAs complete before tensor memory is released
         mma_commit(&sm.drain);
@@ -1575,8 +1598,8 @@ cudaError_t launch_tau_t(const Problem& P0, cudaStream_t s) {
   e = device_sms(&sms);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = static_cast<int64_t>(P.slots) * P.Hq * (P.cu ? 1 : P.B);
-  kern<<<static_cast<unsigned>(std::min<int64_t>(ntiles, sms)), kTauThreads, smem, s>>>(mq, mk, mw,
-                                                                                        P);
+  kern<<<static_cast<unsigned>(std::min<int64_t>(ntiles, sms)), tau_threads(D, BK), smem, s>>>(
+      mq, mk, mw, P);
   return cudaGetLastError();
 }
 
