@@ -16,7 +16,7 @@ FLAG_CUDA_CORES = 1
 FLAG_ALL_FALLBACK = 2
 FLAG_NO_BLOCK_MASK = 8  # ENTMAX_ATTN_FLAG_NO_BLOCK_MASK
 FLAG_TEST_STALL = 4  # test hook of the bounded device waits (ENTMAX_ATTN_FLAG_TEST_STALL)
-FLAG_PENDING_ONLY = 16  # output pass over the tiles the fused tau pass left (PENDING_ONLY)
+FLAG_SUPPORT = 16  # output from the supports the tau pass records (ENTMAX_ATTN_FLAG_SUPPORT)
 FLAG_OUT_FP32 = 32  # fp32 out for bf16 inputs (ENTMAX_ATTN_FLAG_OUT_FP32)
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES
 
@@ -38,9 +38,6 @@ SIGNATURES = {
     "entmax_attn_tau_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),
-    "entmax_attn_tau_out_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_size_t, _c_int,
-                                          _c_int, _c_int, _c_int, _c_int, _c_float, _c_int,
-                                          _c_int, _vp, _c_int, _c_uint, _vp]),
     "entmax_attn_out_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _vp, _c_int, _c_int,
                                       _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),

@@ -245,21 +245,6 @@ def tau_pass(q, k, tau, block_mask, workspace, alpha=1.5, n_iter=10, causal=True
     N.check(rc, "entmax_attn_tau_pass")
 
 
-def tau_out_pass(q, k, v, tau, block_mask, workspace, out, alpha=1.5, n_iter=10, causal=True,
-                 cu_seqlens=None, flags=0, stream=None):
-    """The tau pass that also writes out for every query tile whose rows' supports it held;
-    finish with out_pass(..., flags=FLAG_PENDING_ONLY) on the same workspace."""
-    _check_inputs(q, k, v, cu_seqlens)
-    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
-    rc = N.lib().entmax_attn_tau_out_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(tau),
-                                          _ptr(block_mask), _ptr(workspace),
-                                          workspace.numel() * workspace.element_size(), B, Hq,
-                                          Hkv, T, d, float(alpha), int(n_iter),
-                                          int(bool(causal)), _ptr(cu_seqlens), _DT[q.dtype],
-                                          int(flags), _stream(stream))
-    N.check(rc, "entmax_attn_tau_out_pass")
-
-
 def out_pass(q, k, v, tau, workspace, out, alpha=1.5, causal=True, cu_seqlens=None, flags=0,
              stream=None):
     _check_inputs(q, k, v, cu_seqlens)
@@ -315,16 +300,11 @@ def entmax_attn_two_pass(q, k, v, alpha=1.5, n_iter=10, causal=True, cu_seqlens=
 def entmax_attn_fused(q, k, v, alpha=1.5, n_iter=10, causal=True, cu_seqlens=None, flags=0,
                       workspace=None, stream=None):
     """The forward pass of entmax_attn_fwd through the two-pass entry points with a
-    torch-allocated workspace: tau_out_pass, then out_pass over the pending query tiles.
+    torch-allocated workspace and ENTMAX_ATTN_FLAG_SUPPORT: the tau pass records each row's
+    support, the output pass computes o from the supports (tile pass for the other query tiles).
     Returns (out, tau, block_mask, workspace)."""
-    out, tau, mask = alloc_outputs(q, k, cu_seqlens)
-    if flags & N.FLAG_OUT_FP32:
-        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-    ws = alloc_workspace(q, k, cu_seqlens) if workspace is None else workspace
-    tau_out_pass(q, k, v, tau, mask, ws, out, alpha, n_iter, causal, cu_seqlens, flags, stream)
-    out_pass(q, k, v, tau, ws, out, alpha, causal, cu_seqlens, flags | N.FLAG_PENDING_ONLY,
-             stream)
-    return out, tau, mask, ws
+    return entmax_attn_two_pass(q, k, v, alpha, n_iter, causal, cu_seqlens,
+                                flags | N.FLAG_SUPPORT, workspace, stream)
 
 
 def fallback_tiles(workspace, stream=None) -> int:

@@ -43,6 +43,7 @@ struct Layout {
   int64_t tiles;  // query tiles over all (batch, head)
   int warm_levels;       // warm-up key levels per key group
   int64_t norm_rows;     // key rows with a norm slot (Hq bounds Hkv)
+  int64_t q_rows;        // query rows (one support index each)
   int64_t warm_bytes;    // warm-up tiles of every key group at d = 128
 };
 
@@ -57,12 +58,16 @@ bool make_layout(int B, int Hq, int T, int has_cu, Layout* L) {
   L->tiles = (has_cu ? 1 : static_cast<int64_t>(B)) * Hq * slots;
   L->warm_levels = ea::warm_levels_for(T);
   L->norm_rows = (has_cu ? 1 : static_cast<int64_t>(B)) * Hq * T;
+  L->q_rows = L->norm_rows;
   L->warm_bytes = static_cast<int64_t>(B) * Hq * L->warm_levels * ea::kTile * 128 * 2;
   return L->tiles < (int64_t(1) << 31);
 }
 
 // Workspace: [queue_count | count[tiles] | queue[tiles] | pending[tiles] | list[tiles][nkt_max] |
-// key norms | warm-up tiles], each section 256-byte aligned.
+// key norms | warm-up tiles | support index[q rows] | support lists[tiles][kSupPerTile]], each
+// section 256-byte aligned.  The sections past the lists are optional: without the warm-up
+// sections the tau pass runs without warm-up keys, without the support sections every query
+// tile takes the tile output pass.
 struct WsView {
   int* queue_count;
   int* count;
@@ -71,7 +76,10 @@ struct WsView {
   int* list;
   float* norms;
   void* warm;
-  size_t min_bytes;  // without the warm-up sections
+  int* sup_idx;
+  int2* sup;
+  size_t min_bytes;   // without the warm-up and support sections
+  size_t warm_bytes;  // with the warm-up sections, without the support sections
   size_t bytes;
 };
 
@@ -94,6 +102,11 @@ WsView ws_view(void* base, const Layout& L) {
   off += align256(sizeof(float) * static_cast<size_t>(L.norm_rows));
   v.warm = p + off;
   off += align256(static_cast<size_t>(L.warm_bytes));
+  v.warm_bytes = off;
+  v.sup_idx = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * static_cast<size_t>(L.q_rows));
+  v.sup = reinterpret_cast<int2*>(p + off);
+  off += align256(sizeof(int2) * static_cast<size_t>(L.tiles) * ea::kSupPerTile);
   v.bytes = off;
   return v;
 }
@@ -180,6 +193,8 @@ void attach_workspace(ea::Problem* P, const WsView& v) {
   P->queue = v.queue;
   P->queue_count = v.queue_count;
   P->pending = v.pending;
+  P->sup_idx = v.sup_idx;
+  P->sup = v.sup;
   P->norms = v.norms;
   P->warm = v.warm;
 }
@@ -233,12 +248,11 @@ size_t entmax_attn_workspace_min_bytes(int B, int Hq, int T, int has_cu_seqlens)
 
 namespace {
 
-// The tau pass; with v and out (not null) it also writes o for every query tile whose rows'
-// supports its candidate buffers hold and marks the other tiles pending for the output pass.
-int tau_pass_impl(const void* q, const void* k, const void* v, void* out, float* tau,
-                  uint32_t* block_mask, void* workspace, size_t workspace_bytes, int B, int Hq,
-                  int Hkv, int T, int d, float alpha, int n_iter, int causal,
-                  const int32_t* cu_seqlens, int dtype, unsigned flags, cudaStream_t stream) {
+// The tau pass (ENTMAX_ATTN_FLAG_SUPPORT: also the support lists and pending flags).
+int tau_pass_impl(const void* q, const void* k, float* tau, uint32_t* block_mask,
+                  void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T, int d,
+                  float alpha, int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
+                  unsigned flags, cudaStream_t stream) {
   Layout L;
   ea::Problem P;
   int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
@@ -260,27 +274,24 @@ int tau_pass_impl(const void* q, const void* k, const void* v, void* out, float*
   P.force_fallback = (flags & ENTMAX_ATTN_FLAG_ALL_FALLBACK) ? 1 : 0;
   P.test_stall = (flags & ENTMAX_ATTN_FLAG_TEST_STALL) ? 1 : 0;
   P.no_mask = no_mask ? 1 : 0;
-  const bool fused = out != nullptr;
 
   cudaError_t e = cudaMemsetAsync(wv.queue_count, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e);
   if ((flags & ENTMAX_ATTN_FLAG_OUT_FP32) && !use_tensor_cores(dtype, flags))
     return ENTMAX_ATTN_EINVAL;  // fp32 outputs of bf16 inputs: the tensor-core path only
   P.out_f32 = (flags & ENTMAX_ATTN_FLAG_OUT_FP32) ? 1 : 0;
-  if (fused) {
-    if (use_tensor_cores(dtype, flags)) {
-      // the tensor-core tau kernel writes o and the pending flag of every query tile it solves
-      P.fused_out = 1;
-      P.v = v;
-      P.out = out;
+  if (flags & ENTMAX_ATTN_FLAG_SUPPORT) {
+    if (use_tensor_cores(dtype, flags) && workspace_bytes >= wv.bytes) {
+      // the tensor-core tau kernel records the supports and the pending flag of every tile
+      P.record_support = 1;
     } else {
-      // the CUDA-core tau kernel keeps no key ids: every query tile is left to the output pass
-      // (a nonzero flag; unused slots of a packed batch are skipped by the output pass anyway)
+      // no support lists (CUDA-core tau kernel, or no room for them): every query tile is left
+      // to the tile output pass (a nonzero flag; unused slots are skipped by it anyway)
       e = cudaMemsetAsync(wv.pending, 0xff, sizeof(int) * static_cast<size_t>(L.tiles), stream);
       if (e != cudaSuccess) return cuda_fail(e);
     }
   }
-  if (use_tensor_cores(dtype, flags) && workspace_bytes >= wv.bytes) {
+  if (use_tensor_cores(dtype, flags) && workspace_bytes >= wv.warm_bytes) {
     P.warm_levels = L.warm_levels;
     e = ea::launch_warm(P, stream);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -307,19 +318,8 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
                          void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
                          int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
                          int dtype, unsigned flags, cudaStream_t stream) {
-  return tau_pass_impl(q, k, nullptr, nullptr, tau, block_mask, workspace, workspace_bytes, B,
-                       Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype, flags, stream);
-}
-
-int entmax_attn_tau_out_pass(const void* q, const void* k, const void* v, void* out, float* tau,
-                             uint32_t* block_mask, void* workspace, size_t workspace_bytes, int B,
-                             int Hq, int Hkv, int T, int d, float alpha, int n_iter, int causal,
-                             const int32_t* cu_seqlens, int dtype, unsigned flags,
-                             cudaStream_t stream) {
-  if (!v || !out) return ENTMAX_ATTN_EINVAL;
-  if (!aligned16(v) || !aligned16(out)) return ENTMAX_ATTN_EALIGN;
-  return tau_pass_impl(q, k, v, out, tau, block_mask, workspace, workspace_bytes, B, Hq, Hkv, T,
-                       d, alpha, n_iter, causal, cu_seqlens, dtype, flags, stream);
+  return tau_pass_impl(q, k, tau, block_mask, workspace, workspace_bytes, B, Hq, Hkv, T, d, alpha,
+                       n_iter, causal, cu_seqlens, dtype, flags, stream);
 }
 
 int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,
@@ -346,12 +346,17 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
   P.tau = const_cast<float*>(tau);
   attach_workspace(&P, wv);
   P.no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) ? 1 : 0;
-  P.pending_only = (flags & ENTMAX_ATTN_FLAG_PENDING_ONLY) ? 1 : 0;
+  P.from_support = (flags & ENTMAX_ATTN_FLAG_SUPPORT) ? 1 : 0;
   if ((flags & ENTMAX_ATTN_FLAG_OUT_FP32) && !use_tensor_cores(dtype, flags))
     return ENTMAX_ATTN_EINVAL;  // fp32 outputs of bf16 inputs: the tensor-core path only
   P.out_f32 = (flags & ENTMAX_ATTN_FLAG_OUT_FP32) ? 1 : 0;
-  cudaError_t e = use_tensor_cores(dtype, flags) ? ea::launch_out_tc(P, stream)
-                                                 : ea::launch_out_simt(P, dtype, stream);
+  cudaError_t e = cudaSuccess;
+  // the recorded query tiles from their support lists (only the tensor-core tau pass records)
+  if (P.from_support && use_tensor_cores(dtype, flags) && workspace_bytes >= wv.bytes)
+    e = ea::launch_out_support(P, stream);
+  if (e == cudaSuccess)
+    e = use_tensor_cores(dtype, flags) ? ea::launch_out_tc(P, stream)
+                                       : ea::launch_out_simt(P, dtype, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return ENTMAX_ATTN_OK;
 }
@@ -429,11 +434,12 @@ int fwd_cached(const void* q, const void* k, const void* v, void* out, float* ta
     return entmax_attn_out_pass(q, k, v, tau, c.ptr, need, out, B, Hq, Hkv, T, d, alpha, causal,
                                 cu_seqlens, dtype, flags, stream);
   }
-  rc = entmax_attn_tau_out_pass(q, k, v, out, tau, block_mask, c.ptr, need, B, Hq, Hkv, T, d,
-                                alpha, n_iter, causal, cu_seqlens, dtype, flags, stream);
+  flags |= ENTMAX_ATTN_FLAG_SUPPORT;
+  rc = entmax_attn_tau_pass(q, k, tau, block_mask, c.ptr, need, B, Hq, Hkv, T, d, alpha, n_iter,
+                            causal, cu_seqlens, dtype, flags, stream);
   if (rc != ENTMAX_ATTN_OK) return rc;
   return entmax_attn_out_pass(q, k, v, tau, c.ptr, need, out, B, Hq, Hkv, T, d, alpha, causal,
-                              cu_seqlens, dtype, flags | ENTMAX_ATTN_FLAG_PENDING_ONLY, stream);
+                              cu_seqlens, dtype, flags, stream);
 }
 
 }  // namespace

@@ -68,15 +68,22 @@ struct Problem {
   int warm_levels;     // levels per group; 0 = no warm-up keys
   int kv_major;        // tau pass tile order: 1 = all query tiles of one key group before the
                        // next (keys larger than L2), 0 = slot-major (see tau_tile)
-  // Output from the candidates (tensor-core tau pass): with fused_out the tau pass also writes
-  // o for every query tile whose rows' supports its candidate buffers hold (all but the
-  // overflowed tiles) and sets pending[tile] to 0 there, 1 where the tile output pass must
-  // compute o.  With pending_only the output pass skips the tiles whose pending flag is 0.
+  // Output from the supports (ENTMAX_ATTN_FLAG_SUPPORT): with record_support the tensor-core
+  // tau pass records, for every query tile whose rows' supports its candidate buffers hold, each
+  // row's support -- the keys with p > 0 and their p -- and sets pending[tile] to 0 there, 1
+  // where the tile output pass must compute o (overflowed candidates, or more support entries
+  // than a tile's list holds).  With from_support the output pass computes o of the recorded
+  // tiles from their lists and runs the tile pass over the pending ones only.
   int* pending;        // [tiles] (workspace)
-  int fused_out;
-  int pending_only;
+  int2* sup;           // [tiles][kSupPerTile] (key of the sequence, bits of p) (workspace)
+  int* sup_idx;        // [q rows]: first entry | (entries << 16) of the row in its tile's list
+  int record_support;
+  int from_support;
   int out_f32;         // out is fp32 (bf16 inputs, tensor-core path): no rounding of o to bf16
 };
+
+// Support entries a query tile's list holds (16 per row on average; rows may use more).
+constexpr int kSupPerTile = 2048;
 
 struct TileInfo {
   int valid;        // 0 = unused slot of a packed batch
@@ -278,7 +285,9 @@ struct alignas(16) CandSmemT {
   float s[NC * kCols];
   uint16_t kt[NC * kCols];
   float rowmax[kTile];  // running max of the row over all segments (raw); see feed_warp
-  float tau_r[kTile];   // the row's tau once solved (read by the output gather)
+  float tau_r[kTile];   // the row's tau once solved (read by record_support)
+  int sup_n[kTile];     // support entries of each row, then their first position in the list
+  int sup_over;         // the tile's supports do not fit its list
   float m[kCols];       // segment max of raw scores
   float floor_[kCols];  // pruning floor (raw); -inf when the segment was never pruned
   int cnt[kCols];

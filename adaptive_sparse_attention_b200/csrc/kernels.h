@@ -19,6 +19,9 @@ cudaError_t launch_tau_tc(const Problem& P, cudaStream_t s);
 // Multi-sweep tau search on the tensor cores for the overflow queue (one CTA per SM at most).
 cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t s);
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s);
+// Output of the query tiles that are not pending, from the support lists the tau pass recorded
+// (bf16 values, d in {64, 128}).
+cudaError_t launch_out_support(const Problem& P, cudaStream_t s);
 // Warm-up keys of the tensor-core tau pass (P.norms, P.warm); nothing when P.warm_levels == 0.
 cudaError_t launch_warm(const Problem& P, cudaStream_t s);
 

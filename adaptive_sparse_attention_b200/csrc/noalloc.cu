@@ -59,11 +59,11 @@ extern "C" int entmax_attn_fwd_noalloc(const void* q, const void* k, const void*
     }
     scratch = g_scratch_ptr[dev];
   }
-  int rc = entmax_attn_tau_out_pass(q, k, v, out, tau, block_mask, scratch,
-                                    ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES, B, Hq, Hkv, T, d, alpha,
-                                    n_iter, causal, cu_seqlens, dtype, 0u, stream);
+  int rc = entmax_attn_tau_pass(q, k, tau, block_mask, scratch, ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES,
+                                B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
+                                ENTMAX_ATTN_FLAG_SUPPORT, stream);
   if (rc != ENTMAX_ATTN_OK) return rc;
   return entmax_attn_out_pass(q, k, v, tau, scratch, ENTMAX_ATTN_NOALLOC_SCRATCH_BYTES, out, B,
                               Hq, Hkv, T, d, alpha, causal, cu_seqlens, dtype,
-                              ENTMAX_ATTN_FLAG_PENDING_ONLY, stream);
+                              ENTMAX_ATTN_FLAG_SUPPORT, stream);
 }

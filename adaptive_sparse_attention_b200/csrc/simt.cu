@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads) out_simt_kernel(Problem P) {
   const int slot = gridDim.x - 1 - blockIdx.x;
   const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
-  if (P.pending_only && P.pending[t.tile_id] == 0) return;  // o already written
+  if (P.from_support && P.pending[t.tile_id] == 0) return;  // o from the tile's support list
   const T* kp = as<T>(P.k);
   const T* vp = as<T>(P.v);
   load_q_tile<T, D>(P, t, sm.qs, tid);

@@ -12,8 +12,9 @@
 //               columns 32 g .. 32 g + 31 with g = w / 4, i.e. one 32-key segment of every key
 //               tile, into the segment's candidate buffer (common.cuh); the four segments of a
 //               row share its running max.
-//   then the score warps solve tau per row (4-lane groups), compute the output of the rows
-//   from their candidates (gather_rows), and write the block mask and the compact tile list.
+//   then the score warps solve tau per row (4-lane groups), record each row's support (keys
+//   with p > 0 and their p) from its candidates (record_support), and write the block mask and
+//   the compact tile list.
 //
 // out_tc_kernel (one CTA of 384 threads per query tile, over the listed key tiles only):
 //   warp 0      TMA producer of the query tile and the key tiles (3-stage ring; a key tile is
@@ -427,74 +428,6 @@ __device__ __forceinline__ int warm_steps(const Problem& P, const TileInfo& t) {
   return warm_level(P, t) >= 0 ? 1 : 0;
 }
 
-// Output from the candidates.  Every key with p_ij > 0 has z_ij > tau_i >= m_i - 1, so once a
-// row's candidate buffers hold every key above their floor and tau lies above the floor (what
-// solve_rows checks; a tile that fails is queued for the overflow path), the row's support is
-// exactly its buffer entries with z > tau, and o_i = sum over them of p_ij v_j.  The support of a
-// row is a handful of keys where the tile output pass would multiply whole 128-key tiles of
-// mostly zero p; so the tau kernel computes o itself, right after the solve: p in fp32 from the
-// stored raw score (the value the output pass would recompute) and tau, v_j gathered from global
-// memory (L2), fp32 accumulation, one rounding to bf16 at the store.  The 4 lanes of a row
-// (consecutive threads) split the d columns, so a row's store is one contiguous d-element run.
-template <int D, int BK, class CS>
-__device__ __forceinline__ void gather_rows(const Problem& P, const TileInfo& t, const CS& cs,
-                                            int tid, int nthreads) {
-  constexpr int kDims = D / 4;     // columns per lane
-  constexpr int kVec = kDims / 8;  // 16-byte vectors (8 bf16) per lane
-  const int lane4 = tid & 3;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(P.v) +
-                            (t.khead + t.seq_start) * D + lane4 * kDims;
-  const int64_t ob = (t.qhead + t.seq_start + t.row0) * D + lane4 * kDims;  // element offset
-  for (int r = tid >> 2; r < t.nrows; r += nthreads >> 2) {
-    const float tau = cs.tau_r[r];
-    float acc[kDims];
-#pragma unroll
-    for (int i = 0; i < kDims; ++i) acc[i] = 0.f;
-#pragma unroll 1
-    for (int g = 0; g < kSeg; ++g) {
-      const int col = g * kTile + r;
-      const int n = min(cs.cnt[col], CS::kSlots);
-#pragma unroll 1
-      for (int e = 0; e < n; ++e) {
-        const float x = P.c * cs.s[e * kCols + col] - tau;
-        if (!(x > 0.f)) continue;
-        const float p = entmax_p<BK>(x, P.beta);
-        const int id = cs.kt[e * kCols + col];
-        // key id -> key of the sequence; kept inside the sequence whatever the buffer holds
-        const int j = min((id >> 5) * kTile + g * 32 + (id & 31), t.seq_len - 1);
-        const uint4* src = reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(j) * D);
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-          const uint4 w = __ldg(src + u);
-          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[h]));
-            acc[8 * u + 2 * h] = fmaf(p, f.x, acc[8 * u + 2 * h]);
-            acc[8 * u + 2 * h + 1] = fmaf(p, f.y, acc[8 * u + 2 * h + 1]);
-          }
-        }
-      }
-    }
-    const int64_t oe = ob + static_cast<int64_t>(r) * D;
-    if (P.out_f32) {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(P.out) + oe);
-#pragma unroll
-      for (int u = 0; u < 2 * kVec; ++u)
-        dst[u] = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
-                            __float_as_uint(acc[4 * u + 2]), __float_as_uint(acc[4 * u + 3]));
-    } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + oe);
-#pragma unroll
-      for (int u = 0; u < kVec; ++u)
-        dst[u] = make_uint4(pack_bf16x2(acc[8 * u], acc[8 * u + 1]),
-                            pack_bf16x2(acc[8 * u + 2], acc[8 * u + 3]),
-                            pack_bf16x2(acc[8 * u + 4], acc[8 * u + 5]),
-                            pack_bf16x2(acc[8 * u + 6], acc[8 * u + 7]));
-    }
-  }
-}
-
 template <int D, int BK>
 struct TauSmem {
   static constexpr int kStages = tau_stages(D, BK);
@@ -536,6 +469,83 @@ __device__ __forceinline__ bool score_warps_any(bool flag) {
       : "r"(static_cast<int>(flag)), "n"(32 * kTauScoreWarps)
       : "memory");
   return r != 0;
+}
+
+// Supports from the candidates.  Every key with p_ij > 0 has z_ij > tau_i >= m_i - 1, so once a
+// row's candidate buffers hold every key above their floor and tau lies above the floor (what
+// solve_rows checks; a tile that fails is queued for the overflow path), the row's support is
+// exactly its buffer entries with z > tau.  The support of a row is a handful of keys where the
+// tile output pass would multiply whole 128-key tiles of mostly zero p; so the tau kernel records
+// each row's support -- key j of the sequence and p_ij in fp32 from the stored raw score and tau
+// -- in its query tile's list (rows one after another, kSupPerTile entries per tile), and the
+// output pass computes o_i = sum p_ij v_j from the lists (out_support_kernel).  A tile whose rows
+// need more entries than its list holds is left pending for the tile output pass.  Call from all
+// score threads (one row per 4-lane group) after the barrier that follows solve_rows; it holds
+// two barriers of the score warps.
+template <int BK, class CS>
+__device__ __forceinline__ void record_support(const Problem& P, const TileInfo& t, CS& cs,
+                                               int tid, int lane) {
+  const unsigned full = 0xffffffffu;
+  const int lane4 = tid & 3;
+  const int r = tid >> 2;  // 512 score threads: one row per 4-lane group
+  const bool valid = r < t.nrows;
+  const float tau = valid ? cs.tau_r[r] : 0.f;
+  // this lane's share of the row's entries: e = lane4, lane4 + 4, ... of every segment
+  int n = 0;
+  if (valid) {
+#pragma unroll 1
+    for (int g = 0; g < kSeg; ++g) {
+      const int col = g * kTile + r;
+      const int cnt = min(cs.cnt[col], CS::kSlots);
+      for (int e = lane4; e < cnt; e += 4) n += (P.c * cs.s[e * kCols + col] - tau > 0.f) ? 1 : 0;
+    }
+  }
+  // the row's total and this lane's first entry among the row's four lanes
+  int incl = n;
+  int y = __shfl_up_sync(full, incl, 1);
+  if (lane4 >= 1) incl += y;
+  y = __shfl_up_sync(full, incl, 2);
+  if (lane4 >= 2) incl += y;
+  const int total = __shfl_sync(full, incl, (lane & ~3) | 3);
+  if (lane4 == 3) cs.sup_n[r] = total;
+  score_warps_sync();
+  if (tid < 32) {  // exclusive prefix over the 128 rows: four rows per lane
+    int a[4], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[i] = sum;
+      sum += cs.sup_n[4 * tid + i];
+    }
+    int x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int z = __shfl_up_sync(full, x, o);
+      if (tid >= o) x += z;
+    }
+    const int base = x - sum;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cs.sup_n[4 * tid + i] = base + a[i];
+    if (tid == 31) cs.sup_over = x > kSupPerTile ? 1 : 0;
+  }
+  score_warps_sync();
+  if (cs.sup_over || !valid) return;
+  int2* list = P.sup + t.tile_id * kSupPerTile;
+  const int first = cs.sup_n[r];
+  int at = first + incl - n;
+#pragma unroll 1
+  for (int g = 0; g < kSeg; ++g) {
+    const int col = g * kTile + r;
+    const int cnt = min(cs.cnt[col], CS::kSlots);
+    for (int e = lane4; e < cnt; e += 4) {
+      const float x = P.c * cs.s[e * kCols + col] - tau;
+      if (x > 0.f) {
+        const int id = cs.kt[e * kCols + col];
+        const int j = (id >> 5) * kTile + g * 32 + (id & 31);  // key of the sequence
+        list[at++] = make_int2(j, __float_as_int(entmax_p<BK>(x, P.beta)));
+      }
+    }
+  }
+  if (lane4 == 0) P.sup_idx[t.qhead + t.seq_start + t.row0 + r] = first | (total << 16);
 }
 
 // Query tile L of the tau pass's tile order.  Slot-major: the longest tiles (highest slot) of
@@ -748,9 +758,9 @@ __global__ void __launch_bounds__(tau_threads(D, BK), 1)
       if (score_warps_any(*abort != 0)) break;  // status already records the timeout
       solve_rows<BK>(P, t, cs, tid, kScoreThreads);
       score_warps_sync();
-      if (P.fused_out) {  // o from the candidates, unless the tile goes to the overflow path
-        if (!cs.fallback) gather_rows<D, BK>(P, t, cs, tid, kScoreThreads);
-        if (tid == 0) P.pending[t.tile_id] = cs.fallback ? 1 : 0;
+      if (P.record_support) {  // unless the tile goes to the overflow path (uniform test)
+        if (!cs.fallback) record_support<BK>(P, t, cs, tid, lane);
+        if (tid == 0) P.pending[t.tile_id] = (cs.fallback || cs.sup_over) ? 1 : 0;
       }
       if (warp == 0) emit_tile_prefix(P, t, cs, lane);
       score_warps_sync();
@@ -1053,7 +1063,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   const int slot = gridDim.x - 1 - blockIdx.x;
   const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
-  if (P.pending_only && P.pending[t.tile_id] == 0) return;  // o already written by the tau pass
+  if (P.from_support && P.pending[t.tile_id] == 0) return;  // o from the tile's support list
   // The list comes from the tau pass; clamping keeps every read inside this tile's list and key
   // range even if the workspace was never filled.
   const int cnt = list_count(P, t);
@@ -1284,8 +1294,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const TileInfo ta = map_tile(P, slot, 2 * blockIdx.y, blockIdx.z);
   if (!ta.valid) return;
   const TileInfo tb = map_tile(P, slot, 2 * blockIdx.y + 1, blockIdx.z);
-  // o of both heads already written by the tau pass (one pending head recomputes both)
-  if (P.pending_only && P.pending[ta.tile_id] == 0 && P.pending[tb.tile_id] == 0) return;
+  // o of both heads from their support lists (one pending head recomputes both)
+  if (P.from_support && P.pending[ta.tile_id] == 0 && P.pending[tb.tile_id] == 0) return;
   // Lists from the tau pass, clamped so that no workspace content sends a read outside them.
   const int cnt_a = list_count(P, ta);
   const int cnt_b = list_count(P, tb);
@@ -1529,6 +1539,78 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------- output from the supports --
+// out_support_kernel: o_i = sum_j p_ij v_j over the support list the tau pass recorded for row i
+// (record_support), for every query tile that is not pending.  One CTA of 128 threads per query
+// tile; 8 lanes per row, each owning d / 8 consecutive columns (a value row is one contiguous
+// 2 d-byte read by the 8 lanes), 16 rows at a time, two entries of a row loaded before either is
+// accumulated.  Keys, offsets and counts are clamped to the tile's list and sequence, so an
+// unfilled workspace cannot send a read outside them.
+constexpr int kSupThreads = 128;
+
+template <int D>
+__global__ void __launch_bounds__(kSupThreads)
+    out_support_kernel(Problem P) {
+  const int slot = gridDim.x - 1 - blockIdx.x;
+  const TileInfo t = map_tile(P, slot, blockIdx.y, blockIdx.z);
+  if (!t.valid || P.pending[t.tile_id] != 0) return;
+  constexpr int kCols8 = D / 8;      // columns per lane
+  constexpr int kVec = kCols8 / 8;   // 16-byte vectors per lane and value row
+  const int l8 = threadIdx.x & 7;
+  const int2* list = P.sup + t.tile_id * kSupPerTile;
+  const __nv_bfloat16* vb =
+      static_cast<const __nv_bfloat16*>(P.v) + (t.khead + t.seq_start) * D + l8 * kCols8;
+  for (int r = threadIdx.x >> 3; r < t.nrows; r += kSupThreads / 8) {
+    const int64_t row = t.qhead + t.seq_start + t.row0 + r;
+    const int idx = P.sup_idx[row];
+    const int first = min(idx & 0xffff, kSupPerTile);
+    const int n = min(idx >> 16, kSupPerTile - first);
+    float acc[kCols8];
+#pragma unroll
+    for (int i = 0; i < kCols8; ++i) acc[i] = 0.f;
+    for (int e = 0; e < n; e += 2) {
+      const int2 a = list[first + e];
+      const int2 b = (e + 1 < n) ? list[first + e + 1] : make_int2(a.x, 0);
+      const int ja = min(max(a.x, 0), t.seq_len - 1), jb = min(max(b.x, 0), t.seq_len - 1);
+      const float pa = __int_as_float(a.y), pb = __int_as_float(b.y);
+      uint4 wa[kVec], wb[kVec];
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        wa[u] = __ldg(reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(ja) * D) + u);
+        wb[u] = __ldg(reinterpret_cast<const uint4*>(vb + static_cast<int64_t>(jb) * D) + u);
+      }
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const uint32_t xa[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
+        const uint32_t xb[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xa[h]));
+          const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xb[h]));
+          acc[8 * u + 2 * h] = fmaf(pb, fb.x, fmaf(pa, fa.x, acc[8 * u + 2 * h]));
+          acc[8 * u + 2 * h + 1] = fmaf(pb, fb.y, fmaf(pa, fa.y, acc[8 * u + 2 * h + 1]));
+        }
+      }
+    }
+    const int64_t oe = row * D + l8 * kCols8;  // element offset of this lane's columns
+    if (P.out_f32) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(P.out) + oe);
+#pragma unroll
+      for (int u = 0; u < 2 * kVec; ++u)
+        dst[u] = make_uint4(__float_as_uint(acc[4 * u]), __float_as_uint(acc[4 * u + 1]),
+                            __float_as_uint(acc[4 * u + 2]), __float_as_uint(acc[4 * u + 3]));
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + oe);
+#pragma unroll
+      for (int u = 0; u < kVec; ++u)
+        dst[u] = make_uint4(pack_bf16x2(acc[8 * u], acc[8 * u + 1]),
+                            pack_bf16x2(acc[8 * u + 2], acc[8 * u + 3]),
+                            pack_bf16x2(acc[8 * u + 4], acc[8 * u + 5]),
+                            pack_bf16x2(acc[8 * u + 6], acc[8 * u + 7]));
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------ host side --
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
@@ -1647,6 +1729,14 @@ cudaError_t launch_out_pair_t(const Problem& P, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_support_t(const Problem& P, cudaStream_t s) {
+  if (P.d == 64)
+    out_support_kernel<64><<<tile_grid(P), kSupThreads, 0, s>>>(P);
+  else
+    out_support_kernel<128><<<tile_grid(P), kSupThreads, 0, s>>>(P);
+  return cudaGetLastError();
+}
+
 #define EA_TC_DISPATCH(FN)                                          \
   do {                                                              \
     const int bk = beta_kind(P.beta);                               \
@@ -1679,6 +1769,8 @@ cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t 
   if (bk == kBetaNear3) return launch_sweep_t<128, kBetaNear3>(P, num_ctas, s);
   return launch_sweep_t<128, kBetaGeneral>(P, num_ctas, s);
 }
+cudaError_t launch_out_support(const Problem& P, cudaStream_t s) { return launch_support_t(P, s); }
+
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) {
   // heads 2 j and 2 j + 1 share their key/value head when the group size is even
   if (P.G % 2 == 0) EA_TC_DISPATCH(launch_out_pair_t);

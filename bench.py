@@ -322,11 +322,12 @@ def launches_per_step(w) -> int:
 
 
 # The forward pass, three ways through the C ABI's two-pass entry points:
-#   fused    entmax_attn_tau_out_pass (tau, mask, lists, and o of every query tile whose rows'
-#            supports the tau pass held) + entmax_attn_out_pass over the pending tiles only:
-#            the path entmax_attn_fwd takes, and the step this benchmark times;
-#   tile     entmax_attn_tau_pass + entmax_attn_out_pass over every query tile's active key
-#            tiles (o recomputed tile by tile on the tensor cores), reported beside it;
+#   fused    with ENTMAX_ATTN_FLAG_SUPPORT: the tau pass (tau, mask, lists, and the support of
+#            every row whose candidates it held), then the output pass (o from the supports, the
+#            tile pass over the other query tiles): the path entmax_attn_fwd takes, and the step
+#            this benchmark times;
+#   tile     without the flag: the output pass over every query tile's active key tiles (o
+#            recomputed tile by tile on the tensor cores), reported beside it;
 #   nomask   the variant without block mask (--no-block-mask).
 MODES = ("fused", "tile", "nomask")
 
@@ -353,14 +354,10 @@ class Problem:
         a = (self.q, self.k)
         if ev:
             ev[0].record(s)
-        if mode == "fused":
-            ea.tau_out_pass(*a, self.v, self.tau, self.mask, self.ws, self.out, self.alpha,
-                            w.n_iter, w.causal, self.cu, stream=s)
-            flags = _native.FLAG_PENDING_ONLY
-        else:
-            flags = _native.FLAG_NO_BLOCK_MASK if mode == "nomask" else 0
-            ea.tau_pass(*a, self.tau, self.mask, self.ws, self.alpha, w.n_iter, w.causal,
-                        self.cu, flags=flags, stream=s)
+        flags = {"fused": _native.FLAG_SUPPORT, "tile": 0,
+                 "nomask": _native.FLAG_NO_BLOCK_MASK}[mode]
+        ea.tau_pass(*a, self.tau, self.mask, self.ws, self.alpha, w.n_iter, w.causal, self.cu,
+                    flags=flags, stream=s)
         if ev:
             ev[1].record(s)
         ea.out_pass(*a, self.v, self.tau, self.ws, self.out, self.alpha, w.causal, self.cu,
@@ -528,7 +525,7 @@ def run_native(args, rank, world, local):
         peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock"
     out_flops = 4 * w.d * (dense_pairs if nm else act_pairs)
     achieved = (tau_flops / (mean_tau * 1e-3) if dom_tau else out_flops / (mean_out * 1e-3)) / 1e12
-    kname = ("tau_out_pass" if mode == "fused" else "tau_pass") if dom_tau else "out_pass"
+    kname = "tau_pass" if dom_tau else "out_pass"
     traffic = ncu_traffic(w.name, kname)
     roofline = {"kernel": kname, "bound": bound,
                 "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
@@ -555,8 +552,8 @@ def run_native(args, rank, world, local):
         "config": dict(workload_config(w, world),
                        variant="no_block_mask" if nm else "block_mask",
                        path=("tau pass + output pass over every causal tile" if nm else
-                             "tau pass with the output from its candidates + tile output pass "
-                             "over the overflowed query tiles"),
+                             "tau pass recording each row's support + output from the supports "
+                             "(tile output pass for query tiles without one)"),
                        l2=f"inputs {pb.in_bytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB "
                           f"L2; no flush" if pb.in_bytes > L2_BYTES
                        else "inputs fit in L2; no flush"),

@@ -81,15 +81,21 @@ extern "C" {
                                              mask and no tile lists (block_mask may be NULL), and
                                              the output pass visits every causally valid key tile.
                                              Give it to both passes. */
-#define ENTMAX_ATTN_FLAG_PENDING_ONLY 16u /* output pass only: visit only the query tiles that
-                                             the last entmax_attn_tau_out_pass on this
-                                             workspace left pending (its overflowed tiles) */
+#define ENTMAX_ATTN_FLAG_SUPPORT 16u      /* output from the supports; give it to both passes.
+                                             The tensor-core tau pass records, for every query
+                                             tile whose rows' supports its candidate buffers
+                                             held, each row's support (the keys with p > 0 and
+                                             their p) in the workspace; the output pass computes
+                                             o of those tiles from the lists and runs the tile
+                                             pass over the others only (overflowed candidates,
+                                             supports beyond a tile's list, the CUDA-core path,
+                                             a workspace below entmax_attn_workspace_bytes).
+                                             The path entmax_attn_fwd takes. */
 #define ENTMAX_ATTN_FLAG_OUT_FP32 32u     /* bf16 inputs on the tensor-core path: out is float
                                              (fp32 accumulations stored without rounding to
-                                             bf16), same layout.  Give it to every pass that
-                                             writes out (entmax_attn_tau_out_pass and
-                                             entmax_attn_out_pass); ENTMAX_ATTN_EINVAL with fp32
-                                             inputs or ENTMAX_ATTN_FLAG_CUDA_CORES. */
+                                             bf16), same layout.  Give it to both passes;
+                                             ENTMAX_ATTN_EINVAL with fp32 inputs or
+                                             ENTMAX_ATTN_FLAG_CUDA_CORES. */
 #define ENTMAX_ATTN_FLAG_TEST_STALL 4u    /* test hook of the bounded waits: the tensor-core tau
                                              pass never requests its query tiles, so each of its
                                              CTAs gives up after one wait limit (about 2 s) and
@@ -97,12 +103,12 @@ extern "C" {
                                              status word; its outputs are void.  Use it on a
                                              problem of a few query tiles only. */
 
-/* Full forward pass: entmax_attn_tau_out_pass (tau search, block mask, and the output of every
- * query tile whose rows' supports the tau pass held), then entmax_attn_out_pass over the active
- * tiles of the remaining (overflowed) query tiles.  Writes out, tau and every word of
- * block_mask.  Scratch memory (compact tile lists, overflow queue, pending flags) is allocated
- * by the library on first use per (device, stream) with cudaMallocAsync on `stream`, grown when a
- * larger problem arrives, and kept until entmax_attn_release_workspaces().
+/* Full forward pass: the tau pass (tau search, block mask, and the support of every row whose
+ * candidates it held), then the output pass (o from the supports, and over the active key tiles
+ * of the remaining query tiles): the two-pass form with ENTMAX_ATTN_FLAG_SUPPORT.  Writes out,
+ * tau and every word of block_mask.  Scratch memory (compact tile lists, overflow queue, support
+ * lists) is allocated by the library on first use per (device, stream) with cudaMallocAsync on
+ * `stream`, grown when a larger problem arrives, and kept until entmax_attn_release_workspaces().
  * Returns ENTMAX_ATTN_OK or an error code. */
 int entmax_attn_fwd(const void* q, const void* k, const void* v, void* out, float* tau,
                     uint32_t* block_mask, int B, int Hq, int Hkv, int T, int d, float alpha,
@@ -140,32 +146,20 @@ size_t entmax_attn_workspace_bytes(int B, int Hq, int T, int has_cu_seqlens);
 size_t entmax_attn_workspace_min_bytes(int B, int Hq, int T, int has_cu_seqlens);
 
 /* Tau pass: writes tau, every word of block_mask, and the compact list of active key tiles of
- * every query tile into the workspace.  ENTMAX_ATTN_ENOMEM if workspace_bytes is below
- * entmax_attn_workspace_min_bytes(). */
+ * every query tile into the workspace (with ENTMAX_ATTN_FLAG_SUPPORT also the supports).
+ * ENTMAX_ATTN_ENOMEM if workspace_bytes is below entmax_attn_workspace_min_bytes(). */
 int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
                          void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T,
                          int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
                          int dtype, unsigned flags, cudaStream_t stream);
 
-/* Tau pass with the output: everything entmax_attn_tau_pass writes, and out for every query
- * tile whose rows' supports the pass held in its candidate buffers (AdaSplash page, "AdaSplash
- * with Block Masking": p_ij > 0 needs z_ij > tau_i >= max_j z_ij - 1, and these are the keys the
- * pass keeps to find tau): o_i = sum_j p_ij v_j over those keys, p in fp32 from the pass's own
- * scores and tau, fp32 accumulation, one rounding to the output dtype.  The other query tiles
- * (those whose candidates overflowed into the multi-sweep search; every tile on the CUDA-core
- * path) are marked pending in the workspace: complete out with entmax_attn_out_pass and
- * ENTMAX_ATTN_FLAG_PENDING_ONLY on the same workspace, in stream order.  v and out as in
- * entmax_attn_fwd (device, 16-byte aligned); the other arguments, flags and returns as
- * entmax_attn_tau_pass (ENTMAX_ATTN_EINVAL for a null v or out). */
-int entmax_attn_tau_out_pass(const void* q, const void* k, const void* v, void* out, float* tau,
-                             uint32_t* block_mask, void* workspace, size_t workspace_bytes, int B,
-                             int Hq, int Hkv, int T, int d, float alpha, int n_iter, int causal,
-                             const int32_t* cu_seqlens, int dtype, unsigned flags,
-                             cudaStream_t stream);
-
 /* Output pass: o_i = sum over the listed key tiles of p_ij v_j, with p recomputed from tau
  * (scores on the tensor cores, P rounded to bf16 for the P V product, fp32 accumulation).  With
- * ENTMAX_ATTN_FLAG_PENDING_ONLY only the query tiles entmax_attn_tau_out_pass left pending. */
+ * ENTMAX_ATTN_FLAG_SUPPORT (given to the tau pass too): o_i = sum of p_ij v_j over the support
+ * the tau pass recorded for row i (p in fp32 from the tau pass's own scores, fp32 accumulation,
+ * one rounding to the output dtype), and the tile pass only for the query tiles without a
+ * recorded support (AdaSplash page, "AdaSplash with Block Masking": p_ij > 0 needs
+ * z_ij > tau_i >= max_j z_ij - 1, the keys the tau pass keeps to find tau). */
 int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,
                          const void* workspace, size_t workspace_bytes, void* out, int B, int Hq,
                          int Hkv, int T, int d, float alpha, int causal,

@@ -57,11 +57,11 @@ class GpuResult:
     fallback_tiles: int
 
 
-# The forward pass's paths through the C ABI:
-#   "fused": entmax_attn_tau_out_pass (o of every query tile whose rows' supports the tau pass
-#            held) + entmax_attn_out_pass over the pending tiles -- the path entmax_attn_fwd
-#            takes and bench.py times;
-#   "tile":  entmax_attn_tau_pass + entmax_attn_out_pass over every query tile's active tiles.
+# The forward pass's paths through the C ABI's two passes:
+#   "fused": with ENTMAX_ATTN_FLAG_SUPPORT: the tau pass records each row's support, the output
+#            pass computes o from the supports (tile pass for the query tiles without one) --
+#            the path entmax_attn_fwd takes and bench.py times;
+#   "tile":  without it: the output pass over every query tile's active key tiles.
 PATHS = ("fused", "tile")
 
 

@@ -215,19 +215,23 @@ def test_small_workspace_is_rejected(native):
 @pytest.mark.parametrize("B,Hq,T,packed", [(1, 2, 256, 0), (2, 32, 16384, 0), (4, 32, 32192, 1),
                                            (1, 32, 131072, 0), (1, 8, 1023, 0)])
 def test_workspace_sizes_nest(native, B, Hq, T, packed):
-    """The full workspace adds the warm-up sections after the smallest one: squared norms of
+    """The full workspace adds to the smallest one the warm-up sections -- squared norms of
     (B or 1) * Hq * T key rows and B * Hq * levels warm-up tiles of 128 x 128 bf16, levels being
-    the ranges 1024 * 2^j that fit in T keys."""
+    the ranges 1024 * 2^j that fit in T keys -- and the support sections: one int32 index per
+    query row and 2048 eight-byte entries per query tile (slot)."""
     from adaptive_sparse_attention_b200 import api
     lo, hi = api.workspace_min_bytes(B, Hq, T, bool(packed)), api.workspace_bytes(B, Hq, T, bool(packed))
     levels = 0
     while (1024 << levels) <= T:
         levels += 1
     rows = (1 if packed else B) * Hq * T
+    slots = (T // 128 + B) if packed else -(-T // 128)
+    tiles = (1 if packed else B) * Hq * slots
     def up(x):
         return (x + 255) // 256 * 256
     assert 0 < lo <= hi
-    assert hi - lo == up(4 * rows) + up(B * Hq * levels * 128 * 128 * 2)
+    assert hi - lo == (up(4 * rows) + up(B * Hq * levels * 128 * 128 * 2) + up(4 * rows)
+                       + up(8 * 2048 * tiles))
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -207,32 +207,32 @@ def test_far_apart_scores_give_one_hot_rows(oracle, dtype, path):
 
 
 @pytest.mark.parametrize("name,kw", [SMALL[5], SMALL[8]], ids=[SMALL[5][0], SMALL[8][0]])
-def test_tau_out_pass_writes_exactly_the_settled_tiles(oracle, name, kw):
-    """entmax_attn_tau_out_pass alone (no output pass after it): every query tile it did not
-    leave pending holds its final output, and the tiles it left pending are untouched (the
-    output was NaN-filled before).  Forcing every tile through the overflow path must leave
-    every row untouched."""
+def test_support_path_without_room_for_the_lists(oracle, name, kw):
+    """ENTMAX_ATTN_FLAG_SUPPORT on a workspace with the warm-up sections but no room for the
+    support lists: every query tile takes the tile output pass, with the same results."""
     w, inputs = random_case(dtype="bf16", name=name, seed=19, **kw)
     q, k, v, cu = (t.cuda() if t is not None else None for t in inputs)
-    alpha = oracle.alpha_as_float32(w.alpha)
-    for flags, expect_all_pending in ((0, False), (_native.FLAG_ALL_FALLBACK, True)):
-        out, tau, mask = ea.alloc_outputs(q, k, cu)
-        out.fill_(float("nan"))
-        ws = ea.alloc_workspace(q, k, cu)
-        ea.tau_out_pass(q, k, v, tau, mask, ws, out, alpha, w.n_iter, w.causal, cu, flags=flags)
-        torch.cuda.synchronize()
-        assert ea.status() == 0
-        nan_rows = torch.isnan(out.float()).any(dim=-1).cpu().numpy().ravel()
-        valid_rows = np.concatenate([parity.tile_rows(w, inputs[3], *t)
-                                     for t in parity.all_tiles(w, inputs[3])])
-        if expect_all_pending:
-            assert nan_rows[valid_rows].all()
-            continue
-        ea.out_pass(q, k, v, tau, ws, out, alpha, w.causal, cu, flags=_native.FLAG_PENDING_ONLY)
-        torch.cuda.synchronize()
-        g = parity.GpuResult(out.float().cpu().numpy().reshape(-1, w.d), tau.cpu().numpy().ravel(),
-                             ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, inputs[3]),
-                             ea.fallback_tiles(ws))
-        parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"fused/{name}")
-        # the rows the tau pass wrote are the rows of the tiles it did not queue
-        assert nan_rows[valid_rows].sum() <= g.fallback_tiles * 128
+    B, Hq, Hkv, T, d = ea.api.problem_dims(q, k, cu)
+    full = ea.workspace_bytes(B, Hq, T, cu is not None)
+    ws = torch.empty(full, dtype=torch.uint8, device="cuda")
+    room = ws[:full - 256]  # one byte short of the support lists' end: no support lists
+    out, tau, mask, _ = ea.entmax_attn_fused(q, k, v, oracle.alpha_as_float32(w.alpha),
+                                             w.n_iter, w.causal, cu, workspace=room)
+    torch.cuda.synchronize()
+    assert ea.status() == 0
+    g = parity.GpuResult(out.float().cpu().numpy().reshape(-1, w.d), tau.cpu().numpy().ravel(),
+                         ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, inputs[3]), -1)
+    parity.compare(w, inputs, g, parity.all_tiles(w, inputs[3]), label=f"support_noroom/{name}")
+
+
+@pytest.mark.parametrize("path", parity.PATHS)
+def test_large_supports(oracle, path):
+    """Near-flat scores at alpha = 1.333 (q scaled by 1/4) give supports of tens of keys per
+    row: query tiles whose rows need more entries than a tile's support list holds, or more
+    candidates than the buffers hold, take the tile output pass; every row must still match."""
+    w, (q, k, v, cu) = random_case(B=1, Hq=4, Hkv=2, T=1500, d=128, dtype="bf16", alpha=1.333,
+                                   name="large_supports", seed=37)
+    q = (q.float() / 4).to(q.dtype)
+    inputs = (q, k, v, cu)
+    g = parity.run_gpu(w, inputs, path=path)
+    parity.compare(w, inputs, g, parity.all_tiles(w, cu), label=f"large_supports/{path}")
