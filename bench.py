@@ -83,9 +83,7 @@ def count_pairs(w, bits, cu):
 # hash of the kernel sources at capture time: reported only while the sources are unchanged.
 NCU_TRAFFIC = {
     # (workload, pass): (bytes per launch, sources hash, capture)
-    ("b2_t16k_gqa4_bf16_d128_a2", "out_pass"): (633.9e6, "b6baa11af0ee0f8b",
-                                                "out_pair_kernel, ncu --metrics dram__bytes_*"),
-    ("b2_t16k_gqa4_bf16_d128_a2", "tau_pass"): (563.1e6, "b6baa11af0ee0f8b",
+    ("b2_t16k_gqa4_bf16_d128_a2", "tau_pass"): (626.5e6, "ff78b661ea37d589",
                                                 "tau_tc_kernel, ncu --metrics dram__bytes_*"),
 }
 
@@ -314,11 +312,14 @@ def workload_config(w, world):
             "tile": "128x128", "parallelism": f"dp{world} (independent per-rank problems)"}
 
 
-def launches_per_step(w) -> int:
+def launches_per_step(w, mode: str = "fused") -> int:
     """Kernels of one step on the library's full workspace: the tau kernel, the overflow kernel
-    and the output kernel, plus for bf16 problems with at least 1024 keys the key-norm and
-    warm-up selection kernels of the tau pass."""
-    return 3 + (2 if w.dtype == "bf16" and w.T >= 1024 else 0)
+    and the tile output kernel; for bf16 problems with at least 1024 keys the key-norm and
+    warm-up selection kernels of the tau pass; on the support path with bf16 inputs the kernel
+    that computes o from the supports."""
+    bf16 = w.dtype == "bf16"
+    return (3 + (2 if bf16 and w.T >= 1024 else 0)
+            + (1 if bf16 and mode == "fused" else 0))
 
 
 # The forward pass, three ways through the C ABI's two-pass entry points:
@@ -440,7 +441,7 @@ def run_native(args, rank, world, local):
     # the tile path (every query tile's output recomputed over its active key tiles on the
     # tensor cores), on the same inputs, for comparison: same warm-up, same step count
     tile = None
-    if not nm:
+    if not nm and not args.step_only:
         ms_t, tt_tau, tt_out, _ = pb.time("tile", args.steps, args.warmup, world)
         ms_t = max_over_ranks(ms_t, world)
         out_tile = float(np.mean(tt_out))
@@ -471,8 +472,8 @@ def run_native(args, rank, world, local):
             ea.entmax_attn_fwd_host(qh, kh, vh, pb.alpha, w.n_iter, w.causal, cu, out=outh,
                                     tau=tauh, block_mask=maskh, stream=stream, synchronize=False)
 
-    e2e_steps = max(2, min(args.steps, 5))
-    for _ in range(2):
+    e2e_steps = 0 if args.step_only else max(2, min(args.steps, 5))
+    for _ in range(2 if e2e_steps else 0):
         fwd_e2e()
     torch.cuda.synchronize()
     barrier(world)
@@ -482,7 +483,7 @@ def run_native(args, rank, world, local):
         fwd_e2e()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_one = e0.elapsed_time(e1) / e2e_steps
+    e2e_one = e0.elapsed_time(e1) / e2e_steps if e2e_steps else float("nan")
     e2e_ms = max_over_ranks(e2e_one, world)
     e2e_rate = job_rate(eff_flops, e2e_one, world)
     assert ea.status(stream) == 0
@@ -490,7 +491,7 @@ def run_native(args, rank, world, local):
                                                     + mask.numel() * 4)
 
     others = []
-    for name in secondary(args):
+    for name in ([] if args.step_only else secondary(args)):
         w2 = WORKLOADS[name]
         p2 = Problem(w2, rank, local)
         ms2, t2_tau, t2_out, nfb2 = p2.time("fused", args.steps, args.warmup, world)
@@ -535,7 +536,7 @@ def run_native(args, rank, world, local):
                                       else "4 d flops per valid pair inside active tiles"))}
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.step_only:
         fl, nr, dt, nt, thr = oracle_tile_sample(w, pb.host, args.cpu_budget)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"{nt} whole 128-row query tiles ({nr} rows) drawn uniformly, "
@@ -569,12 +570,12 @@ def run_native(args, rank, world, local):
         "tile_path": tile,
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_rate / 1e12, "unit": "TFLOP/s",
+        "e2e": None if args.step_only else {"value": e2e_rate / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": pb.in_bytes,
                 "d2h_bytes_per_step": d2h_bytes,
                 "entry": ("entmax_attn_fwd_no_block_mask + torch copies" if nm
                           else "entmax_attn_fwd_host (pinned host buffers)")},
-        "gpu_launches": launches_per_step(w) * args.steps,
+        "gpu_launches": launches_per_step(w, mode) * args.steps,
         "clocks": clk.summary(),
         "other_workloads": others,
     }
@@ -714,6 +715,9 @@ def main():
     ap.add_argument("--also", default="auto",
                     help="other workloads timed in the same run (comma list, 'none'; 'auto': "
                          "the 16K workload beside the 128K one and back)")
+    ap.add_argument("--step-only", action="store_true",
+                    help="time the step only (no tile-path comparison, e2e, cpu baseline or "
+                         "second workload): for profiler launch lists")
     ap.add_argument("--no-block-mask", action="store_true",
                     help="time the variant without block mask (output pass over every causal "
                          "tile); the effective FLOPs keep counting active tiles only")

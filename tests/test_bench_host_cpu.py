@@ -54,5 +54,7 @@ def test_clock_summary_reads_median_clock_and_active_reasons():
 
 def test_launches_per_step():
     assert bench.launches_per_step(WORKLOADS["t256_fp32_d64_a1.5"]) == 3
-    assert bench.launches_per_step(WORKLOADS["t4k_bf16_d64_a1.5"]) == 5
-    assert bench.launches_per_step(WORKLOADS["b2_t16k_gqa4_bf16_d128_a2"]) == 5
+    assert bench.launches_per_step(WORKLOADS["t4k_bf16_d64_a1.5"]) == 6
+    assert bench.launches_per_step(WORKLOADS["b2_t16k_gqa4_bf16_d128_a2"]) == 6
+    assert bench.launches_per_step(WORKLOADS["b2_t16k_gqa4_bf16_d128_a2"], "tile") == 5
+    assert bench.launches_per_step(WORKLOADS["b2_t16k_gqa4_bf16_d128_a2"], "nomask") == 5
