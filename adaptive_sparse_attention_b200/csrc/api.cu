@@ -346,14 +346,16 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
   P.tau = const_cast<float*>(tau);
   attach_workspace(&P, wv);
   P.no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) ? 1 : 0;
-  P.from_support = (flags & ENTMAX_ATTN_FLAG_SUPPORT) ? 1 : 0;
+  // with the support sections (the tau pass recorded into them), the recorded query tiles from
+  // their lists and the tile pass for the pending ones; without, the tile pass for all
+  P.from_support =
+      ((flags & ENTMAX_ATTN_FLAG_SUPPORT) && workspace_bytes >= wv.bytes) ? 1 : 0;
   if ((flags & ENTMAX_ATTN_FLAG_OUT_FP32) && !use_tensor_cores(dtype, flags))
     return ENTMAX_ATTN_EINVAL;  // fp32 outputs of bf16 inputs: the tensor-core path only
   P.out_f32 = (flags & ENTMAX_ATTN_FLAG_OUT_FP32) ? 1 : 0;
   cudaError_t e = cudaSuccess;
-  // the recorded query tiles from their support lists (only the tensor-core tau pass records)
-  if (P.from_support && use_tensor_cores(dtype, flags) && workspace_bytes >= wv.bytes)
-    e = ea::launch_out_support(P, stream);
+  // only the tensor-core tau pass records supports; the CUDA-core path left every tile pending
+  if (P.from_support && use_tensor_cores(dtype, flags)) e = ea::launch_out_support(P, stream);
   if (e == cudaSuccess)
     e = use_tensor_cores(dtype, flags) ? ea::launch_out_tc(P, stream)
                                        : ea::launch_out_simt(P, dtype, stream);
@@ -385,6 +387,8 @@ int entmax_attn_bwd(const void* q, const void* k, const void* v, const void* dou
   P.tau = const_cast<float*>(tau);
   attach_workspace(&P, wv);
   P.no_mask = (flags & ENTMAX_ATTN_FLAG_NO_BLOCK_MASK) ? 1 : 0;
+  P.from_support =
+      ((flags & ENTMAX_ATTN_FLAG_SUPPORT) && workspace_bytes >= wv.bytes) ? 1 : 0;
   const size_t kv_bytes = sizeof(float) * static_cast<size_t>(cu_seqlens ? 1 : B) * Hkv * T * d;
   cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, stream);

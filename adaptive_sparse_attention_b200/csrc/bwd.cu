@@ -20,6 +20,11 @@
 //                     their dk and dv, summed over the tile's rows, into fp32 global memory with
 //                     atomics (several query tiles and the query heads of a group meet on each
 //                     key).
+//   bwd_support_kernel  with ENTMAX_ATTN_FLAG_SUPPORT, for every query tile whose rows' supports
+//                     the forward recorded (bf16): the same gradients over each row's support
+//                     list alone -- w, u, delta, ds, dq from the listed keys, dk and dv added
+//                     with vector atomics.  The two kernels above then take only the other
+//                     (pending) query tiles.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -119,6 +124,7 @@ __global__ void __launch_bounds__(kBT) bwd_delta_kernel(Problem P, const T* g, f
   const int tid = threadIdx.x, r = tid >> 1, hf = tid & 1;
   const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
+  if (P.from_support && P.pending[t.tile_id] == 0) return;  // bwd_support_kernel's tile
   load_tiles<T, D>(P, t, g, sm, tid);
   const bool row_ok = r < t.nrows;
   const int jmax = row_ok ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
@@ -154,6 +160,7 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(Problem P, const T* g, co
   const int tid = threadIdx.x, r = tid >> 1, hf = tid & 1;
   const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
   if (!t.valid) return;
+  if (P.from_support && P.pending[t.tile_id] == 0) return;  // bwd_support_kernel's tile
   load_tiles<T, D>(P, t, g, sm, tid);
   const bool row_ok = r < t.nrows;
   const int jmax = row_ok ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
@@ -241,6 +248,153 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(Problem P, const T* g, co
   }
 }
 
+// ------------------------------------------------------------------ backward from the supports --
+// w = p^(2 - alpha) (= [z - tau]^(beta - 1)) from the p the forward recorded.
+template <int BK>
+__device__ __forceinline__ float weight_from_p(float p, float two_minus_alpha) {
+  if (BK == kBetaOne) return 1.f;          // alpha = 2
+  if (BK == kBetaTwo) return sqrtf(p);     // alpha = 1.5
+  return exp2f(two_minus_alpha * __log2f(p));
+}
+
+// bf16 row slice of kCols consecutive elements (16-byte aligned) into fp32 registers.
+template <int kCols>
+__device__ __forceinline__ void load_slice(const __nv_bfloat16* src, float (&x)[kCols]) {
+#pragma unroll
+  for (int u = 0; u < kCols / 8; ++u) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src) + u);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[h]));
+      x[8 * u + 2 * h] = f.x;
+      x[8 * u + 2 * h + 1] = f.y;
+    }
+  }
+}
+
+// Sum over the 8 lanes of a row group (lanes 8 m .. 8 m + 7 of the warp).
+__device__ __forceinline__ float sum8(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  return x;
+}
+
+// One CTA of 128 threads per query tile that is not pending; 8 lanes per row, each owning D / 8
+// consecutive columns, 16 rows at a time.  First sweep over the row's support list: u = g . v_j
+// and w from p -> delta = sum w u / sum w; second sweep: ds = w (u - delta), dq += ds k_j, and
+// dk_j += ds q / sqrt(d), dv_j += p g with float4 atomics.  Every lane of a row group runs the
+// same trip counts (the shuffles need the whole warp), and list offsets, counts and keys are
+// clamped to the tile's list and sequence.
+constexpr int kBSupThreads = 128;
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kBSupThreads)
+    bwd_support_kernel(Problem P, const __nv_bfloat16* g, float* delta, float* dq, float* dk,
+                       float* dv) {
+  const TileInfo t = map_tile(P, gridDim.x - 1 - blockIdx.x, blockIdx.y, blockIdx.z);
+  if (!t.valid || P.pending[t.tile_id] != 0) return;
+  constexpr int kCols = D / 8;
+  const int l8 = threadIdx.x & 7;
+  const float scale = rsqrtf(static_cast<float>(D));
+  const float tma = 2.f - P.alpha;
+  const int2* list = P.sup + t.tile_id * kSupPerTile;
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(P.q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(P.k);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(P.v);
+  const int64_t kv0 = t.khead + t.seq_start;  // key row of the sequence's first key
+  // row groups of a warp run a common trip count: the warp's largest support
+  for (int r0 = 0; r0 < t.nrows; r0 += kBSupThreads / 8) {
+    const int r = r0 + (threadIdx.x >> 3);
+    const bool ok = r < t.nrows;
+    const int64_t row = t.qhead + t.seq_start + t.row0 + (ok ? r : 0);
+    const int idx = ok ? P.sup_idx[row] : 0;
+    const int first = min(idx & 0xffff, kSupPerTile);
+    const int n = ok ? min(max(idx >> 16, 0), kSupPerTile - first) : 0;
+    int nmax = n;
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) nmax = max(nmax, __shfl_xor_sync(0xffffffffu, nmax, o));
+    float gi[kCols];
+    load_slice<kCols>(g + row * D + l8 * kCols, gi);
+    float sw = 0.f, swu = 0.f;
+    for (int e = 0; e < nmax; ++e) {
+      const bool has = e < n;
+      const int2 en = has ? list[first + e] : make_int2(0, 0);
+      const int j = min(max(en.x, 0), t.seq_len - 1);
+      float vj[kCols];
+      load_slice<kCols>(vb + (kv0 + j) * D + l8 * kCols, vj);
+      float u = 0.f;
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) u = fmaf(gi[c], vj[c], u);
+      u = sum8(u);
+      const float p = __int_as_float(en.y);
+      const float w = (has && p > 0.f) ? weight_from_p<BK>(p, tma) : 0.f;
+      sw += w;
+      swu = fmaf(w, u, swu);
+    }
+    const float dl = sw > 0.f ? swu / sw : 0.f;
+    float qi[kCols], aq[kCols];
+    load_slice<kCols>(qb + row * D + l8 * kCols, qi);
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) aq[c] = 0.f;
+    for (int e = 0; e < nmax; ++e) {
+      const bool has = e < n;
+      const int2 en = has ? list[first + e] : make_int2(0, 0);
+      const int j = min(max(en.x, 0), t.seq_len - 1);
+      float vj[kCols], kj[kCols];
+      load_slice<kCols>(vb + (kv0 + j) * D + l8 * kCols, vj);
+      load_slice<kCols>(kb + (kv0 + j) * D + l8 * kCols, kj);
+      float u = 0.f;
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) u = fmaf(gi[c], vj[c], u);
+      u = sum8(u);
+      if (!has) continue;  // the shuffles are done; the rest is this row group's own
+      const float p = __int_as_float(en.y);
+      const float w = p > 0.f ? weight_from_p<BK>(p, tma) : 0.f;
+      const float ds = w * (u - dl);
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) aq[c] = fmaf(ds, kj[c], aq[c]);
+      float4* dkr = reinterpret_cast<float4*>(dk + (kv0 + j) * D + l8 * kCols);
+      float4* dvr = reinterpret_cast<float4*>(dv + (kv0 + j) * D + l8 * kCols);
+      const float dss = ds * scale;
+#pragma unroll
+      for (int c = 0; c < kCols; c += 4) {
+        atomicAdd(dkr + c / 4, make_float4(dss * qi[c], dss * qi[c + 1], dss * qi[c + 2],
+                                           dss * qi[c + 3]));
+        atomicAdd(dvr + c / 4, make_float4(p * gi[c], p * gi[c + 1], p * gi[c + 2],
+                                           p * gi[c + 3]));
+      }
+    }
+    if (!ok) continue;
+    float4* dqr = reinterpret_cast<float4*>(dq + row * D + l8 * kCols);
+#pragma unroll
+    for (int c = 0; c < kCols; c += 4)
+      dqr[c / 4] = make_float4(aq[c] * scale, aq[c + 1] * scale, aq[c + 2] * scale,
+                               aq[c + 3] * scale);
+    if (l8 == 0) delta[row] = dl;
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_support_d(const Problem& P, const void* g, float* delta, float* dq,
+                                 float* dk, float* dv, cudaStream_t s) {
+  const dim3 grid(P.slots, P.Hq, P.cu ? 1 : P.B);
+  const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(g);
+  switch (beta_kind(P.beta)) {
+    case kBetaOne:
+      bwd_support_kernel<D, kBetaOne><<<grid, kBSupThreads, 0, s>>>(P, gb, delta, dq, dk, dv);
+      break;
+    case kBetaTwo:
+      bwd_support_kernel<D, kBetaTwo><<<grid, kBSupThreads, 0, s>>>(P, gb, delta, dq, dk, dv);
+      break;
+    default:
+      bwd_support_kernel<D, kBetaGeneral><<<grid, kBSupThreads, 0, s>>>(P, gb, delta, dq, dk,
+                                                                       dv);
+  }
+  return cudaGetLastError();
+}
+
 template <typename T, int D, int BK>
 cudaError_t launch_bwd_t(const Problem& P, const void* g, float* delta, float* dq, float* dk,
                          float* dv, cudaStream_t s) {
@@ -273,6 +427,11 @@ cudaError_t launch_bwd_d(const Problem& P, const void* g, float* delta, float* d
 
 cudaError_t launch_bwd(const Problem& P, int dtype, const void* g, float* delta, float* dq,
                        float* dk, float* dv, cudaStream_t s) {
+  if (P.from_support && dtype == 1) {  // the recorded tiles from their supports, then the others
+    cudaError_t e = P.d == 64 ? launch_bwd_support_d<64>(P, g, delta, dq, dk, dv, s)
+                              : launch_bwd_support_d<128>(P, g, delta, dq, dk, dv, s);
+    if (e != cudaSuccess) return e;
+  }
   if (dtype == 0)
     return P.d == 64 ? launch_bwd_d<float, 64>(P, g, delta, dq, dk, dv, s)
                      : launch_bwd_d<float, 128>(P, g, delta, dq, dk, dv, s);

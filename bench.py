@@ -587,12 +587,18 @@ BWD_METRIC = "effective TFLOP/s of the entmax attention backward pass (dq, dk, d
 
 
 def run_backward(args, rank, world, local):
-    """The backward pass (entmax_attn_bwd) of the workload, after one forward pass whose tau
-    and compact lists it reuses.  A step is one backward call over resident inputs and upstream
-    gradient.  Effective FLOPs: 10 d per valid pair inside active tiles (recomputed scores,
-    dout v^T, and the dq, dk, dv products); the kernels execute 14 d (scores and dout v^T are
-    formed in both of their sweeps), which the roofline line counts against the fp32 FMA peak of
-    the CUDA cores the pass runs on."""
+    """The backward pass (entmax_attn_bwd) of the workload, after one forward pass (with
+    ENTMAX_ATTN_FLAG_SUPPORT) whose tau, compact lists and support lists it reuses.  A step is
+    one backward call with the same flag over resident inputs and upstream gradient: the rows
+    with a recorded support from their supports (bwd_support_kernel), the other query tiles over
+    their listed key tiles on the CUDA cores.  Effective FLOPs: 10 d per valid pair inside
+    active tiles, the work of the pages' tile-based backward (recomputed scores, dout v^T, and
+    the dq, dk, dv products), a fixed count per workload.  The support kernel is a gather and
+    scatter bound by memory, so its roofline counts the bytes the step must move (q, dout, k, v
+    read once; dq, dk, dv and delta written once) against the measured HBM bandwidth.  The tile
+    path (every query tile over its listed key tiles) is timed beside it where it takes under a
+    few seconds per step."""
+    from adaptive_sparse_attention_b200 import _native
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     q, k, v, cu = make_inputs(w, seed=rank)
@@ -604,10 +610,16 @@ def run_backward(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     out, tau, mask = ea.alloc_outputs(qd, kd, cud)
     ws = ea.alloc_workspace(qd, kd, cud)
-    ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, stream=stream)
-    ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, stream=stream)
+    sup = _native.FLAG_SUPPORT
+    ea.tau_pass(qd, kd, tau, mask, ws, alpha, w.n_iter, w.causal, cud, flags=sup, stream=stream)
+    ea.out_pass(qd, kd, vd, tau, ws, out, alpha, w.causal, cud, flags=sup, stream=stream)
+
+    def bwd(flags):
+        return ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud, flags=flags,
+                                  stream=stream)
+
     for _ in range(args.warmup):
-        grads = ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud, stream=stream)
+        grads = bwd(sup)
     torch.cuda.synchronize()
     assert ea.status(stream) == 0
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -616,47 +628,67 @@ def run_backward(args, rank, world, local):
     with ClockSampler(local) as clk:
         start.record(stream)
         for _ in range(args.steps):
-            grads = ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud,
-                                       stream=stream)
+            grads = bwd(sup)
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     total_ms = start.elapsed_time(stop)
-    ms_step = max_over_ranks(total_ms / args.steps, world)
+    ms_one = total_ms / args.steps
+    ms_step = max_over_ranks(ms_one, world)
     assert ea.status(stream) == 0
+    nfb = ea.fallback_tiles(ws, stream)
     bits = ea.decode_block_mask(mask.cpu().numpy(), w.B, w.Hq, w.T, cu)
     act_pairs, _ = count_pairs(w, bits, cu)
     eff_flops = 10 * w.d * act_pairs
-    value = job_rate(eff_flops, total_ms / args.steps, world) / 1e12
-    peaks, _ = load_peaks()
-    peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
-    achieved = 14 * w.d * act_pairs / (total_ms / args.steps * 1e-3) / 1e12
-    roofline = {"kernel": "bwd_grad_kernel + bwd_delta_kernel", "bound": "alu",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None,
-                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock",
-                "algorithmic": "14 d flops per valid pair inside active tiles (both sweeps)"}
+    value = job_rate(eff_flops, ms_one, world) / 1e12
+    peaks, peak_src = load_peaks()
+    esz = q.element_size()
+    bytes_step = (2 * q.numel() * esz + 2 * k.numel() * esz   # q, dout, k, v read
+                  + q.numel() * 4 + 2 * k.numel() * 4          # dq, dk, dv written (fp32)
+                  + tau.numel() * 4)                           # delta written
+    achieved = bytes_step / (ms_one * 1e-3) / 1e9
+    roofline = {"kernel": "entmax_attn_bwd (bwd_support_kernel)", "bound": "hbm",
+                "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic": "q, dout, k, v read once; dq, dk, dv (fp32) and delta written "
+                               "once"}
+
+    tile = None
+    tile_steps = 0 if (args.step_only or w.T > 32768) else min(args.steps, 3)
+    if tile_steps:
+        bwd(0)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(tile_steps):
+            bwd(0)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms_t = max_over_ranks(t0.elapsed_time(t1) / tile_steps, world)
+        tile = {"ms_per_step": ms_t, "value": job_rate(eff_flops, ms_t, world) / 1e12,
+                "steps": tile_steps}
 
     # end to end: H2D of the upstream gradient from pinned memory, the backward call, D2H of
     # dq, dk and dv, every step (forward state resident)
     gh = g.pin_memory()
     dq, dk, dv, _ = grads
     hosts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = 0 if args.step_only else max(2, min(args.steps, 5))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(e2e_steps):
         gd.copy_(gh, non_blocking=True)
-        res = ea.entmax_attn_bwd(qd, kd, vd, gd, tau, ws, alpha, w.causal, cud, stream=stream)
+        res = bwd(sup)
         for hst, dev_t in zip(hosts, res[:3]):
             hst.copy_(dev_t, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world) if e2e_steps else None
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.step_only:
         from oracle import backward as obwd  # the timed CPU baseline only
         import time
         # a bounded sample: the oracle backward of the workload's first (batch, head) over a
@@ -686,14 +718,19 @@ def run_backward(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": dict(workload_config(w, world), variant="backward",
-                       grads="fp32 dq, dk, dv"),
+                       grads="fp32 dq, dk, dv",
+                       path="rows with a recorded support from their supports; other query "
+                            "tiles over their listed key tiles"),
         "active_tile_pair_fraction": None,
+        "overflow_tiles": nfb,
+        "tile_path": tile,
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "e2e": {"value": job_rate(eff_flops, e2e_ms, world) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": g.numel() * g.element_size(),
-                "d2h_bytes_per_step": sum(t.numel() * 4 for t in (dq, dk, dv))},
-        "gpu_launches": 2 * args.steps,
+        "e2e": None if e2e_ms is None else {
+            "value": job_rate(eff_flops, e2e_ms, world) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": e2e_ms, "h2d_bytes_per_step": g.numel() * g.element_size(),
+            "d2h_bytes_per_step": sum(t.numel() * 4 for t in (dq, dk, dv))},
+        "gpu_launches": (3 if w.dtype == "bf16" else 2) * args.steps,
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -90,7 +90,9 @@ extern "C" {
                                              pass over the others only (overflowed candidates,
                                              supports beyond a tile's list, the CUDA-core path,
                                              a workspace below entmax_attn_workspace_bytes).
-                                             The path entmax_attn_fwd takes. */
+                                             The path entmax_attn_fwd takes.  Give the
+                                             output pass (and entmax_attn_bwd) this flag only
+                                             after a tau pass with it on the same workspace. */
 #define ENTMAX_ATTN_FLAG_OUT_FP32 32u     /* bf16 inputs on the tensor-core path: out is float
                                              (fp32 accumulations stored without rounding to
                                              bf16), same layout.  Give it to both passes;
@@ -181,7 +183,10 @@ int entmax_attn_out_pass(const void* q, const void* k, const void* v, const floa
  *   dk, dv: fp32, the layout of k / v, fully written (zeroed, then accumulated over the query
  *          heads of each group).
  * Computed on the CUDA cores in fp32 from the stored inputs.  flags: ENTMAX_ATTN_FLAG_NO_BLOCK_MASK
- * visits every causally valid key tile instead of the lists (for a tau pass run with that flag).
+ * visits every causally valid key tile instead of the lists (for a tau pass run with that flag);
+ * ENTMAX_ATTN_FLAG_SUPPORT (for a forward run with that flag on this workspace, bf16) computes
+ * the gradients of every row with a recorded support from its support list alone, and visits
+ * the listed key tiles only for the other query tiles.
  * Device pointers 16-byte aligned (workspace 256), asynchronous on `stream`.  Returns
  * ENTMAX_ATTN_OK, ENTMAX_ATTN_EINVAL (as the forward, or a null pointer), ENTMAX_ATTN_EALIGN,
  * ENTMAX_ATTN_ENOMEM (workspace below entmax_attn_workspace_min_bytes) or ENTMAX_ATTN_ECUDA. */

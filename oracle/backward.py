@@ -90,6 +90,48 @@ def attention_backward(q, k, v, dout, alpha: float, causal: bool = True, cu_seql
     return dq, dk, dv, delta
 
 
+def row_gradients(q, k, v, dout, alpha: float, causal: bool = True, cu_seqlens=None, rows=()):
+    """dq and delta of the given query rows only, in fp64: the same formulas as
+    ``attention_backward`` (each row's dq and delta depend on that row alone), for checking
+    sampled rows of problems too large for the full oracle.  rows are flat indices into
+    q.reshape(-1, d) (fixed length: (b * Hq + h) * T + t; packed: h * T + token).  Returns
+    (dq [len(rows), d], delta [len(rows)])."""
+    qf, kf, vf, gf = _f64(q), _f64(k), _f64(v), _f64(dout)
+    packed = cu_seqlens is not None
+    if packed:
+        qf, kf, vf, gf = qf[None], kf[None], vf[None], gf[None]
+    B, Hq, T, d = qf.shape
+    G = Hq // kf.shape[1]
+    scale = 1.0 / np.sqrt(d)
+    beta = 1.0 / (alpha - 1.0)
+    seqs = _sequences(T, cu_seqlens)
+    starts = np.array([st for st, _ in seqs])
+    rows = np.asarray(rows, dtype=np.int64)
+    dq = np.zeros((rows.size, d))
+    delta = np.zeros(rows.size)
+    for n_, row in enumerate(rows):
+        tok = int(row % T)
+        h = int((row // T) % Hq)
+        b = int(row // (T * Hq))
+        sidx = int(np.searchsorted(starts, tok, side="right") - 1)
+        start, length = seqs[sidx]
+        t = tok - start
+        n = t + 1 if causal else length
+        K = kf[b, h // G, start:start + n]
+        V = vf[b, h // G, start:start + n]
+        qi, gi = qf[b, h, tok], gf[b, h, tok]
+        s = K @ qi * scale
+        p, tau = oracle.entmax_vec((alpha - 1.0) * s, alpha)
+        x = (alpha - 1.0) * s - tau
+        w = np.zeros_like(p)
+        w[p > 0.0] = x[p > 0.0] ** (beta - 1.0)
+        u = V @ gi
+        dl = float(w @ u) / float(w.sum())
+        delta[n_] = dl
+        dq[n_] = (w * (u - dl)) @ K * scale
+    return dq, delta
+
+
 def attention_forward_fp64(q, k, v, alpha: float, causal: bool = True, cu_seqlens=None):
     """The forward output in fp64 from fp64 inputs (exact tau per row), for numerical
     differentiation in the tests: the same definition as ``oracle.attention_rows`` without its

@@ -99,3 +99,17 @@ def test_value_gradient_total_equals_dout_total():
     # sum_j dv_j = sum_i (sum_j p_ij) g_i = sum_i g_i, per (batch, kv head) over its query heads
     want = g.reshape(2, 2, 2, 6, 3).sum(axis=(2, 3))
     np.testing.assert_allclose(dv.sum(axis=2), want, atol=1e-12)
+
+
+@pytest.mark.parametrize("packed", [None, (5, 1, 9)], ids=["fixed", "packed"])
+@pytest.mark.parametrize("causal", [True, False])
+def test_row_gradients_equal_the_full_backward(packed, causal):
+    """row_gradients (dq and delta of chosen rows, for sampled checks at large sizes) equals
+    the full backward oracle on every row of small problems, GQA and packed included."""
+    rng = np.random.default_rng(11)
+    q, k, v, g, cu = _problem(rng, 2, 4, 2, 12, 8, packed)
+    dq, _, _, delta = bwd.attention_backward(q, k, v, g, 1.5, causal, cu)
+    rows = np.arange(dq.reshape(-1, dq.shape[-1]).shape[0])[::-1]  # every row, in reverse
+    rdq, rdelta = bwd.row_gradients(q, k, v, g, 1.5, causal, cu, rows)
+    np.testing.assert_allclose(rdq, dq.reshape(-1, dq.shape[-1])[rows], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(rdelta, delta.reshape(-1)[rows], rtol=1e-12, atol=1e-12)
