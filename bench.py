@@ -85,6 +85,8 @@ NCU_TRAFFIC = {
     # (workload, pass): (bytes per launch, sources hash, capture)
     ("b2_t16k_gqa4_bf16_d128_a2", "tau_pass"): (626.5e6, "ff78b661ea37d589",
                                                 "tau_tc_kernel, ncu --metrics dram__bytes_*"),
+    ("t128k_gqa4_bf16_d128_a1.5", "tau_pass"): (1535.9e6, "ff78b661ea37d589",
+                                                "tau_tc_kernel, ncu --metrics dram__bytes_*"),
 }
 
 
@@ -390,6 +392,33 @@ class Problem:
         return (start.elapsed_time(stop) / steps, [e[0].elapsed_time(e[1]) for e in evs],
                 [e[1].elapsed_time(e[2]) for e in evs], nfb)
 
+    def time_e2e(self, steps, world):
+        """ms per call of entmax_attn_fwd_host on pinned host copies of the inputs and outputs
+        (CUDA events on the stream the call completes on), after two untimed calls."""
+        w, q, k, v, cu = self.w, *self.host
+        qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+        outh = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        tauh = torch.empty(self.tau.shape, dtype=self.tau.dtype).pin_memory()
+        maskh = torch.empty(self.mask.shape, dtype=self.mask.dtype).pin_memory()
+
+        def call():
+            ea.entmax_attn_fwd_host(qh, kh, vh, self.alpha, w.n_iter, w.causal, cu, out=outh,
+                                    tau=tauh, block_mask=maskh, stream=self.stream,
+                                    synchronize=False)
+
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for _ in range(steps):
+            call()
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        assert ea.status(self.stream) == 0
+        return e0.elapsed_time(e1) / steps
+
     def pair_counts(self):
         """(pairs inside active tiles, all causally valid pairs) from the last masked tau pass."""
         w = self.w
@@ -498,11 +527,15 @@ def run_native(args, rank, world, local):
         a2, d2 = p2.pair_counts()
         ms2_max = max_over_ranks(ms2, world)
         v2 = job_rate(4 * w2.d * a2, ms2, world) / 1e12
+        e2 = p2.time_e2e(max(2, min(args.steps, 5)), world)
         others.append({"workload": name, "value": v2, "unit": "TFLOP/s", "ms_per_step": ms2_max,
                        "frac_of_bf16_peak": None, "ms_tau_pass": float(np.mean(t2_tau)),
                        "ms_out_pass": float(np.mean(t2_out)),
                        "active_tile_pair_fraction": a2 / d2, "overflow_tiles": nfb2,
-                       "tau_pass_tflops": 2 * w2.d * d2 / (float(np.mean(t2_tau)) * 1e-3) / 1e12})
+                       "tau_pass_tflops": 2 * w2.d * d2 / (float(np.mean(t2_tau)) * 1e-3) / 1e12,
+                       "e2e": {"value": job_rate(4 * w2.d * a2, e2, world) / 1e12,
+                               "unit": "TFLOP/s", "ms_per_step": max_over_ranks(e2, world),
+                               "entry": "entmax_attn_fwd_host (pinned host buffers)"}})
         del p2
         torch.cuda.empty_cache()
 
