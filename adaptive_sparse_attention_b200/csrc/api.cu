@@ -480,9 +480,25 @@ int entmax_attn_route_chunks(const void* q, const void* summaries, float* pi, fl
   if ((reinterpret_cast<uintptr_t>(q) % esz) || (reinterpret_cast<uintptr_t>(summaries) % esz) ||
       (reinterpret_cast<uintptr_t>(pi) & 3u) || (reinterpret_cast<uintptr_t>(tau) & 3u))
     return ENTMAX_ATTN_EALIGN;
-  cudaError_t e = ea::launch_route_chunks(q, summaries, pi, tau, B, Hq, Hkv, T, d, nc, chunk_size,
-                                          alpha, n_iter, causal, estimate_diagonal,
-                                          scaling_factor, dtype, stream);
+  // the scores on the tensor cores where the shapes allow (bf16, d = 64 or 128, TMA-aligned
+  // inputs, row counts within the tensor map's 32-bit coordinates), then the search
+  const int64_t q_rows = static_cast<int64_t>(B) * Hq * T;
+  const bool tc = dtype == ENTMAX_ATTN_BF16 && (d == 64 || d == 128) && aligned16(q) &&
+                  aligned16(summaries) && q_rows < (int64_t(1) << 31) &&
+                  static_cast<int64_t>(B) * Hkv * nc < (int64_t(1) << 31);
+  cudaError_t e = cudaSuccess;
+  if (tc) {
+    int err = ENTMAX_ATTN_OK;
+    int* st = status_ptr(&err);
+    if (!st) return err;
+    // the CUDA-core search kernel's own z scale, computed the same way
+    const float zscale = (alpha - 1.f) * scaling_factor / sqrtf(static_cast<float>(d));
+    e = ea::launch_route_scores_tc(q, summaries, pi, B, Hq, Hkv, T, d, nc, zscale, st, stream);
+  }
+  if (e == cudaSuccess)
+    e = ea::launch_route_chunks(q, summaries, pi, tau, B, Hq, Hkv, T, d, nc, chunk_size, alpha,
+                                n_iter, causal, estimate_diagonal, scaling_factor, dtype,
+                                tc ? 1 : 0, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return ENTMAX_ATTN_OK;
 }

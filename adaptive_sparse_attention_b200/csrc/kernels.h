@@ -30,11 +30,17 @@ cudaError_t launch_warm(const Problem& P, cudaStream_t s);
 cudaError_t launch_bwd(const Problem& P, int dtype, const void* g, float* delta, float* dq,
                        float* dk, float* dv, cudaStream_t s);
 
-// Entmax block routing over chunk summaries (pi fp32 [B, Hq, T, nc], tau fp32 [B, Hq, T]).
+// Entmax block routing over chunk summaries (pi fp32 [B, Hq, T, nc], tau fp32 [B, Hq, T]);
+// with scores_ready the rows of pi already hold z = (alpha - 1) scaling q . sigma / sqrt(d).
 cudaError_t launch_route_chunks(const void* q, const void* sig, float* pi, float* tau, int B,
                                 int Hq, int Hkv, int T, int d, int nc, int chunk, float alpha,
                                 int n_iter, int causal, int diag, float scaling, int dtype,
-                                cudaStream_t s);
+                                int scores_ready, cudaStream_t s);
+// z = zscale q . sigma for every (query row, chunk) into z [B, Hq, T, nc] on the tensor cores
+// (bf16, d in {64, 128}, q and sig 16-byte aligned); status: the device status word.
+cudaError_t launch_route_scores_tc(const void* q, const void* sig, float* z, int B, int Hq,
+                                   int Hkv, int T, int d, int nc, float zscale, int* status,
+                                   cudaStream_t s);
 
 // Row-wise alpha-entmax of a [rows, n] matrix x (row stride ldx elements) into p (row stride
 // ldp); dtype 0 = fp32, 1 = bf16 for both x and p; tau may be null.

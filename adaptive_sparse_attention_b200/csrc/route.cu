@@ -6,7 +6,8 @@
 // before their own and, with estimate_diagonal, their own (causal), or every chunk.
 // One warp per query row.  Lane l owns the chunks l, l + 32, ...: it writes their z = (alpha - 1) s
 // into the row of pi, reads them back at every search step and finally overwrites them with p, so
-// no lane ever reads an element another lane writes.
+// no lane ever reads an element another lane writes.  With scores_ready the rows of pi already
+// hold z for every chunk (route_scores_kernel, tensor cores), and the warp only searches.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -22,7 +23,7 @@ __global__ void __launch_bounds__(32 * kRouteRowsPerCta)
     route_chunks_kernel(const T* __restrict__ q, const T* __restrict__ sig, float* __restrict__ pi,
                         float* __restrict__ tau, int B, int Hq, int Hkv, int T_, int d, int nc,
                         int chunk, float alpha, float beta, float zscale, int n_iter, int causal,
-                        int diag) {
+                        int diag, int scores_ready) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRouteRowsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int64_t rows = static_cast<int64_t>(B) * Hq * T_;
@@ -45,11 +46,16 @@ __global__ void __launch_bounds__(32 * kRouteRowsPerCta)
   const unsigned full = 0xffffffffu;
   float m = -INFINITY;
   for (int c = lane; c < n; c += 32) {
-    const T* sc = sg + static_cast<int64_t>(c) * d;
-    float acc = 0.f;
-    for (int e = 0; e < d; ++e) acc = fmaf(load_elem(qr, e), load_elem(sc, e), acc);
-    const float z = zscale * acc;
-    pr[c] = z;
+    float z;
+    if (scores_ready) {
+      z = pr[c];
+    } else {
+      const T* sc = sg + static_cast<int64_t>(c) * d;
+      float acc = 0.f;
+      for (int e = 0; e < d; ++e) acc = fmaf(load_elem(qr, e), load_elem(sc, e), acc);
+      z = zscale * acc;
+      pr[c] = z;
+    }
     m = fmaxf(m, z);
   }
 #pragma unroll
@@ -87,7 +93,8 @@ __global__ void __launch_bounds__(32 * kRouteRowsPerCta)
 template <typename T>
 cudaError_t launch_route_t(const void* q, const void* sig, float* pi, float* tau, int B, int Hq,
                            int Hkv, int T_, int d, int nc, int chunk, float alpha, int n_iter,
-                           int causal, int diag, float scaling, cudaStream_t s) {
+                           int causal, int diag, float scaling, int scores_ready,
+                           cudaStream_t s) {
   const float beta = 1.f / (alpha - 1.f);
   const float zscale = (alpha - 1.f) * scaling / sqrtf(static_cast<float>(d));
   const int64_t rows = static_cast<int64_t>(B) * Hq * T_;
@@ -98,7 +105,7 @@ cudaError_t launch_route_t(const void* q, const void* sig, float* pi, float* tau
 #define EA_ROUTE_LAUNCH(BKV)                                                                   \
   route_chunks_kernel<T, BKV><<<grid, block, 0, s>>>(qp, sp, pi, tau, B, Hq, Hkv, T_, d, nc,   \
                                                      chunk, alpha, beta, zscale, n_iter,       \
-                                                     causal, diag)
+                                                     causal, diag, scores_ready)
   switch (beta_kind(beta)) {
     case kBetaOne: EA_ROUTE_LAUNCH(kBetaOne); break;
     case kBetaTwo: EA_ROUTE_LAUNCH(kBetaTwo); break;
@@ -114,11 +121,12 @@ cudaError_t launch_route_t(const void* q, const void* sig, float* pi, float* tau
 cudaError_t launch_route_chunks(const void* q, const void* sig, float* pi, float* tau, int B,
                                 int Hq, int Hkv, int T, int d, int nc, int chunk, float alpha,
                                 int n_iter, int causal, int diag, float scaling, int dtype,
-                                cudaStream_t s) {
+                                int scores_ready, cudaStream_t s) {
   return dtype == 0 ? launch_route_t<float>(q, sig, pi, tau, B, Hq, Hkv, T, d, nc, chunk, alpha,
-                                            n_iter, causal, diag, scaling, s)
+                                            n_iter, causal, diag, scaling, scores_ready, s)
                     : launch_route_t<__nv_bfloat16>(q, sig, pi, tau, B, Hq, Hkv, T, d, nc, chunk,
-                                                    alpha, n_iter, causal, diag, scaling, s);
+                                                    alpha, n_iter, causal, diag, scaling,
+                                                    scores_ready, s);
 }
 
 }  // namespace ea

@@ -1611,6 +1611,100 @@ __global__ void __launch_bounds__(kSupThreads)
   }
 }
 
+// ------------------------------------------------------------------ routing scores (tcgen05) --
+// route_scores_kernel: z[b, h, i, c] = zscale * q_i . sigma_c (sigma: the chunk summaries of kv
+// head floor(h / G)) for one 128-row x 128-chunk tile per CTA: the query and summary tiles come
+// in by TMA, one thread issues the d / 16 tcgen05.mma of the 128 x 128 product into TMEM, and the
+// four warps read their 32 rows back (thread = row) and store the row's 128 values (fp32, clipped
+// to the rows and chunks of the head).  Boxes past a head's rows read the next head's rows (never
+// stored) or, past the tensor, zeros.  Every wait is bounded as in the other kernels.
+constexpr int kRouteThreads = 128;
+
+template <int D>
+struct RouteSmem {
+  alignas(1024) __nv_bfloat16 q[kTile * D];
+  alignas(1024) __nv_bfloat16 s[kTile * D];
+  uint64_t full;
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+    route_scores_kernel(const __grid_constant__ CUtensorMap tmq,
+                        const __grid_constant__ CUtensorMap tms, float* __restrict__ z, int T,
+                        int nc, int Hq, int G, int Hkv, float zscale, int* status) {
+  extern __shared__ unsigned char smem_raw[];
+  RouteSmem<D>& sm = *reinterpret_cast<RouteSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.z, b = bh / Hq, h = bh % Hq;
+  const int i0 = blockIdx.x * kTile, c0 = blockIdx.y * kTile;
+  volatile int* abort = &sm.abort;
+  constexpr uint32_t kTileBytes = kTile * D * 2;
+  if (tid == 0) {
+    mbar_init(&sm.full, 1);
+    mbar_init(&sm.done, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc(&sm.tmem_base, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (tid == 0) {
+    mbar_expect_tx(&sm.full, 2 * kTileBytes);
+    const int qrow = bh * T + i0;
+    const int srow = (b * Hkv + h / G) * nc + c0;
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_2d(sm.q + hh * kTile * 64, &tmq, &sm.full, hh * 64, qrow);
+      tma_load_2d(sm.s + hh * kTile * 64, &tms, &sm.full, hh * 64, srow);
+    }
+    if (mbar_wait(&sm.full, 0, abort, status)) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+#pragma unroll
+      for (int k16 = 0; k16 < D / 16; ++k16)
+        mma_ss(tmem, kmajor_desc(smem_u32(sm.q), kTile, k16), kmajor_desc(smem_u32(sm.s), kTile, k16),
+               idesc, k16 > 0 ? 1u : 0u);
+      mma_commit(&sm.done);
+    } else {
+      mbar_wait(&sm.full, 0, abort, status);  // bounded: the copies land before the CTA exits
+    }
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&sm.done, 0, abort, status) && !*abort;
+  tc_fence_after();
+  const int r = warp * 32 + lane;  // row of the tile == TMEM lane
+  float* zr = z + (static_cast<int64_t>(bh) * T + i0 + r) * nc + c0;
+  const bool row_ok = i0 + r < T;
+#pragma unroll 1
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t u[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(32 * cc), u);
+    if (!ok || !row_ok) continue;
+    const int cb = c0 + 32 * cc;
+    if (cb + 32 <= nc && (nc & 3) == 0) {  // whole 32-chunk run, 16-byte aligned row
+      float4* dst = reinterpret_cast<float4*>(zr + 32 * cc);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[e] = make_float4(zscale * __uint_as_float(u[4 * e]), zscale * __uint_as_float(u[4 * e + 1]),
+                             zscale * __uint_as_float(u[4 * e + 2]),
+                             zscale * __uint_as_float(u[4 * e + 3]));
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (cb + e < nc) zr[32 * cc + e] = zscale * __uint_as_float(u[e]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 // ------------------------------------------------------------------------------ host side --
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
@@ -1737,6 +1831,23 @@ cudaError_t launch_support_t(const Problem& P, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_route_scores_d(const void* q, const void* sig, float* z, int B, int Hq,
+                                  int Hkv, int T, int nc, float zscale, int* status,
+                                  cudaStream_t s) {
+  CUtensorMap mq, ms;
+  cudaError_t e = make_map(&mq, q, static_cast<int64_t>(B) * Hq * T, D);
+  if (e == cudaSuccess) e = make_map(&ms, sig, static_cast<int64_t>(B) * Hkv * nc, D);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(RouteSmem<D>) + 1024;
+  auto kern = route_scores_kernel<D>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((T + kTile - 1) / kTile, (nc + kTile - 1) / kTile, B * Hq);
+  kern<<<grid, kRouteThreads, smem, s>>>(mq, ms, z, T, nc, Hq, Hq / Hkv, Hkv, zscale, status);
+  return cudaGetLastError();
+}
+
 #define EA_TC_DISPATCH(FN)                                          \
   do {                                                              \
     const int bk = beta_kind(P.beta);                               \
@@ -1770,6 +1881,13 @@ cudaError_t launch_tau_tc_fallback(const Problem& P, int num_ctas, cudaStream_t 
   return launch_sweep_t<128, kBetaGeneral>(P, num_ctas, s);
 }
 cudaError_t launch_out_support(const Problem& P, cudaStream_t s) { return launch_support_t(P, s); }
+
+cudaError_t launch_route_scores_tc(const void* q, const void* sig, float* z, int B, int Hq,
+                                   int Hkv, int T, int d, int nc, float zscale, int* status,
+                                   cudaStream_t s) {
+  return d == 64 ? launch_route_scores_d<64>(q, sig, z, B, Hq, Hkv, T, nc, zscale, status, s)
+                 : launch_route_scores_d<128>(q, sig, z, B, Hq, Hkv, T, nc, zscale, status, s);
+}
 
 cudaError_t launch_out_tc(const Problem& P, cudaStream_t s) {
   // heads 2 j and 2 j + 1 share their key/value head when the group size is even

@@ -63,3 +63,14 @@ def test_routing_4k_heads(oracle):
     """4096 tokens, eight query heads over two kv heads, d = 128, chunks of 64 (64 chunks)."""
     q, sig = _case(1, 8, 2, 4096, 128, 64, "bf16", seed=42)
     _check(q, sig, 1.5, 10, 64, True, True)
+
+
+@pytest.mark.parametrize("T,d,C", [(1000, 128, 7), (2304, 64, 16), (8192, 128, 16)],
+                         ids=["ragged_nc143", "d64_nc144", "nc512"])
+def test_routing_tensor_core_scores(oracle, T, d, C):
+    """bf16 with d = 64 or 128: the chunk scores come from the tensor cores (128-row x 128-chunk
+    tiles), the search from the CUDA cores.  Ragged row and chunk counts (a chunk count that is
+    not a multiple of 4 takes the element-wise store), and 512 chunks per row."""
+    q, sig = _case(1, 4, 2, T, d, C, "bf16", seed=43)
+    _check(q, sig, 1.5, 10, C, True, True)
+    _check(q, sig, 2.0, 10, C, False, True)
