@@ -44,6 +44,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace ea {
 namespace {
@@ -61,198 +62,6 @@ constexpr uint32_t kTauColQ = 128 * kTauSBufs;  // TMEM columns of the query til
 constexpr uint32_t kTauTmemCols = 512;          // allocation (a power of two >= 32)
 static_assert(kTauColQ + 128 / 2 <= kTauTmemCols, "score buffers + Q (d <= 128) fit in TMEM");
 constexpr int kOutStages = 3;             // key tiles and value tiles in flight in the out pass
-constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every mbarrier wait
-constexpr int kTimeoutCode = 4;           // ENTMAX_ATTN_ETIMEOUT
-
-// ------------------------------------------------------------------------------ PTX wrappers --
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for the phase with the given parity.  Returns false (and raises the abort flag,
-// recording the timeout) if the phase did not complete within kWaitNs, or if another thread of
-// the CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitNs) {
-        *abort = 1;
-        atomicExch(status, kTimeoutCode);
-        return false;
-      }
-    }
-  }
-}
-
-// Asks for a box of the map to be brought into L2 ahead of its load.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// TMA store of one 128-row x 64-column box from shared memory (128-byte swizzle, as the map
-// describes) to global coordinates (x, y); the calling thread then waits until the copy has read
-// shared memory, so the buffer may be reused or the CTA may exit.
-__device__ __forceinline__ void tma_store_2d_and_wait(const CUtensorMap* map, const void* src,
-                                                      int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(x), "r"(y), "r"(smem_u32(src))
-      : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* holder, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(holder)),
-               "r"(ncols));
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1) << 46;  // descriptor version
-  d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
-  return d;
-}
-
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulate.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
-                                                  bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
-// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (lane = thread).
-// 32 consecutive TMEM columns of this warp's lanes into registers, waiting for the load in the
-// same asm statement: the registers are defined only once the data has arrived, so the compiler
-// cannot move a use of them ahead of the wait.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];\n"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
 
 // 32 consecutive output elements from fp32 words (TMEM), at element offset e of out: rounded to
 // bf16, or stored as fp32 when the caller asked for fp32 outputs (P.out_f32).  16-byte stores.
@@ -331,54 +140,6 @@ __device__ __forceinline__ void p_row32(const uint32_t (&u)[32], float c, float 
               : 0.f;
       pk[e] = pack_bf16x2(p0, p1);
     }
-  }
-}
-
-// Descriptor of a K-major 128B-swizzled operand tile of R rows whose d columns sit in 64-column
-// halves of R x 128 bytes; k16 selects the 16-column (32-byte) slice of the K dimension.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int rows, int k16) {
-  const uint32_t half = static_cast<uint32_t>(k16 >> 2) * static_cast<uint32_t>(rows) * 128u;
-  return sw128_desc(base + half + static_cast<uint32_t>(k16 & 3) * 32u, 16u, 1024u);
-}
-
-// Descriptor of the value tile as the MN-major B operand of O += P V: 128 keys (K) x d (N),
-// stored as 64-column halves of 128 rows x 128 bytes; k16 selects keys [16 k16, 16 k16 + 16).
-__device__ __forceinline__ uint64_t value_desc(uint32_t base, int k16) {
-  return sw128_desc(base + static_cast<uint32_t>(k16) * 2048u, 128u * 128u, 1024u);
-}
-
-// A shared-memory descriptor moved by a byte offset (the start address field holds address / 16
-// in 14 bits; every shared-memory address here is below 256 KB, so the field cannot overflow).
-__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
-  return desc + static_cast<uint64_t>(bytes >> 4);
-}
-
-// 32 raw scores of this thread's row from TMEM columns [ta, ta + 32), keys j0 + i; keys at or
-// past jmax (outside the row's causal / sequence range) read as -inf.
-__device__ __forceinline__ void tmem_row32(uint32_t ta, int j0, int jmax, float (&x)[32]) {
-  uint32_t u[32];
-  tmem_ld32(ta, u);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]);
-  if (j0 + 32 > jmax) {  // diagonal or ragged tile
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (j0 + i >= jmax) x[i] = -INFINITY;
-  }
-}
-
-// N (8 or 16) 32-bit words into N consecutive TMEM columns of this warp's lanes.
-template <int N>
-__device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t (&w)[N]) {
-  static_assert(N == 8 || N == 16, "8 or 16 columns");
-  if constexpr (N == 16) {
-    tmem_st16(taddr, w);
-  } else {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
-            taddr),
-        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-        : "memory");
   }
 }
 
@@ -1707,34 +1468,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 
 // ------------------------------------------------------------------------------ host side --
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D map over a [rows, d] bf16 matrix, box of 128 rows x 64 columns, 128-byte swizzle.
-cudaError_t make_map(CUtensorMap* map, const void* base, int64_t rows, int d) {
-  auto enc = get_encoder();
-  if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTile)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 int64_t q_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) * P.Hq * P.T; }
 int64_t kv_rows(const Problem& P) { return static_cast<int64_t>(P.cu ? 1 : P.B) * P.Hkv * P.T; }
 int64_t warm_rows(const Problem& P) {
@@ -1742,14 +1475,6 @@ int64_t warm_rows(const Problem& P) {
 }
 
 dim3 tile_grid(const Problem& P) { return dim3(P.slots, P.Hq, P.cu ? 1 : P.B); }
-
-// Streaming multiprocessors of the current device (one persistent CTA each).
-cudaError_t device_sms(int* sms) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
-  return e;
-}
 
 // Keys above this many bytes do not stay in L2 (126 MB) next to the streaming queries.
 constexpr int64_t kKeysInL2Bytes = 96ll << 20;
