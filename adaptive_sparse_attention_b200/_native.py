@@ -38,6 +38,10 @@ SIGNATURES = {
     "entmax_attn_tau_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _c_float, _c_int, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),
+    "entmax_attn_screen_bytes": (_c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "entmax_attn_tau_pass_screened": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _vp, _c_size_t,
+                                               _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                               _c_int, _c_int, _vp, _c_int, _c_uint, _vp]),
     "entmax_attn_out_pass": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_size_t, _vp, _c_int, _c_int,
                                       _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _c_int,
                                       _c_uint, _vp]),

@@ -245,6 +245,42 @@ def tau_pass(q, k, tau, block_mask, workspace, alpha=1.5, n_iter=10, causal=True
     N.check(rc, "entmax_attn_tau_pass")
 
 
+def screen_bytes(B, Hq, Hkv, T, packed: bool) -> int:
+    return int(N.lib().entmax_attn_screen_bytes(B, Hq, Hkv, T, int(packed)))
+
+
+def alloc_screen(q, k, cu_seqlens):
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    n = screen_bytes(B, Hq, Hkv, T, cu_seqlens is not None)
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def tau_pass_screened(q, k, tau, block_mask, workspace, screen, alpha=1.5, n_iter=10,
+                      causal=True, cu_seqlens=None, flags=0, stream=None):
+    """The tau pass with the FP8 screen of its key tiles (bf16, d = 128); same outputs as
+    tau_pass.  screen: a uint8 device buffer of screen_bytes(...) bytes."""
+    _check_inputs(q, k, None, cu_seqlens)
+    B, Hq, Hkv, T, d = problem_dims(q, k, cu_seqlens)
+    rc = N.lib().entmax_attn_tau_pass_screened(
+        _ptr(q), _ptr(k), _ptr(tau), _ptr(block_mask), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(screen),
+        screen.numel() * screen.element_size(), B, Hq, Hkv, T, d, float(alpha), int(n_iter),
+        int(bool(causal)), _ptr(cu_seqlens), _DT[q.dtype], int(flags), _stream(stream))
+    N.check(rc, "entmax_attn_tau_pass_screened")
+
+
+def entmax_attn_screened(q, k, v, alpha=1.5, n_iter=10, causal=True, cu_seqlens=None, flags=0,
+                         workspace=None, screen=None, stream=None):
+    """The forward pass with the FP8-screened tau pass (and the same flags for the output pass).
+    Returns (out, tau, block_mask, workspace, screen)."""
+    out, tau, mask = alloc_outputs(q, k, cu_seqlens)
+    ws = alloc_workspace(q, k, cu_seqlens) if workspace is None else workspace
+    scr = alloc_screen(q, k, cu_seqlens) if screen is None else screen
+    tau_pass_screened(q, k, tau, mask, ws, scr, alpha, n_iter, causal, cu_seqlens, flags, stream)
+    out_pass(q, k, v, tau, ws, out, alpha, causal, cu_seqlens, flags, stream)
+    return out, tau, mask, ws, scr
+
+
 def out_pass(q, k, v, tau, workspace, out, alpha=1.5, causal=True, cu_seqlens=None, flags=0,
              stream=None):
     _check_inputs(q, k, v, cu_seqlens)

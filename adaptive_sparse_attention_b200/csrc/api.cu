@@ -252,7 +252,8 @@ namespace {
 int tau_pass_impl(const void* q, const void* k, float* tau, uint32_t* block_mask,
                   void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int T, int d,
                   float alpha, int n_iter, int causal, const int32_t* cu_seqlens, int dtype,
-                  unsigned flags, cudaStream_t stream) {
+                  unsigned flags, cudaStream_t stream, const int* scr_list = nullptr,
+                  const int* scr_count = nullptr) {
   Layout L;
   ea::Problem P;
   int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
@@ -274,6 +275,8 @@ int tau_pass_impl(const void* q, const void* k, float* tau, uint32_t* block_mask
   P.force_fallback = (flags & ENTMAX_ATTN_FLAG_ALL_FALLBACK) ? 1 : 0;
   P.test_stall = (flags & ENTMAX_ATTN_FLAG_TEST_STALL) ? 1 : 0;
   P.no_mask = no_mask ? 1 : 0;
+  P.scr_list = scr_list;
+  P.scr_count = scr_count;
 
   cudaError_t e = cudaMemsetAsync(wv.queue_count, 0, sizeof(int), stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -312,6 +315,43 @@ int tau_pass_impl(const void* q, const void* k, float* tau, uint32_t* block_mask
 
 }  // namespace
 
+namespace {
+
+// FP8 screen sections: [q8 | q statistics | k8 | key-tile statistics | lists | counts].
+struct ScreenView {
+  void* q8;
+  void* qst;
+  void* k8;
+  void* kst;
+  int* list;
+  int* count;
+  size_t bytes;
+};
+
+ScreenView screen_view(void* base, const Layout& L, int B, int Hq, int Hkv, int T, bool packed) {
+  ScreenView v;
+  char* p = static_cast<char*>(base);
+  const size_t nb = packed ? 1 : static_cast<size_t>(B);
+  const size_t qrows = nb * Hq * T, krows = nb * Hkv * T, ktiles = nb * Hkv * L.slots;
+  size_t off = 0;
+  v.q8 = p + off;
+  off += align256(qrows * 128);
+  v.qst = p + off;
+  off += align256(qrows * 16);
+  v.k8 = p + off;
+  off += align256(krows * 128);
+  v.kst = p + off;
+  off += align256(ktiles * 16);
+  v.list = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * static_cast<size_t>(L.tiles) * L.nkt_max);
+  v.count = reinterpret_cast<int*>(p + off);
+  off += align256(sizeof(int) * static_cast<size_t>(L.tiles));
+  v.bytes = off;
+  return v;
+}
+
+}  // namespace
+
 extern "C" {
 
 int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* block_mask,
@@ -320,6 +360,36 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
                          int dtype, unsigned flags, cudaStream_t stream) {
   return tau_pass_impl(q, k, tau, block_mask, workspace, workspace_bytes, B, Hq, Hkv, T, d, alpha,
                        n_iter, causal, cu_seqlens, dtype, flags, stream);
+}
+
+size_t entmax_attn_screen_bytes(int B, int Hq, int Hkv, int T, int has_cu_seqlens) {
+  Layout L;
+  if (Hkv < 1 || Hq % Hkv != 0 || !make_layout(B, Hq, T, has_cu_seqlens != 0, &L)) return 0;
+  return screen_view(nullptr, L, B, Hq, Hkv, T, has_cu_seqlens != 0).bytes;
+}
+
+int entmax_attn_tau_pass_screened(const void* q, const void* k, float* tau, uint32_t* block_mask,
+                                  void* workspace, size_t workspace_bytes, void* screen,
+                                  size_t screen_bytes, int B, int Hq, int Hkv, int T, int d,
+                                  float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
+                                  int dtype, unsigned flags, cudaStream_t stream) {
+  Layout L;
+  ea::Problem P;
+  int rc = check_and_describe(q, k, B, Hq, Hkv, T, d, alpha, n_iter, causal, cu_seqlens, dtype,
+                              &L, &P);
+  if (rc != ENTMAX_ATTN_OK) return rc;
+  if (dtype != ENTMAX_ATTN_BF16 || d != 128 || !use_tensor_cores(dtype, flags) || !screen)
+    return ENTMAX_ATTN_EINVAL;  // the screen runs on the tensor cores, bf16, d = 128
+  if (reinterpret_cast<uintptr_t>(screen) & 255u) return ENTMAX_ATTN_EALIGN;
+  const ScreenView sv = screen_view(screen, L, B, Hq, Hkv, T, cu_seqlens != nullptr);
+  if (screen_bytes < sv.bytes) return ENTMAX_ATTN_ENOMEM;
+  int err = ENTMAX_ATTN_OK;
+  P.status = status_ptr(&err);
+  if (!P.status) return err;
+  cudaError_t e = ea::launch_screen(P, sv.q8, sv.qst, sv.k8, sv.kst, sv.list, sv.count, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return tau_pass_impl(q, k, tau, block_mask, workspace, workspace_bytes, B, Hq, Hkv, T, d, alpha,
+                       n_iter, causal, cu_seqlens, dtype, flags, stream, sv.list, sv.count);
 }
 
 int entmax_attn_out_pass(const void* q, const void* k, const void* v, const float* tau,

@@ -80,6 +80,10 @@ struct Problem {
   int record_support;
   int from_support;
   int out_f32;         // out is fp32 (bf16 inputs, tensor-core path): no rounding of o to bf16
+  // FP8 screen (entmax_attn_tau_pass_screened): per query tile the key tiles the tensor-core
+  // tau kernel visits (ascending, [tiles][nkt_max]) and their count; null = every causal tile
+  const int* scr_list;
+  const int* scr_count;
 };
 
 // Support entries a query tile's list holds (16 per row on average; rows may use more).
@@ -134,6 +138,24 @@ __device__ __forceinline__ TileInfo map_tile(const Problem& P, int slot, int h, 
   t.nkt = P.causal ? t.qt + 1 : nqt;
   t.tile_id = ((int64_t)b * P.Hq + h) * P.slots + slot;
   return t;
+}
+
+// Query tile L of the tau pass's tile order.  Slot-major: the longest tiles (highest slot) of
+// every head first, so that the tiles a persistent CTA takes in turn shrink as the pass runs
+// out.  Key-group-major (P.kv_major, when the keys do not fit in L2): all query tiles of one
+// (batch or sequence, kv head) -- its G heads, longest slot first -- before the next group, so
+// that the CTAs running at a time sweep the keys of one or two groups, which stay in L2, instead
+// of every group's; the load balance is a little worse (the tile lengths saw-tooth per group).
+__device__ __forceinline__ TileInfo tau_tile(const Problem& P, int L, int per_slot) {
+  if (P.kv_major) {
+    const int per_group = P.slots * P.G;
+    const int grp = L / per_group, r = L - grp * per_group;
+    const int hk = grp % P.Hkv;
+    return map_tile(P, P.slots - 1 - r / P.G, hk * P.G + r % P.G, grp / P.Hkv);
+  }
+  const int slot = P.slots - 1 - L / per_slot;
+  const int hb = L % per_slot;
+  return map_tile(P, slot, hb % P.Hq, hb / P.Hq);
 }
 
 // Warm-up keys.  A row's candidate threshold is (running max) - 1/c, and it is loose until the

@@ -30,6 +30,13 @@ cudaError_t launch_warm(const Problem& P, cudaStream_t s);
 cudaError_t launch_bwd(const Problem& P, int dtype, const void* g, float* delta, float* dq,
                        float* dk, float* dv, cudaStream_t s);
 
+// FP8 screen of the tau pass (screen.cu, bf16, d = 128): e4m3 copies of q (per row) and k (per
+// 128-key tile) with their scales and error norms, then per query tile the ascending list of key
+// tiles the bf16 tau pass must visit and its count.  q8 [q rows][128] bytes, qst float4 [q rows],
+// k8 [kv rows][128] bytes, kst float4 [(B or 1) Hkv slots], list [tiles][nkt_max], count [tiles].
+cudaError_t launch_screen(const Problem& P, void* q8, void* qst, void* k8, void* kst, int* list,
+                          int* count, cudaStream_t s);
+
 // Entmax block routing over chunk summaries (pi fp32 [B, Hq, T, nc], tau fp32 [B, Hq, T]);
 // with scores_ready the rows of pi already hold z = (alpha - 1) scaling q . sigma / sqrt(d).
 cudaError_t launch_route_chunks(const void* q, const void* sig, float* pi, float* tau, int B,

@@ -182,6 +182,16 @@ __device__ __forceinline__ int snake_tile(int r) {
   return r * g + ((r & 1) ? g - 1 - c : c);
 }
 
+// Key tiles the tau kernel visits for query tile t: every causally valid one, or with the FP8
+// screen the tile's list (clamped into the tile's key range, so that no workspace content sends a
+// read outside it); scr_tile gives the i-th.
+__device__ __forceinline__ int scr_count(const Problem& P, const TileInfo& t) {
+  return P.scr_count ? min(max(P.scr_count[t.tile_id], 0), t.nkt) : t.nkt;
+}
+__device__ __forceinline__ int scr_tile(const Problem& P, const TileInfo& t, int i) {
+  return P.scr_list ? clamp_kt(P.scr_list[t.tile_id * P.nkt_max + i], t.nkt) : i;
+}
+
 // Steps of a query tile in the tau pass: with a warm-up level (warm_level), step 0 is the
 // product with the level's 128 warm-up keys, which only raises the rows' thresholds; the key
 // tiles 0 .. nkt - 1 follow in order.
@@ -309,24 +319,6 @@ __device__ __forceinline__ void record_support(const Problem& P, const TileInfo&
   if (lane4 == 0) P.sup_idx[t.qhead + t.seq_start + t.row0 + r] = first | (total << 16);
 }
 
-// Query tile L of the tau pass's tile order.  Slot-major: the longest tiles (highest slot) of
-// every head first, so that the tiles a persistent CTA takes in turn shrink as the pass runs
-// out.  Key-group-major (P.kv_major, when the keys do not fit in L2): all query tiles of one
-// (batch or sequence, kv head) -- its G heads, longest slot first -- before the next group, so
-// that the CTAs running at a time sweep the keys of one or two groups, which stay in L2, instead
-// of every group's; the load balance is a little worse (the tile lengths saw-tooth per group).
-__device__ __forceinline__ TileInfo tau_tile(const Problem& P, int L, int per_slot) {
-  if (P.kv_major) {
-    const int per_group = P.slots * P.G;
-    const int grp = L / per_group, r = L - grp * per_group;
-    const int hk = grp % P.Hkv;
-    return map_tile(P, P.slots - 1 - r / P.G, hk * P.G + r % P.G, grp / P.Hkv);
-  }
-  const int slot = P.slots - 1 - L / per_slot;
-  const int hb = L % per_slot;
-  return map_tile(P, slot, hb % P.Hq, hb / P.Hq);
-}
-
 template <int D, int BK>
 __global__ void __launch_bounds__(tau_threads(D, BK), 1)
     tau_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -399,7 +391,7 @@ __global__ void __launch_bounds__(tau_threads(D, BK), 1)
               tma_prefetch_2d(&tmq, h * 64, static_cast<int>(tn.qhead + tn.seq_start + tn.row0));
         }
         ++it;
-        const int lvl = warm_level(P, t), ws = lvl >= 0 ? 1 : 0, nsteps = t.nkt + ws;
+        const int lvl = warm_level(P, t), ws = lvl >= 0 ? 1 : 0, nsteps = scr_count(P, t) + ws;
         const int wrow = (t.grp * P.warm_levels + lvl) * kTile;
         for (int i = 0; i < nsteps; ++i, ++gk) {
           const int s = gk % kStages;
@@ -413,9 +405,10 @@ __global__ void __launch_bounds__(tau_threads(D, BK), 1)
             for (int h = 0; h < D / 64; ++h)
               tma_load_2d(sm.k[s] + h * kTile * 64, &tmw, &sm.k_full[s], h * 64, wrow);
           } else {
+            const int kt = scr_tile(P, t, i - ws);
             for (int h = 0; h < D / 64; ++h)
               tma_load_2d(sm.k[s] + h * kTile * 64, &tmk, &sm.k_full[s], h * 64,
-                          krow0 + (i - ws) * kTile);
+                          krow0 + kt * kTile);
           }
         }
       }
@@ -440,7 +433,7 @@ __global__ void __launch_bounds__(tau_threads(D, BK), 1)
         if (!t.valid) continue;
         if (!mbar_wait(&sm.q_full, it & 1, abort, P.status)) break;
         ++it;
-        const int nsteps = t.nkt + warm_steps(P, t);
+        const int nsteps = scr_count(P, t) + warm_steps(P, t);
         for (int i = 0; i < nsteps; ++i, ++gk) {
           if (gk % kMmaWarps != mine) continue;
           const int s = gk % kStages, b = gk % kMainSBufs;
@@ -488,13 +481,13 @@ __global__ void __launch_bounds__(tau_threads(D, BK), 1)
       score_warps_sync();
       if (tid < kMaxWords) cs.words[tid] = 0u;
       if (tid == 0) cs.fallback = P.force_fallback;
-      const int ws = warm_steps(P, t), nsteps = t.nkt + ws;
+      const int ws = warm_steps(P, t), nsteps = scr_count(P, t) + ws;
       const int jmax = (r < t.nrows) ? (P.causal ? t.row0 + r + 1 : t.seq_len) : 0;
       RowCand rc;
       rc.init(1.f / P.c);
       for (int i = 0; i < nsteps; ++i, ++gs) {
         const int b = gs % kMainSBufs;
-        const int kt = i - ws;  // -1: the warm-up keys
+        const int kt = i < ws ? -1 : scr_tile(P, t, i - ws);  // -1: the warm-up keys
         // the warp leaves together: feed_warp needs all 32 lanes
         if (!__all_sync(0xffffffffu,
                         mbar_wait(&sm.s_full[b], (gs / kMainSBufs) & 1, abort, P.status)))

@@ -318,10 +318,11 @@ def launches_per_step(w, mode: str = "fused") -> int:
     """Kernels of one step on the library's full workspace: the tau kernel, the overflow kernel
     and the tile output kernel; for bf16 problems with at least 1024 keys the key-norm and
     warm-up selection kernels of the tau pass; on the support path with bf16 inputs the kernel
-    that computes o from the supports."""
+    that computes o from the supports; with the FP8 screen its two prep kernels and its sweep."""
     bf16 = w.dtype == "bf16"
     return (3 + (2 if bf16 and w.T >= 1024 else 0)
-            + (1 if bf16 and mode == "fused" else 0))
+            + (1 if bf16 and mode in ("fused", "screen") else 0)
+            + (3 if mode == "screen" else 0))  # the screen's two prep kernels and its sweep
 
 
 # The forward pass, three ways through the C ABI's two-pass entry points:
@@ -331,8 +332,9 @@ def launches_per_step(w, mode: str = "fused") -> int:
 #            this benchmark times;
 #   tile     without the flag: the output pass over every query tile's active key tiles (o
 #            recomputed tile by tile on the tensor cores), reported beside it;
-#   nomask   the variant without block mask (--no-block-mask).
-MODES = ("fused", "tile", "nomask")
+#   nomask   the variant without block mask (--no-block-mask);
+#   screen   the fused step with the FP8-screened tau pass (--fp8-screen).
+MODES = ("fused", "tile", "nomask", "screen")
 
 
 class Problem:
@@ -350,6 +352,7 @@ class Problem:
         self.stream = torch.cuda.current_stream(self.dev)
         self.out, self.tau, self.mask = ea.alloc_outputs(self.q, self.k, self.cu)
         self.ws = ea.alloc_workspace(self.q, self.k, self.cu)
+        self.screen = None
 
     def step(self, mode, ev=None):
         from adaptive_sparse_attention_b200 import _native
@@ -357,10 +360,16 @@ class Problem:
         a = (self.q, self.k)
         if ev:
             ev[0].record(s)
-        flags = {"fused": _native.FLAG_SUPPORT, "tile": 0,
+        flags = {"fused": _native.FLAG_SUPPORT, "tile": 0, "screen": _native.FLAG_SUPPORT,
                  "nomask": _native.FLAG_NO_BLOCK_MASK}[mode]
-        ea.tau_pass(*a, self.tau, self.mask, self.ws, self.alpha, w.n_iter, w.causal, self.cu,
-                    flags=flags, stream=s)
+        if mode == "screen":
+            if self.screen is None:
+                self.screen = ea.alloc_screen(self.q, self.k, self.cu)
+            ea.tau_pass_screened(*a, self.tau, self.mask, self.ws, self.screen, self.alpha,
+                                 w.n_iter, w.causal, self.cu, flags=flags, stream=s)
+        else:
+            ea.tau_pass(*a, self.tau, self.mask, self.ws, self.alpha, w.n_iter, w.causal, self.cu,
+                        flags=flags, stream=s)
         if ev:
             ev[1].record(s)
         ea.out_pass(*a, self.v, self.tau, self.ws, self.out, self.alpha, w.causal, self.cu,
@@ -419,6 +428,24 @@ class Problem:
         assert ea.status(self.stream) == 0
         return e0.elapsed_time(e1) / steps
 
+    def screen_kept(self):
+        """(key tiles the FP8 screen kept, all causally valid key tiles) of the last screened
+        tau pass, from the documented order of the screen buffer's sections."""
+        w, cu = self.w, self.host[3]
+        up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+        nb = 1 if cu is not None else w.B
+        slots, _ = ea.mask_layout(w.B, w.Hq, w.T, cu is not None)
+        nkt = -(-w.T // TILE)
+        tiles = nb * w.Hq * slots
+        off = (up(nb * w.Hq * w.T * 128) + up(nb * w.Hq * w.T * 16) + up(nb * w.Hkv * w.T * 128)
+               + up(nb * w.Hkv * slots * 16) + up(4 * tiles * nkt))
+        kept = int(self.screen[off:off + 4 * tiles].view(torch.int32).sum().item())
+        total = 0
+        for slot0, nq, start, L in ea.tile_slot_table(w.B, w.T, None if cu is None else
+                                                      cu.tolist()):
+            total += (nq * (nq + 1) // 2 if w.causal else nq * nq) * w.Hq
+        return kept, total
+
     def pair_counts(self):
         """(pairs inside active tiles, all causally valid pairs) from the last masked tau pass."""
         w = self.w
@@ -450,7 +477,7 @@ def run_native(args, rank, world, local):
     w = WORKLOADS[args.workload]
     pb = Problem(w, rank, local)
     nm = args.no_block_mask
-    mode = "nomask" if nm else "fused"
+    mode = "nomask" if nm else ("screen" if args.fp8_screen else "fused")
     clk = ClockSampler(local)  # samples the clocks during the timed region only
     ms_one, t_tau, t_out, nfb = pb.time(mode, args.steps, args.warmup, world, sampler=clk)
     ms_step = max_over_ranks(ms_one, world)
@@ -586,8 +613,9 @@ def run_native(args, rank, world, local):
         "config": dict(workload_config(w, world),
                        variant="no_block_mask" if nm else "block_mask",
                        path=("tau pass + output pass over every causal tile" if nm else
-                             "tau pass recording each row's support + output from the supports "
-                             "(tile output pass for query tiles without one)"),
+                             ("FP8 screen of the key tiles, then " if mode == "screen" else "")
+                             + "tau pass recording each row's support + output from the "
+                             "supports (tile output pass for query tiles without one)"),
                        l2=f"inputs {pb.in_bytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB "
                           f"L2; no flush" if pb.in_bytes > L2_BYTES
                        else "inputs fit in L2; no flush"),
@@ -600,6 +628,8 @@ def run_native(args, rank, world, local):
         "tau_pass_hbm_gbs": (q.numel() * q.element_size() + k.numel() * k.element_size()
                              + tau.numel() * 4 + mask.numel() * 4) / (mean_tau * 1e-3) / 1e9,
         "overflow_tiles": nfb,
+        "fp8_screen_kept_tiles": (dict(zip(("kept", "causal"), pb.screen_kept()))
+                                  if mode == "screen" else None),
         "tile_path": tile,
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -788,6 +818,8 @@ def main():
     ap.add_argument("--step-only", action="store_true",
                     help="time the step only (no tile-path comparison, e2e, cpu baseline or "
                          "second workload): for profiler launch lists")
+    ap.add_argument("--fp8-screen", action="store_true",
+                    help="time the step with the FP8-screened tau pass (bf16, d = 128)")
     ap.add_argument("--no-block-mask", action="store_true",
                     help="time the variant without block mask (output pass over every causal "
                          "tile); the effective FLOPs keep counting active tiles only")

@@ -155,6 +155,26 @@ int entmax_attn_tau_pass(const void* q, const void* k, float* tau, uint32_t* blo
                          int d, float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
                          int dtype, unsigned flags, cudaStream_t stream);
 
+/* FP8 screening of the tau pass (AdaSplash page, "AdaSplash with Block Masking": the pass needs
+ * only the keys that can carry p > 0, z_ij > tau_i >= max_j z_ij - 1).  A first sweep scores every
+ * causal key tile on the tensor cores from e4m3 copies of q (one scale per row) and k (one scale
+ * per 128-key tile) and bounds each score's error rigorously (Cauchy-Schwarz on the quantisation
+ * errors, plus the accumulation); a key tile in which no row can reach its running lower bound
+ * of the row max minus 1 (z units) holds no candidate and not the row max.  The bf16 tau pass
+ * then scores only the other key tiles.  The results are those of entmax_attn_tau_pass (same
+ * flags, workspace and outputs; give the output pass the same flags).  bf16 inputs on the tensor
+ * cores with d = 128 only (ENTMAX_ATTN_EINVAL otherwise).  screen: device memory of at least
+ * entmax_attn_screen_bytes(...) bytes, 256-byte aligned, owned by the caller (e4m3 copies of q
+ * and k, their statistics, per query tile the screened key tiles); ENTMAX_ATTN_ENOMEM if smaller.
+ * It costs one fp8 product per causal tile (half the tensor time of a bf16 one) and a bound test
+ * per row and key tile, so it pays only where the screen removes more than half of the tiles. */
+size_t entmax_attn_screen_bytes(int B, int Hq, int Hkv, int T, int has_cu_seqlens);
+int entmax_attn_tau_pass_screened(const void* q, const void* k, float* tau, uint32_t* block_mask,
+                                  void* workspace, size_t workspace_bytes, void* screen,
+                                  size_t screen_bytes, int B, int Hq, int Hkv, int T, int d,
+                                  float alpha, int n_iter, int causal, const int32_t* cu_seqlens,
+                                  int dtype, unsigned flags, cudaStream_t stream);
+
 /* Output pass: o_i = sum over the listed key tiles of p_ij v_j, with p recomputed from tau
  * (scores on the tensor cores, P rounded to bf16 for the P V product, fp32 accumulation).  With
  * ENTMAX_ATTN_FLAG_SUPPORT (given to the tau pass too): o_i = sum of p_ij v_j over the support

@@ -344,3 +344,25 @@ def test_host_entry_point_argument_checks(native):
     for vals in bad:
         ptr, keep = cu(vals)
         assert call(B=len(vals) - 1, T=300, cu=ptr) == native.EINVAL, vals
+
+
+def test_screened_tau_pass_argument_checks(native):
+    """entmax_attn_tau_pass_screened: bf16 on the tensor cores with d = 128 only, a 256-byte
+    aligned screen buffer of entmax_attn_screen_bytes() bytes (fake pointers, never launched)."""
+    lib = native.lib()
+    p = _fake(0x10000)
+    need = lib.entmax_attn_screen_bytes(1, 2, 1, 300, 0)
+    assert need > 0
+    assert lib.entmax_attn_screen_bytes(1, 3, 2, 300, 0) == 0  # Hq not a multiple of Hkv
+    ws = lib.entmax_attn_workspace_bytes(1, 2, 300, 0)
+
+    def call(d=128, dtype=native.BF16, flags=0, screen=p, sbytes=need):
+        return lib.entmax_attn_tau_pass_screened(p, p, p, p, p, ws, screen, sbytes, 1, 2, 1, 300,
+                                                 d, 1.5, 10, 1, None, dtype, flags, None)
+
+    assert call(d=64) == native.EINVAL
+    assert call(dtype=native.FP32) == native.EINVAL
+    assert call(flags=native.FLAG_CUDA_CORES) == native.EINVAL
+    assert call(screen=None) == native.EINVAL
+    assert call(screen=_fake(0x10010)) == native.EALIGN
+    assert call(sbytes=need - 1) == native.ENOMEM
