@@ -261,16 +261,25 @@ __device__ __forceinline__ void record_support(const Problem& P, const TileInfo&
   const int r = tid >> 2;  // 512 score threads: one row per 4-lane group
   const bool valid = r < t.nrows;
   const float tau = valid ? cs.tau_r[r] : 0.f;
-  // this lane's share of the row's entries: e = lane4, lane4 + 4, ... of every segment
-  int n = 0;
+  // This lane's share of the row's entries: e = lane4 + 4 i of every segment g, bit
+  // g * kPer + i of take when the entry lies in the support.  The test is made once and the
+  // writes below follow the bits: evaluated twice, z - tau of a key within rounding of tau could
+  // come out on different sides (the compiler may fuse the product and the difference in one place
+  // and not in the other), and the row would write one entry more or less than it counted, into
+  // the next row's part of the list.
+  constexpr int kPer = CS::kSlots / 4;
+  static_assert(kSeg * kPer <= 32, "one bit per entry of a lane's share");
+  uint32_t take = 0u;
   if (valid) {
 #pragma unroll 1
     for (int g = 0; g < kSeg; ++g) {
       const int col = g * kTile + r;
       const int cnt = min(cs.cnt[col], CS::kSlots);
-      for (int e = lane4; e < cnt; e += 4) n += (P.c * cs.s[e * kCols + col] - tau > 0.f) ? 1 : 0;
+      for (int e = lane4, i = 0; e < cnt; e += 4, ++i)
+        if (P.c * cs.s[e * kCols + col] - tau > 0.f) take |= 1u << (g * kPer + i);
     }
   }
+  const int n = __popc(take);
   // the row's total and this lane's first entry among the row's four lanes
   int incl = n;
   int y = __shfl_up_sync(full, incl, 1);
@@ -307,9 +316,10 @@ __device__ __forceinline__ void record_support(const Problem& P, const TileInfo&
   for (int g = 0; g < kSeg; ++g) {
     const int col = g * kTile + r;
     const int cnt = min(cs.cnt[col], CS::kSlots);
-    for (int e = lane4; e < cnt; e += 4) {
-      const float x = P.c * cs.s[e * kCols + col] - tau;
-      if (x > 0.f) {
+    for (int e = lane4, i = 0; e < cnt; e += 4, ++i) {
+      if ((take >> (g * kPer + i)) & 1u) {
+        // p from z - tau once more (a difference recomputed at or below 0 gives p = 0)
+        const float x = fmaxf(P.c * cs.s[e * kCols + col] - tau, 0.f);
         const int id = cs.kt[e * kCols + col];
         const int j = (id >> 5) * kTile + g * 32 + (id & 31);  // key of the sequence
         list[at++] = make_int2(j, __float_as_int(entmax_p<BK>(x, P.beta)));
