@@ -266,7 +266,8 @@ __device__ __forceinline__ void record_support(const Problem& P, const TileInfo&
   // writes below follow the bits: evaluated twice, z - tau of a key within rounding of tau could
   // come out on different sides (the compiler may fuse the product and the difference in one place
   // and not in the other), and the row would write one entry more or less than it counted, into
-  // the next row's part of the list.
+  // the next row's part of the list.  z - tau is rounded step by step (no fused multiply-add), so
+  // the value the writes recompute is the one tested.
   constexpr int kPer = CS::kSlots / 4;
   static_assert(kSeg * kPer <= 32, "one bit per entry of a lane's share");
   uint32_t take = 0u;
@@ -276,7 +277,8 @@ __device__ __forceinline__ void record_support(const Problem& P, const TileInfo&
       const int col = g * kTile + r;
       const int cnt = min(cs.cnt[col], CS::kSlots);
       for (int e = lane4, i = 0; e < cnt; e += 4, ++i)
-        if (P.c * cs.s[e * kCols + col] - tau > 0.f) take |= 1u << (g * kPer + i);
+        if (__fsub_rn(__fmul_rn(P.c, cs.s[e * kCols + col]), tau) > 0.f)
+          take |= 1u << (g * kPer + i);
     }
   }
   const int n = __popc(take);
@@ -318,8 +320,7 @@ __device__ __forceinline__ void record_support(const Problem& P, const TileInfo&
     const int cnt = min(cs.cnt[col], CS::kSlots);
     for (int e = lane4, i = 0; e < cnt; e += 4, ++i) {
       if ((take >> (g * kPer + i)) & 1u) {
-        // p from z - tau once more (a difference recomputed at or below 0 gives p = 0)
-        const float x = fmaxf(P.c * cs.s[e * kCols + col] - tau, 0.f);
+        const float x = __fsub_rn(__fmul_rn(P.c, cs.s[e * kCols + col]), tau);  // > 0, as tested
         const int id = cs.kt[e * kCols + col];
         const int j = (id >> 5) * kTile + g * 32 + (id & 31);  // key of the sequence
         list[at++] = make_int2(j, __float_as_int(entmax_p<BK>(x, P.beta)));
