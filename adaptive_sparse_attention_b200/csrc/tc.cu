@@ -551,6 +551,10 @@ struct SweepSmem {
   alignas(1024) __nv_bfloat16 k[kTauStages][kTile * D];
   float part[2][3][kSeg][kTile];  // per-sweep partials, double-buffered by sweep parity
   uint32_t words[kMaxWords];
+  int sup_cnt[kSeg][kTile];  // support entries of each (segment, row), counted by the mask round
+  int sup_first[kTile];      // the row's first position in the tile's support list
+  int sup_total[kTile];
+  int sup_over;              // the tile's supports do not fit its list
   uint64_t q_full;
   uint64_t k_full[kTauStages];
   uint64_t k_empty[kTauStages];
@@ -559,7 +563,8 @@ struct SweepSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int kind;  // what the current round over the tile does (row max, search step, mask bits)
+  int kind;  // what the current round over the tile does (row max, search step, mask bits,
+             // support entries)
 };
 
 template <int D, int BK>
@@ -643,11 +648,18 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       sr.init(0.f, 1, P.alpha);
     }
     // One sweep of S over the tile's key range per round; what a round does (row max, one
-    // search step, mask bits) is decided by the score warps at the end of the round before and
-    // published in sm.kind behind a CTA barrier, so that every role runs the same rounds.  The
-    // search stops as soon as every row of the tile has settled (at most n_iter steps).
+    // search step, mask bits, support entries) is decided by the score warps at the end of the
+    // round before and published in sm.kind behind a CTA barrier, so that every role runs the
+    // same rounds.  The search stops as soon as every row of the tile has settled (at most
+    // n_iter steps).  With the supports recorded (P.record_support), the mask round also counts
+    // each row's keys with z > tau, and when the tile's rows fit its list one more round writes
+    // them there (key and p, as the main kernel's record_support does): the tile then leaves the
+    // pending set and its output and gradients come from the lists as well.  Both rounds test
+    // z - tau rounded step by step on the same products, so that they agree key by key.
+    int sup_at = 0, sup_left = 0;  // score threads: this (row, segment)'s next entry and quota
+    bool sup_done = false;
     for (;;) {
-      const int kind = sm.kind;  // 0 row max, 1 search step, 2 mask bits
+      const int kind = sm.kind;  // 0 row max, 1 search step, 2 mask bits, 4 support entries
       if (warp == kTauTmaWarp) {
         if (lane == 0) {
           const int krow0 = static_cast<int>(t.khead + t.seq_start);
@@ -715,15 +727,66 @@ __global__ void __launch_bounds__(kTauThreads, 1)
                 a2 += p2;
               }
             }
-          } else {
-            bool any = false;
+          } else if (kind == 2) {
+            int n = 0;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) any |= (P.c * x[e] > tau);
-            if (any) atomicOr(&sm.words[kt >> 5], 1u << (kt & 31));
+            for (int e = 0; e < 32; ++e) n += (__fsub_rn(__fmul_rn(P.c, x[e]), tau) > 0.f) ? 1 : 0;
+            if (n) atomicOr(&sm.words[kt >> 5], 1u << (kt & 31));
+            a0 += static_cast<float>(n);  // exact: at most 32 per key tile, 2^24 in all
+          } else if (sup_left > 0) {  // kind 4: this (row, segment)'s entries, in key order
+            int2* list = P.sup + t.tile_id * kSupPerTile;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float y = __fsub_rn(__fmul_rn(P.c, x[e]), tau);
+              if (y > 0.f && sup_left > 0) {
+                list[sup_at++] = make_int2(kt * kTile + seg * 32 + e,
+                                           __float_as_int(entmax_p<BK>(y, P.beta)));
+                --sup_left;
+              }
+            }
           }
         }
         int next = 3;  // done
-        if (kind != 2) {
+        if (kind == 2 && P.record_support) {
+          // the rows' places in the tile's list: segments one after another within a row, rows
+          // one after another; the tile keeps its pending flag if they do not fit
+          sm.sup_cnt[seg][r] = valid ? static_cast<int>(a0) : 0;
+          score_warps_sync();
+          if (tid < 32) {  // exclusive prefix over the 128 rows: four rows per lane
+            int a[4], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = 4 * tid + i;
+              const int n = sm.sup_cnt[0][row] + sm.sup_cnt[1][row] + sm.sup_cnt[2][row] +
+                            sm.sup_cnt[3][row];
+              sm.sup_total[row] = n;
+              a[i] = sum;
+              sum += n;
+            }
+            int x = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const int z = __shfl_up_sync(full, x, o);
+              if (tid >= o) x += z;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sm.sup_first[4 * tid + i] = x - sum + a[i];
+            if (tid == 31) sm.sup_over = x > kSupPerTile ? 1 : 0;
+          }
+          score_warps_sync();
+          sup_at = sm.sup_first[r];
+#pragma unroll
+          for (int q2 = 0; q2 < kSeg; ++q2) sup_at += (q2 < seg) ? sm.sup_cnt[q2][r] : 0;
+          sup_left = sm.sup_cnt[seg][r];
+          if (!sm.sup_over) next = 4;
+        } else if (kind == 4) {
+          // the entries a row counted but did not find again (none while the tensor cores
+          // return the same products for the same operands) are left as p = 0 at key 0
+          int2* list = P.sup + t.tile_id * kSupPerTile;
+          for (; sup_left > 0; --sup_left) list[sup_at++] = make_int2(0, 0);
+          sup_done = true;
+        }
+        if (kind != 2 && kind != 4) {
           const int pb = steps_done & 1;
           sm.part[pb][0][seg][r] = a0;
           sm.part[pb][1][seg][r] = a1;
@@ -764,8 +827,13 @@ __global__ void __launch_bounds__(kTauThreads, 1)
       tc_fence_after();
       if (sm.kind == 3) break;
     }
-    if (warp < kTauScoreWarps && seg == 0 && valid)
-      P.tau[t.qhead + t.seq_start + t.row0 + r] = sr.tau;
+    if (warp < kTauScoreWarps && seg == 0 && valid) {
+      const int64_t row = t.qhead + t.seq_start + t.row0 + r;
+      P.tau[row] = sr.tau;
+      if (sup_done) P.sup_idx[row] = sm.sup_first[r] | (sm.sup_total[r] << 16);
+    }
+    // the tile's lists are complete: it leaves the pending set (the output pass runs after)
+    if (tid == 0 && sup_done && !*abort) P.pending[t.tile_id] = 0;
     ++tcount;
     tc_fence_before();
     __syncthreads();
