@@ -800,6 +800,222 @@ def run_backward(args, rank, world, local):
     return 0
 
 
+ROUTE_METRIC = "query rows/s of entmax block routing over chunk summaries"
+ROUTE_CHUNK = 64  # tokens per chunk (the routing entry point's default)
+
+
+def run_routing(args, rank, world, local):
+    """Entmax block routing (DashAttention page, "How it works", stage 2): every query row of
+    the workload's q scored against the summaries of the chunks it may see (the chunks before
+    its own plus its own, estimate_diagonal), then alpha-entmax over those scores, giving the
+    routing priors pi and tau.  The summaries are synthetic: the mean of each 64-key chunk of the
+    workload's keys (the page builds them with learned weights).  A step is one
+    entmax_attn_route_chunks call over resident inputs (the score kernel on the tensor cores,
+    then the row search, which keeps each row's scores in its row of pi between steps).  Its
+    roofline counts the bytes the call must move -- q and the summaries read once, pi (fp32) and
+    tau written once -- against the measured HBM bandwidth."""
+    w = WORKLOADS[args.workload]
+    if w.T > 32768 or w.seqlens:
+        raise SystemExit("--routing takes a fixed-length workload of at most 32K tokens")
+    dev = torch.device("cuda", local)
+    q, k, _, _ = make_inputs(w, seed=rank)
+    nc = -(-w.T // ROUTE_CHUNK)
+    kp = torch.nn.functional.pad(k.float(), (0, 0, 0, nc * ROUTE_CHUNK - w.T))
+    sig = kp.view(w.B, w.Hkv, nc, ROUTE_CHUNK, w.d).mean(dim=3).to(q.dtype).contiguous()
+    qd, sd = q.to(dev), sig.to(dev)
+    alpha = _alpha_f32(w.alpha)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ea.route_chunks(qd, sd, alpha, ROUTE_CHUNK, w.n_iter, w.causal, True, 1.0,
+                               stream=stream)
+
+    for _ in range(args.warmup):
+        pi, tau = step()
+    torch.cuda.synchronize()
+    assert ea.status(stream) == 0
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            pi, tau = step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_one = start.elapsed_time(stop) / args.steps
+    ms_step = max_over_ranks(ms_one, world)
+    assert ea.status(stream) == 0
+    rows = w.B * w.Hq * w.T
+    value = job_rate(rows, ms_one, world)
+    peaks, peak_src = load_peaks()
+    bytes_step = (q.numel() * q.element_size() + sig.numel() * sig.element_size()
+                  + pi.numel() * 4 + tau.numel() * 4)
+    achieved = bytes_step / (ms_one * 1e-3) / 1e9
+    roofline = {"kernel": "entmax_attn_route_chunks (route_scores_kernel + route_chunks_kernel)",
+                "bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]),
+                "unit": "GB/s", "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic": "q and the summaries read once; pi (fp32) and tau written once"}
+
+    # end to end: q and the summaries in from pinned memory, pi and tau out, every step
+    qh, sh = q.pin_memory(), sig.pin_memory()
+    pih = torch.empty(pi.shape, dtype=pi.dtype).pin_memory()
+    tauh = torch.empty(tau.shape, dtype=tau.dtype).pin_memory()
+    e2e_steps = 0 if args.step_only else max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        qd.copy_(qh, non_blocking=True)
+        sd.copy_(sh, non_blocking=True)
+        pi, tau = step()
+        pih.copy_(pi, non_blocking=True)
+        tauh.copy_(tau, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world) if e2e_steps else None
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline and not args.step_only:
+        from oracle import routing as orout  # the timed CPU baseline only
+        import time
+        # a bounded sample: the oracle over the first rows of the first (batch, head), grown
+        # until it takes about a third of the budget (a causal row prefix sees the same chunks)
+        n, spent = 256, 0.0
+        while spent < args.cpu_budget / 3 and n <= w.T:
+            t0 = time.perf_counter()
+            orout.route_chunks(q[:1, :1, :n], sig[:1, :1, :-(-n // ROUTE_CHUNK)], alpha,
+                               ROUTE_CHUNK, w.causal, True, 1.0)
+            spent = time.perf_counter() - t0
+            done = n
+            n *= 2
+        cpu = {"value": done / spent, "unit": "rows/s", "cores": 1, "kind": "oracle",
+               "sample": f"oracle routing of one head's first {done} rows, {spent:.1f} s "
+                         "(numpy fp64 per row, one thread)"}
+
+    line = {
+        "metric": ROUTE_METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == "fp32" else "bf16 scores, f32 search", "data": "synthetic",
+        "config": dict(workload_config(w, world), variant="routing", chunk_size=ROUTE_CHUNK,
+                       chunks=nc, estimate_diagonal=True,
+                       summaries="mean of each chunk's keys"),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": None if e2e_ms is None else {
+            "value": job_rate(rows, e2e_ms, world), "unit": "rows/s", "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": q.numel() * q.element_size() + sig.numel() * sig.element_size(),
+            "d2h_bytes_per_step": pi.numel() * 4 + tau.numel() * 4},
+        "gpu_launches": (2 if w.dtype == "bf16" and w.d in (64, 128) else 1) * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+ROWS_METRIC = "rows/s of row-wise alpha-entmax"
+ROWS_SHAPE = (8192, 16384)  # rows x row length: 8192 score rows of a 16K context
+
+
+def run_rows(args, rank, world, local):
+    """The standalone row-wise alpha-entmax ("Triton Entmax" section of the AdaSplash page) of a
+    bf16 matrix of 8192 rows of 16384 scores (standard normal, so a row's support is a few keys
+    above its max minus 1 / (alpha - 1)), alpha 1.5, 10 search steps.  A step is one
+    entmax_attn_rows call over the resident matrix.  Its roofline counts the bytes the call must
+    move -- x read once, p (bf16) and tau written once -- against the measured HBM bandwidth."""
+    dev = torch.device("cuda", local)
+    n_rows, n = ROWS_SHAPE
+    gen = torch.Generator().manual_seed(2000 + rank)
+    x = torch.randn(n_rows, n, generator=gen).to(torch.bfloat16)
+    xd = x.to(dev)
+    alpha, n_iter = _alpha_f32(1.5), 10
+    stream = torch.cuda.current_stream(dev)
+    p_out = torch.empty_like(xd)
+    t_out = torch.empty(n_rows, dtype=torch.float32, device=dev)
+
+    def step():
+        return ea.entmax_rows(xd, alpha, n_iter, out=p_out, tau=t_out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ea.status(stream) == 0
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_one = start.elapsed_time(stop) / args.steps
+    ms_step = max_over_ranks(ms_one, world)
+    assert ea.status(stream) == 0
+    value = job_rate(n_rows, ms_one, world)
+    peaks, peak_src = load_peaks()
+    bytes_step = 2 * x.numel() * 2 + n_rows * 4
+    achieved = bytes_step / (ms_one * 1e-3) / 1e9
+    roofline = {"kernel": "entmax_attn_rows (entmax_rows_kernel)", "bound": "hbm", "achieved": achieved,
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic": "x read once; p (bf16) and tau written once"}
+
+    xh = x.pin_memory()
+    ph = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    th = torch.empty(n_rows, dtype=torch.float32).pin_memory()
+    e2e_steps = 0 if args.step_only else max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        xd.copy_(xh, non_blocking=True)
+        step()
+        ph.copy_(p_out, non_blocking=True)
+        th.copy_(t_out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world) if e2e_steps else None
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline and not args.step_only:
+        from oracle import oracle as orc  # the timed CPU baseline only
+        import time
+        xs = x.float().numpy()
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_budget / 3 and done < n_rows:
+            orc.entmax_vec(xs[done], alpha)
+            done += 1
+        spent = time.perf_counter() - t0
+        cpu = {"value": done / spent, "unit": "rows/s", "cores": 1, "kind": "oracle",
+               "sample": f"oracle entmax of the first {done} rows, {spent:.1f} s (fp64 C, exact "
+                         "tau by sort, one thread)"}
+
+    line = {
+        "metric": ROWS_METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in/out, f32 search", "data": "synthetic",
+        "config": {"workload": f"rows_{n_rows}x{n}_bf16_a1.5", "rows": n_rows, "row_length": n,
+                   "alpha": 1.5, "n_iter": n_iter, "values": "standard normal",
+                   "parallelism": f"dp{world} (independent per-rank problems)"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": None if e2e_ms is None else {
+            "value": job_rate(n_rows, e2e_ms, world), "unit": "rows/s", "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": x.numel() * 2 + n_rows * 4},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -812,6 +1028,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (entmax_attn_bwd) instead of the forward pass")
+    ap.add_argument("--rows", action="store_true",
+                    help="time the standalone row-wise alpha-entmax (entmax_attn_rows) of an "
+                         "8192 x 16384 bf16 matrix")
+    ap.add_argument("--routing", action="store_true",
+                    help="time entmax block routing over chunk summaries of the workload "
+                         "(entmax_attn_route_chunks; fixed length, at most 32K tokens)")
     ap.add_argument("--also", default="auto",
                     help="other workloads timed in the same run (comma list, 'none'; 'auto': "
                          "the 16K workload beside the 128K one and back)")
@@ -834,6 +1056,10 @@ def main():
     try:
         if args.backward:
             return run_backward(args, rank, world, local)
+        if args.routing:
+            return run_routing(args, rank, world, local)
+        if args.rows:
+            return run_rows(args, rank, world, local)
         return run_native(args, rank, world, local)
     finally:
         if world > 1:

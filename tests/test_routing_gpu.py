@@ -74,3 +74,12 @@ def test_routing_tensor_core_scores(oracle, T, d, C):
     q, sig = _case(1, 4, 2, T, d, C, "bf16", seed=43)
     _check(q, sig, 1.5, 10, C, True, True)
     _check(q, sig, 2.0, 10, C, False, True)
+
+
+@pytest.mark.parametrize("dtype,d", [("fp32", 32), ("bf16", 64)])
+def test_routing_more_chunks_than_registers(oracle, dtype, d):
+    """Rows that see more than 512 chunks (two-token chunks of 1200 tokens: up to 600): the
+    search keeps their scores in the row of pi instead of in registers."""
+    q, sig = _case(1, 2, 1, 1200, d, 2, dtype, seed=44)
+    _check(q, sig, 1.5, 10, 2, True, True)
+    _check(q, sig, 2.0, 10, 2, False, True)
