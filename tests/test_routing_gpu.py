@@ -77,9 +77,9 @@ def test_routing_tensor_core_scores(oracle, T, d, C):
 
 
 @pytest.mark.parametrize("dtype,d", [("fp32", 32), ("bf16", 64)])
-def test_routing_more_chunks_than_registers(oracle, dtype, d):
-    """Rows that see more than 512 chunks (two-token chunks of 1200 tokens: up to 600): the
-    search keeps their scores in the row of pi instead of in registers."""
+def test_routing_many_chunks(oracle, dtype, d):
+    """Rows that see up to 600 chunks (two-token chunks of 1200 tokens): 19 per lane of the
+    row's warp, past the 512 of the other cases."""
     q, sig = _case(1, 2, 1, 1200, d, 2, dtype, seed=44)
     _check(q, sig, 1.5, 10, 2, True, True)
     _check(q, sig, 2.0, 10, 2, False, True)
