@@ -540,6 +540,7 @@ int entmax_attn_route_chunks(const void* q, const void* summaries, float* pi, fl
                              int n_iter, int causal, int estimate_diagonal, float scaling_factor,
                              int dtype, cudaStream_t stream) {
   if (!q || !summaries || !pi || B < 1 || Hq < 1 || Hkv < 1 || T < 1 || Hq % Hkv != 0 ||
+      B > 65535 || Hq > 65535 ||  // the search kernel's grid: (row blocks, heads, batches)
       d < 1 || d > 1024 || chunk_size < 1 || !std::isfinite(alpha) || !(alpha > 1.f) ||
       n_iter < 1 || n_iter > 1000 || (causal != 0 && causal != 1) ||
       (estimate_diagonal != 0 && estimate_diagonal != 1) || !std::isfinite(scaling_factor) ||

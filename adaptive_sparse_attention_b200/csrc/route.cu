@@ -24,14 +24,12 @@ __global__ void __launch_bounds__(32 * kRouteRowsPerCta)
                         float* __restrict__ tau, int B, int Hq, int Hkv, int T_, int d, int nc,
                         int chunk, float alpha, float beta, float zscale, int n_iter, int causal,
                         int diag, int scores_ready) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRouteRowsPerCta + (threadIdx.x >> 5);
+  // grid: (row blocks of one (batch, head), heads, batches) -- no index divisions
+  const int i = blockIdx.x * kRouteRowsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const int64_t rows = static_cast<int64_t>(B) * Hq * T_;
-  if (row >= rows) return;  // whole warps leave together
-  const int i = static_cast<int>(row % T_);
-  const int64_t bh = row / T_;
-  const int h = static_cast<int>(bh % Hq);
-  const int b = static_cast<int>(bh / Hq);
+  if (i >= T_) return;  // whole warps leave together
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t row = (static_cast<int64_t>(b) * Hq + h) * T_ + i;
   const int hk = h / (Hq / Hkv);
   int n = nc;
   if (causal) n = min(nc, i / chunk + (diag ? 1 : 0));
@@ -97,8 +95,8 @@ cudaError_t launch_route_t(const void* q, const void* sig, float* pi, float* tau
                            cudaStream_t s) {
   const float beta = 1.f / (alpha - 1.f);
   const float zscale = (alpha - 1.f) * scaling / sqrtf(static_cast<float>(d));
-  const int64_t rows = static_cast<int64_t>(B) * Hq * T_;
-  const dim3 grid(static_cast<unsigned>((rows + kRouteRowsPerCta - 1) / kRouteRowsPerCta));
+  const dim3 grid(static_cast<unsigned>((T_ + kRouteRowsPerCta - 1) / kRouteRowsPerCta),
+                  static_cast<unsigned>(Hq), static_cast<unsigned>(B));
   const dim3 block(32 * kRouteRowsPerCta);
   const T* qp = static_cast<const T*>(q);
   const T* sp = static_cast<const T*>(sig);

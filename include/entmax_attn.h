@@ -245,8 +245,9 @@ int entmax_attn_rows(const void* x, long long ldx, void* p, long long ldp, float
  * tau fp32 [B, Hq, T] (may be NULL), +inf for a row that sees no chunk (its pi is all zero).
  * q and summaries share the dtype (ENTMAX_ATTN_FP32 or ENTMAX_ATTN_BF16), d <= 1024.  Device
  * pointers, aligned to their element size (pi, tau to 4 bytes); asynchronous on `stream`.
- * Returns ENTMAX_ATTN_OK, ENTMAX_ATTN_EINVAL (a size < 1, Hq not a multiple of Hkv, d > 1024,
- * alpha <= 1 or not finite, n_iter outside [1, 1000], causal or estimate_diagonal not 0/1,
+ * Returns ENTMAX_ATTN_OK, ENTMAX_ATTN_EINVAL (a size < 1, B or Hq above 65535, Hq not a multiple
+ * of Hkv, d > 1024, alpha <= 1 or not finite, n_iter outside [1, 1000], causal or
+ * estimate_diagonal not 0/1,
  * scaling_factor not finite, bad dtype, null q, summaries or pi), ENTMAX_ATTN_EALIGN or
  * ENTMAX_ATTN_ECUDA. */
 int entmax_attn_route_chunks(const void* q, const void* summaries, float* pi, float* tau, int B,
