@@ -306,6 +306,8 @@ def test_route_chunks_argument_checks(native):
     assert call(a1=None) == native.EINVAL       # null summaries
     assert call(a2=None) == native.EINVAL       # null pi
     assert call(a5=3) == native.EINVAL          # Hq not a multiple of Hkv
+    assert call(a4=65536) == native.EINVAL      # B above the search grid's 65535
+    assert call(a5=65536, a6=1) == native.EINVAL  # Hq above it
     assert call(a8=2000) == native.EINVAL       # d > 1024
     assert call(a9=0) == native.EINVAL          # chunk_size < 1
     assert call(a10=1.0) == native.EINVAL       # alpha <= 1
