@@ -82,14 +82,15 @@ extern "C" {
                                              the output pass visits every causally valid key tile.
                                              Give it to both passes. */
 #define ENTMAX_ATTN_FLAG_SUPPORT 16u      /* output from the supports; give it to both passes.
-                                             The tensor-core tau pass records, for every query
-                                             tile whose rows' supports its candidate buffers
-                                             held, each row's support (the keys with p > 0 and
-                                             their p) in the workspace; the output pass computes
-                                             o of those tiles from the lists and runs the tile
-                                             pass over the others only (overflowed candidates,
-                                             supports beyond a tile's list, the CUDA-core path,
-                                             a workspace below entmax_attn_workspace_bytes).
+                                             The tensor-core tau pass records each row's support
+                                             (the keys with p > 0 and their p) in the workspace,
+                                             from its candidate buffers or, for query tiles whose
+                                             buffers overflowed, from an extra sweep of its
+                                             overflow kernel; the output pass computes o of those
+                                             tiles from the lists and runs the tile pass over
+                                             the others only (supports beyond a tile's list, the
+                                             CUDA-core path, a workspace below
+                                             entmax_attn_workspace_bytes).
                                              The path entmax_attn_fwd takes.  Give the
                                              output pass (and entmax_attn_bwd) this flag only
                                              after a tau pass with it on the same workspace. */
