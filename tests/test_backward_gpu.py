@@ -34,6 +34,10 @@ CASES = [
     ("fp32_t129", dict(B=1, Hq=2, Hkv=2, T=129, d=64, alpha=1.5), "fp32", 0),
     ("no_block_mask", dict(B=1, Hq=2, Hkv=1, T=260, d=128, alpha=1.5), "bf16",
      _native.FLAG_NO_BLOCK_MASK),
+    # every query tile through the overflow kernel: on the support path its lists come from that
+    # kernel's extra sweep
+    ("all_fallback_varlen", dict(B=None, Hq=4, Hkv=2, T=None, d=128, alpha=1.5,
+                                 seqlens=[200, 1, 330]), "bf16", _native.FLAG_ALL_FALLBACK),
 ]
 
 
