@@ -2,8 +2,9 @@
 // Activation)"): for every row x of a matrix, p = [(alpha - 1) x - tau]_+^(1/(alpha - 1)) with
 // tau such that sum(p) = 1, found by the same bracketed Halley + bisection search as the
 // attention kernels' tau pass (Search in common.cuh), stopping early once tau has settled.
-// One warp per row; the row is re-read from global memory (L1) at every search step, so any
-// row length works.
+// One warp per row.  The search steps sum over the row's window (the keys that can carry p > 0),
+// gathered once into shared memory; a row whose window does not fit re-reads the row from global
+// memory (L1) at every step, so any row length works.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -13,6 +14,7 @@ namespace ea {
 namespace {
 
 constexpr int kRowsPerCta = 8;
+constexpr int kRowWin = 1024;  // window scores a warp keeps in shared memory
 
 template <typename T, int BK>
 __global__ void __launch_bounds__(32 * kRowsPerCta)
@@ -32,6 +34,57 @@ __global__ void __launch_bounds__(32 * kRowsPerCta)
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(full, m, o));
   Search sr;
   sr.init(am1 * m, n, alpha);
+  // Every key with p > 0 has z = (alpha - 1) x > tau >= m_z - 1, the lower end of the bracket,
+  // which tau never leaves; so the warp gathers the z of that window (widened by a rounding
+  // margin: keys below tau add nothing to any step) into a shared-memory list, and the steps sum
+  // over the list instead of sweeping the whole row each time.  A row with more than kRowWin keys
+  // in the window sweeps the row at every step.
+  __shared__ float win_all[kRowsPerCta][kRowWin];
+  float* win = win_all[threadIdx.x >> 5];
+  {
+    const float floor_z = sr.lo - 1e-3f * (fabsf(sr.lo) + 1.f);
+    const unsigned below = (1u << lane) - 1u;
+    int w = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const float z = j < n ? am1 * load_elem(xr, j) : -INFINITY;
+      const bool in = z > floor_z;
+      const unsigned bal = __ballot_sync(full, in);
+      const int at = w + __popc(bal & below);
+      if (in && at < kRowWin) win[at] = z;
+      w += __popc(bal);
+    }
+    if (w <= kRowWin) {
+      __syncwarp();  // the list is visible to every lane of the warp
+      for (int it = 0; it < n_iter; ++it) {
+        const float t = sr.tau;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+        for (int e = lane; e < w; e += 32) {
+          const float y = win[e] - t;
+          if (y > 0.f) {
+            float a, b, c;
+            entmax_powers<BK>(y, beta, a, b, c);
+            s0 += a;
+            s1 += b;
+            s2 += c;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          s0 += __shfl_xor_sync(full, s0, o);
+          s1 += __shfl_xor_sync(full, s1, o);
+          s2 += __shfl_xor_sync(full, s2, o);
+        }
+        sr.step<BK>(s0, s1, s2, beta);
+        if (sr.settled()) break;
+      }
+      const float t = sr.tau;
+      for (int j = lane; j < n; j += 32)
+        store_elem(pr, j, entmax_p<BK>(am1 * load_elem(xr, j) - t, beta));
+      if (tau && lane == 0) tau[row] = t;
+      return;
+    }
+  }
   for (int it = 0; it < n_iter; ++it) {
     const float t = sr.tau;
     float s0 = 0.f, s1 = 0.f, s2 = 0.f;
