@@ -69,11 +69,12 @@ struct Problem {
   int kv_major;        // tau pass tile order: 1 = all query tiles of one key group before the
                        // next (keys larger than L2), 0 = slot-major (see tau_tile)
   // Output from the supports (ENTMAX_ATTN_FLAG_SUPPORT): with record_support the tensor-core
-  // tau pass records, for every query tile whose rows' supports its candidate buffers hold, each
-  // row's support -- the keys with p > 0 and their p -- and sets pending[tile] to 0 there, 1
-  // where the tile output pass must compute o (overflowed candidates, or more support entries
-  // than a tile's list holds).  With from_support the output pass computes o of the recorded
-  // tiles from their lists and runs the tile pass over the pending ones only.
+  // tau pass records each row's support -- the keys with p > 0 and their p -- from its candidate
+  // buffers, or for a query tile whose buffers overflowed from an extra sweep of the overflow
+  // kernel, and sets pending[tile] to 0 for a recorded tile, 1 where the tile output pass must
+  // compute o (more support entries than a tile's list holds).  With from_support the output
+  // pass computes o of the recorded tiles from their lists and runs the tile pass over the
+  // pending ones only.
   int* pending;        // [tiles] (workspace)
   int2* sup;           // [tiles][kSupPerTile] (key of the sequence, bits of p) (workspace)
   int* sup_idx;        // [q rows]: first entry | (entries << 16) of the row in its tile's list

@@ -542,9 +542,10 @@ __global__ void __launch_bounds__(tau_threads(D, BK), 1)
 // tau_tc_sweep_kernel: the exact tau search for query tiles whose candidate buffers overflowed,
 // with no candidate buffers at all.  S = Q K^T is recomputed on the tensor cores for every sweep
 // over the tile's key range: one sweep for the row max, one per search step (the sums of
-// (z - tau)^beta, ^(beta - 1), ^(beta - 2) over all keys with z > tau), one for the mask bits.
-// Roles as in tau_tc_kernel; the four segment threads of a row combine their partial results
-// through shared memory after every sweep.  CTAs loop over the overflow queue.
+// (z - tau)^beta, ^(beta - 1), ^(beta - 2) over all keys with z > tau), one for the mask bits
+// and, with the supports recorded, one for the support lists.  Roles as in tau_tc_kernel; the
+// four segment threads of a row combine their partial results through shared memory after every
+// sweep.  CTAs loop over the overflow queue.
 
 template <int D>
 struct SweepSmem {
