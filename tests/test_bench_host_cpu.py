@@ -35,6 +35,13 @@ def test_traffic_is_reported_only_for_the_captured_sources(monkeypatch):
     assert bench.ncu_traffic("other", "out_pass") is None
 
 
+def test_capture_hash_ignores_comments_but_not_code():
+    src = "int f(int x) {  // the tile count\n  /* two\n lines */ return x + 1;\n}\n"
+    assert bench._code_only(src) == bench._code_only(src.replace("the tile count", "rows"))
+    assert bench._code_only(src) == bench._code_only(src.replace("\n  ", "\n\n      "))
+    assert bench._code_only(src) != bench._code_only(src.replace("x + 1", "x + 2"))
+
+
 def test_clock_summary_reads_median_clock_and_active_reasons():
     s = bench.ClockSampler(0)
     row = "0, {sm}, 1965, 900.5, 0x0, Not Active, Not Active, Not Active, {cap}"
